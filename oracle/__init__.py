@@ -1,0 +1,36 @@
+"""CPU oracle for MoE token dispatch / combine — TEST INFRASTRUCTURE.
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg may import this package. The product path never does, and this package
+imports nothing from the product.
+"""
+
+from .oracle import (
+    build,
+    library_path,
+    rows_max,
+    num_experts,
+    route_topk,
+    layout,
+    permute,
+    combine,
+    permute_backward,
+    combine_backward,
+    bf16_from_f32,
+    COUNTER_NAMES,
+)
+
+__all__ = [
+    "build",
+    "library_path",
+    "rows_max",
+    "num_experts",
+    "route_topk",
+    "layout",
+    "permute",
+    "combine",
+    "permute_backward",
+    "combine_backward",
+    "bf16_from_f32",
+    "COUNTER_NAMES",
+]
