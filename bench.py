@@ -1,0 +1,529 @@
+#!/usr/bin/env python3
+"""Benchmark: MoE dispatch + combine on B200, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ht] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+router top-k -> dispatch layout -> permute -> (identity experts) -> combine,
+plus combine-backward and permute-backward for workloads that train
+(``ultraep``). Inputs are resident in HBM when the timed region starts and
+rotate over several buffer sets whose total size exceeds the 126 MB L2, so no
+step reads inputs that a previous step left in L2.
+
+N > 1 (torchrun, one process per GPU): each rank processes its own batch
+(data-parallel, independent seeds, no collective on the data path); timing is
+the max over ranks; ``value`` counts the tokens of all ranks.
+
+``--impl reference`` times the plain CPU oracle on this machine's host cores
+on a bounded sample of the same workload (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from synthetic import get_workload, make_inputs  # noqa: E402
+
+METRIC = "dispatch+combine tokens/s and effective HBM GB/s (% of B200 peak), 1 GPU"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------- helpers
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest():
+    """Digest of the kernel sources, to tell whether a stored ncu capture still applies."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "combine_moe_route_tokens_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(kernel: str, workload: str):
+    """dram read+write bytes per launch from a committed ncu summary, if the kernel is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[workload][kernel]
+        if e.get("source_digest") == source_digest():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle",
+        0x2: "applications_clocks_setting",
+        0x4: "sw_power_cap",
+        0x8: "hw_slowdown",
+        0x10: "sync_boost",
+        0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml_unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {
+            "sm_mhz": statistics.median(self.samples) if self.samples else None,
+            "sm_max_mhz": self.max_mhz,
+            "reasons": names,
+            "samples": len(self.samples),
+        }
+
+
+# ------------------------------------------------------------- GPU arm
+
+
+class Step:
+    """One step of the hot path with every C-ABI argument marshalled up front."""
+
+    def __init__(self, w, moe, native, torch, sets, device):
+        self.w = w
+        self.torch = torch
+        self.lib = native.lib()
+        p = moe.Problem(N=w.N, H=w.H, k=w.k, E_log=w.E_log, R=w.R, capacity=w.capacity,
+                        num_replicas=w.num_replicas)
+        self.problem = p
+        self.layout = moe.Layout.allocate(p, device)
+        self.sets = sets
+        N, H, k = w.N, w.H, w.k
+        RM = p.rows_max
+        self.idx = torch.empty((N, k), dtype=torch.int32, device=device)
+        self.probs = torch.empty((N, k), dtype=torch.float32, device=device)
+        self.send = torch.empty((RM, H), dtype=torch.bfloat16, device=device)
+        self.out = torch.empty((N, H), dtype=torch.bfloat16, device=device)
+        if w.backward:
+            self.gy = torch.empty((RM, H), dtype=torch.bfloat16, device=device)
+            self.gp = torch.empty((N, k), dtype=torch.float32, device=device)
+            self.gh = torch.empty((N, H), dtype=torch.bfloat16, device=device)
+        self._p = p.c_struct()
+        self._L = self.layout.c_struct()
+        self.stream = torch.cuda.current_stream(device)
+        self._s = ctypes.c_void_p(self.stream.cuda_stream)
+        vp = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+        P, L = ctypes.byref(self._p), ctypes.byref(self._L)
+        ws = self.layout.workspace
+        self.calls = []
+        for s in sets:
+            c = [
+                ("route", self.lib.moe_route_topk,
+                 (vp(s["logits"]), None, N, w.E_log, k, vp(self.idx), vp(self.probs), self._s)),
+                ("layout", self.lib.moe_dispatch_layout,
+                 (P, vp(self.idx), vp(self.probs), L, vp(ws), ws.numel(), self._s)),
+                ("permute", self.lib.moe_permute, (P, L, vp(s["hidden"]), vp(self.send), self._s)),
+                ("combine", self.lib.moe_combine, (P, L, vp(self.send), vp(self.probs), vp(self.out), self._s)),
+            ]
+            if w.backward:
+                c += [
+                    ("combine_backward", self.lib.moe_combine_backward,
+                     (P, L, vp(s["grad_out"]), vp(self.send), vp(self.probs), vp(self.gy), vp(self.gp), self._s)),
+                    ("permute_backward", self.lib.moe_permute_backward, (P, L, vp(self.gy), vp(self.gh), self._s)),
+                ]
+            self.calls.append(c)
+        self.kernel_names = [name for name, _, _ in self.calls[0]]
+
+    def run(self, i, events=None):
+        for n, (name, fn, args) in enumerate(self.calls[i % len(self.calls)]):
+            if events is not None:
+                events[n][0].record(self.stream)
+            rc = fn(*args)
+            if rc != 0:
+                raise RuntimeError(f"{name} returned {rc}")
+            if events is not None:
+                events[n][1].record(self.stream)
+
+
+def algorithmic_bytes(w, p, kept_rows):
+    """Bytes each kernel must move at least once (see the design notes)."""
+    N, H, k, E = w.N, w.H, w.k, w.E_log
+    RM = p.rows_max
+    row = H * 2
+    return {
+        "route": N * E * 4 + N * k * 8,
+        "layout": N * k * 8 + N * k * (4 + 4 + 4 + 1) + RM * (4 * 4 + 1) + w.R * N * k * 4,
+        "permute": N * row + RM * row + N * k * 4 + RM,
+        "combine": kept_rows * row + N * row + N * k * 8,
+        "combine_backward": N * row + kept_rows * row + RM * row + N * k * 8 + N * k * 4,
+        "permute_backward": kept_rows * row + N * row + N * k * 4,
+    }
+
+
+def run_ours(args, ws, rank, local):
+    import torch
+    import torch.distributed as tdist
+
+    import combine_moe_route_tokens_b200 as moe
+    from combine_moe_route_tokens_b200 import _native
+    from combine_moe_route_tokens_b200.build import build
+
+    if ws > 1:
+        tdist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    build()
+    moe.load_library()
+
+    w = get_workload(args.workload)
+    host = make_inputs(w, grad=w.backward, seed_offset=rank)
+    set_bytes = sum(v.nbytes for v in host.values())
+    nsets = max(2, min(8, math.ceil(2 * L2_BYTES / set_bytes)))
+    # one generated batch; the other sets are token-rotated copies of it (same distribution,
+    # different buffers and different token order)
+    base = {
+        "logits": torch.from_numpy(host["logits"]).to(device),
+        "hidden": torch.from_numpy(host["hidden"].view(np.int16)).to(device).view(torch.bfloat16),
+    }
+    if w.backward:
+        base["grad_out"] = torch.from_numpy(host["grad_out"].view(np.int16)).to(device).view(torch.bfloat16)
+    sets = []
+    for s in range(nsets):
+        shift = (s * 7919) % max(w.N, 1)
+        sets.append({key: torch.roll(v, shifts=shift, dims=0).contiguous() for key, v in base.items()})
+    del base
+    step = Step(w, moe, _native, torch, sets, device)
+
+    def barrier():
+        if ws > 1:
+            tdist.barrier()
+
+    # warm-up
+    for i in range(args.warmup):
+        step.run(i)
+    torch.cuda.synchronize()
+    kept = [int(v) for v in step.layout["counters"].tolist()][1]
+
+    nk = len(step.kernel_names)
+    events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nk)]
+              for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        t0.record(step.stream)
+        for i in range(args.steps):
+            step.run(args.warmup + i, events[i])
+        t1.record(step.stream)
+        torch.cuda.synchronize()
+    barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    per_kernel_ms = {name: [] for name in step.kernel_names}
+    for i in range(args.steps):
+        for n, name in enumerate(step.kernel_names):
+            per_kernel_ms[name].append(events[i][n][0].elapsed_time(events[i][n][1]))
+    status = step.layout.status()
+    if status != 0:
+        raise RuntimeError(f"device status {status:#x} after the timed steps")
+    if ws > 1:
+        t = torch.tensor([elapsed_ms], device=device, dtype=torch.float64)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    # end to end through the public API: pinned host inputs in, result out, every step
+    e2e = None
+    if not args.no_e2e:
+        pin = {key: torch.from_numpy(v if v.dtype != np.uint16 else v.view(np.int16)).pin_memory()
+               for key, v in host.items()}
+        out_host = torch.empty((w.N, w.H), dtype=torch.int16).pin_memory()
+        dst = step.sets[0]
+        views = {key: (dst[key].view(torch.int16) if dst[key].dtype == torch.bfloat16 else dst[key])
+                 for key in pin}
+        h2d = sum(t.numel() * t.element_size() for t in pin.values())
+        d2h = out_host.numel() * out_host.element_size()
+
+        def e2e_step(i):
+            for key in pin:
+                views[key].copy_(pin[key], non_blocking=True)
+            step.run(0)
+            out_host.copy_(step.out.view(torch.int16), non_blocking=True)
+
+        for i in range(max(1, min(args.warmup, 3))):
+            e2e_step(i)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(step.stream)
+        for i in range(args.steps):
+            e2e_step(i)
+        e1.record(step.stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = e0.elapsed_time(e1)
+        if ws > 1:
+            t = torch.tensor([e_ms], device=device, dtype=torch.float64)
+            tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {
+            "value": w.N * args.steps * ws / (e_ms / 1e3),
+            "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h,
+            "ms_per_step": e_ms / args.steps,
+        }
+
+    if ws > 1:
+        tdist.barrier()
+        tdist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    peak, peak_kind = measured_peaks()
+    abytes = algorithmic_bytes(w, step.problem, kept)
+    kernels = {}
+    for name in step.kernel_names:
+        avg_ms = statistics.mean(per_kernel_ms[name])
+        kernels[name] = {
+            "us": round(avg_ms * 1e3, 2),
+            "algorithmic_bytes": abytes[name],
+            "gbs": round(abytes[name] / (avg_ms * 1e-3) / 1e9, 1),
+        }
+    dominant = max(step.kernel_names, key=lambda n: kernels[n]["us"])
+    ach = kernels[dominant]["gbs"]
+    ms_step = elapsed_ms / args.steps
+    path_bytes = sum(abytes[n] for n in step.kernel_names)
+    result = {
+        "metric": METRIC,
+        "value": round(w.N * args.steps * ws / (elapsed_ms / 1e3), 1),
+        "unit": "tokens/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            **w.describe(),
+            "parallelism": f"dp{ws}: independent batch per GPU, no collective on the data path",
+            "step": "+".join(step.kernel_names),
+            "l2": f"inputs rotated over {nsets} buffer sets ({nsets * set_bytes / 2**20:.0f} MiB > 126 MB L2), no flush",
+        },
+        "effective_gbs": round(path_bytes / (ms_step * 1e-3) / 1e9, 1),
+        "effective_hbm_frac": round(path_bytes / (ms_step * 1e-3) / 1e9 / peak, 3),
+        "kernels": kernels,
+        "roofline": {
+            "kernel": dominant,
+            "bound": "hbm",
+            "achieved": ach,
+            "peak": peak,
+            "peak_source": f"{peak_kind} hbm_gbs",
+            "unit": "GB/s",
+            "frac": round(ach / peak, 3),
+            "traffic": stored_traffic(dominant, w.name),
+        },
+        "gpu_launches": args.steps * len(step.kernel_names),
+        "clocks": sampler.summary(),
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline and ws == 1:
+        result["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
+    return result
+
+
+# --------------------------------------------------------- CPU (oracle) arm
+
+
+def oracle_step(oracle, w, d):
+    """The whole path on the CPU oracle for the batch in ``d``."""
+    idx, probs = oracle.route_topk(d["logits"], w.k)
+    L = oracle.layout(idx, probs, E_log=w.E_log, R=w.R, C=w.capacity, num_replicas=w.num_replicas,
+                      local_topk=True)
+    send = oracle.permute(d["hidden"], L["dest_row"], L["rows_max"])
+    out = oracle.combine(send, L["dest_row"], probs)
+    if w.backward:
+        gy, gp = oracle.combine_backward(d["grad_out"], send, L["dest_row"], L["row_token"], L["row_prob"])
+        oracle.permute_backward(gy, L["dest_row"])
+    return out
+
+
+def sample_workload(w, target_s, oracle):
+    """A token sample of the workload sized to take about ``target_s`` per oracle step."""
+    n = max(16, min(w.N, 64))
+    ws = w.scaled(n)
+    d = make_inputs(ws, grad=w.backward)
+    t = time.perf_counter()
+    oracle_step(oracle, ws, d)
+    dt = max(time.perf_counter() - t, 1e-4)
+    n = int(max(16, min(w.N, n * target_s / dt)))
+    ws = w.scaled(n)
+    return ws, make_inputs(ws, grad=w.backward)
+
+
+def cpu_baseline(w, budget_s=10.0):
+    import oracle
+
+    oracle.build()
+    ws, d = sample_workload(w, min(2.0, budget_s / 5), oracle)
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while time.perf_counter() < t_end or not times:
+        t = time.perf_counter()
+        oracle_step(oracle, ws, d)
+        times.append(time.perf_counter() - t)
+    med = statistics.median(times)
+    return {
+        "value": round(ws.N / med, 1),
+        "unit": "tokens/s",
+        "cores": 1,
+        "kind": "oracle",
+        "sample": f"first {ws.N} of {w.N} tokens of '{w.name}' (same H/E/k/R), whole path per run, "
+                  f"median of {len(times)} runs, single-threaded C oracle",
+        "host_cpus": os.cpu_count(),
+    }
+
+
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return None
+    import oracle
+
+    oracle.build()
+    w = get_workload(args.workload)
+    per_step = max(0.02, min(1.0, 120.0 / max(1, args.steps + args.warmup)))
+    wsamp, d = sample_workload(w, per_step, oracle)
+    for _ in range(args.warmup):
+        oracle_step(oracle, wsamp, d)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(oracle, wsamp, d)
+    dt = time.perf_counter() - t
+    value = wsamp.N * args.steps / dt
+    sample = (f"first {wsamp.N} of {w.N} tokens of '{w.name}' per step (same H/E/k/R), "
+              f"single-threaded C oracle")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {**w.describe(), "parallelism": "host cores of rank 0"},
+        "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="ht", help="tiny | ht | qwen3 | capacity | ultraep")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    ws, rank, local = dist_env()
+    if args.gpus != ws and ws > 1:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={ws}")
+    if args.impl == "reference":
+        res = run_reference(args, ws, rank)
+    else:
+        res = run_ours(args, ws, rank, local)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

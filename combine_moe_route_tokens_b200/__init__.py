@@ -1,0 +1,324 @@
+"""MoE token dispatch and combine on one B200 — Python binding of libmoert.so.
+
+Argument marshalling only: every step runs in the CUDA kernels behind the C
+ABI of include/moe_rt.h. PyTorch supplies device memory and the stream. The
+functions keep the C names:
+
+    moe_route_topk        router softmax + top-k
+    moe_dispatch_layout   reroute, histogram, ordinals, capacity, scan, splits, row maps
+    moe_permute           send[dest_row[t, j]] = hidden[t]
+    moe_combine           out[t] = bf16(sum_j p[t, j] * y[dest_row[t, j]]), fp32, ascending j
+    moe_permute_backward  grad_hidden[t] = bf16(sum_j grad_send[dest_row[t, j]])
+    moe_combine_backward  grad_y[row] = bf16(p * grad_out[t]); grad_probs[t, j] = <grad_out[t], y[row]>
+
+All calls are stream-ordered on the current torch stream (or ``stream=``)
+and never synchronise with the host.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Dict, Optional
+
+import ctypes
+
+import torch
+
+from . import _native
+from ._native import (
+    MoeError,
+    MOE_DEV_EXPERT_RANGE,
+    MOE_DEV_ROW_RANGE,
+    MOE_DEV_TIMEOUT,
+    MOE_FLAG_NONE,
+    MOE_FLAG_TEST_BARRIER_TIMEOUT,
+)
+
+COUNTER_NAMES = (
+    "assignments_total",
+    "kept",
+    "dropped",
+    "padded",
+    "split_sum_in",
+    "split_sum_out",
+    "num_rows",
+    "error",
+)
+
+__all__ = [
+    "Problem",
+    "Layout",
+    "MoeError",
+    "moe_route_topk",
+    "moe_dispatch_layout",
+    "moe_permute",
+    "moe_combine",
+    "moe_permute_backward",
+    "moe_combine_backward",
+    "load_library",
+    "COUNTER_NAMES",
+    "MOE_DEV_EXPERT_RANGE",
+    "MOE_DEV_ROW_RANGE",
+    "MOE_DEV_TIMEOUT",
+    "MOE_FLAG_NONE",
+    "MOE_FLAG_TEST_BARRIER_TIMEOUT",
+]
+
+
+def load_library():
+    """Load libmoert.so (raises if it is missing; there is no fallback)."""
+    return _native.lib()
+
+
+@dataclass(frozen=True)
+class Problem:
+    """The problem statement: hidden [N,H] bf16, top-k ids/probs [N,k], E_log experts on R ranks."""
+
+    N: int
+    H: int
+    k: int
+    E_log: int
+    R: int
+    capacity: int = 0
+    num_replicas: int = 0
+    flags: int = MOE_FLAG_NONE
+
+    @property
+    def E(self) -> int:
+        return self.E_log + self.num_replicas
+
+    @property
+    def E_loc(self) -> int:
+        return self.E // self.R
+
+    def c_struct(self) -> _native.MoeProblem:
+        return _native.MoeProblem(
+            N=self.N,
+            H=self.H,
+            k=self.k,
+            E_log=self.E_log,
+            num_replicas=self.num_replicas,
+            R=self.R,
+            capacity=self.capacity,
+            flags=self.flags,
+        )
+
+    @property
+    def rows_max(self) -> int:
+        p = self.c_struct()
+        v = _native.lib().moe_rows_max(ctypes.byref(p))
+        if v < 0:
+            _native.check("moe_rows_max", int(v))
+        return int(v)
+
+    @property
+    def workspace_bytes(self) -> int:
+        p = self.c_struct()
+        n = ctypes.c_size_t(0)
+        _native.check("moe_layout_workspace_bytes",
+                      _native.lib().moe_layout_workspace_bytes(ctypes.byref(p), ctypes.byref(n)))
+        return int(n.value)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+@dataclass
+class Layout:
+    """Device buffers of every dispatch-layout output plus the layout workspace."""
+
+    problem: Problem
+    tensors: Dict[str, torch.Tensor] = field(default_factory=dict)
+    workspace: Optional[torch.Tensor] = None
+
+    @classmethod
+    def allocate(cls, problem: Problem, device=None, local_topk: bool = True) -> "Layout":
+        device = torch.device("cuda") if device is None else torch.device(device)
+        N, k, E, R, E_log = problem.N, problem.k, problem.E, problem.R, problem.E_log
+        NK = N * k
+        RM = problem.rows_max
+        i32, f32, u8 = torch.int32, torch.float32, torch.uint8
+        t = {
+            "phys_idx": torch.empty((N, k), dtype=i32, device=device),
+            "ordinal": torch.empty((N, k), dtype=i32, device=device),
+            "dest_row": torch.empty((N, k), dtype=i32, device=device),
+            "drop_mask": torch.empty((N, k), dtype=u8, device=device),
+            "counts_logical": torch.empty(E_log, dtype=i32, device=device),
+            "placement": torch.empty(E_log, dtype=i32, device=device),
+            "counts_raw": torch.empty(E, dtype=i32, device=device),
+            "tokens_per_expert": torch.empty(E, dtype=i32, device=device),
+            "expert_offsets": torch.empty(E + 1, dtype=i32, device=device),
+            "input_splits": torch.empty(R, dtype=i32, device=device),
+            "output_splits": torch.empty(R, dtype=i32, device=device),
+            "rank_offsets": torch.empty(R + 1, dtype=i32, device=device),
+            "counters": torch.empty(8, dtype=i32, device=device),
+            "num_rows": torch.empty(1, dtype=i32, device=device),
+            "status": torch.zeros(1, dtype=torch.int32, device=device),
+            "row_token": torch.empty(RM, dtype=i32, device=device),
+            "row_slot": torch.empty(RM, dtype=i32, device=device),
+            "row_local_expert": torch.empty(RM, dtype=i32, device=device),
+            "row_prob": torch.empty(RM, dtype=f32, device=device),
+            "pad_mask": torch.empty(RM, dtype=u8, device=device),
+        }
+        if local_topk:
+            t["local_topk"] = torch.empty((R, N, k), dtype=i32, device=device)
+        ws = torch.zeros(problem.workspace_bytes, dtype=u8, device=device)
+        assert NK >= 0
+        return cls(problem=problem, tensors=t, workspace=ws)
+
+    def __getitem__(self, name: str) -> torch.Tensor:
+        return self.tensors[name]
+
+    def c_struct(self) -> _native.MoeLayout:
+        return _native.MoeLayout(**{name: (self.tensors[name].data_ptr() if name in self.tensors else None)
+                                    for name in _native.LAYOUT_FIELDS})
+
+    @property
+    def device(self) -> torch.device:
+        return self.tensors["dest_row"].device
+
+    def status(self) -> int:
+        """Device status bits (MOE_DEV_*) OR-ed by every call on this layout. Synchronises."""
+        return int(self.tensors["status"].item()) & 0xFFFFFFFF
+
+    def clear_status(self) -> None:
+        self.tensors["status"].zero_()
+
+    def reset_workspace(self) -> None:
+        """Zero the layout workspace (needed again only after a MOE_DEV_TIMEOUT)."""
+        self.workspace.zero_()
+
+    def counters(self) -> Dict[str, int]:
+        """dispatch_counters as a dict. Synchronises."""
+        return dict(zip(COUNTER_NAMES, (int(v) for v in self.tensors["counters"].tolist())))
+
+
+def moe_route_topk(logits: torch.Tensor, k: int, token_mask: Optional[torch.Tensor] = None,
+                   topk_idx: Optional[torch.Tensor] = None, topk_probs: Optional[torch.Tensor] = None,
+                   stream=None):
+    """Softmax over E + top-k. Returns (topk_idx [N,k] int32, topk_probs [N,k] fp32)."""
+    _need(logits, "logits", torch.float32)
+    if logits.dim() != 2:
+        raise ValueError("logits must be [N, E]")
+    N, E = logits.shape
+    if token_mask is not None:
+        _need(token_mask, "token_mask", torch.uint8, (N,), logits.device)
+    if topk_idx is None:
+        topk_idx = torch.empty((N, k), dtype=torch.int32, device=logits.device)
+    if topk_probs is None:
+        topk_probs = torch.empty((N, k), dtype=torch.float32, device=logits.device)
+    _need(topk_idx, "topk_idx", torch.int32, (N, k), logits.device)
+    _need(topk_probs, "topk_probs", torch.float32, (N, k), logits.device)
+    rc = _native.lib().moe_route_topk(_ptr(logits), _ptr(token_mask), N, E, k, _ptr(topk_idx), _ptr(topk_probs),
+                                      _stream(stream))
+    _native.check("moe_route_topk", rc)
+    return topk_idx, topk_probs
+
+
+def moe_dispatch_layout(problem: Problem, topk_idx: torch.Tensor, topk_probs: Optional[torch.Tensor],
+                        layout: Optional[Layout] = None, stream=None) -> Layout:
+    """Every dispatch-layout output in one launch; returns the (reusable) Layout."""
+    _need(topk_idx, "topk_idx", torch.int32, (problem.N, problem.k))
+    if topk_probs is not None:
+        _need(topk_probs, "topk_probs", torch.float32, (problem.N, problem.k), topk_idx.device)
+    if layout is None:
+        layout = Layout.allocate(problem, topk_idx.device)
+    elif layout.problem != problem:
+        raise ValueError("layout was allocated for a different problem")
+    p = problem.c_struct()
+    L = layout.c_struct()
+    rc = _native.lib().moe_dispatch_layout(ctypes.byref(p), _ptr(topk_idx), _ptr(topk_probs), ctypes.byref(L),
+                                           _ptr(layout.workspace), layout.workspace.numel(), _stream(stream))
+    _native.check("moe_dispatch_layout", rc)
+    return layout
+
+
+def moe_permute(problem: Problem, layout: Layout, hidden: torch.Tensor, send: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    """send[dest_row[t,j]] = hidden[t]; pad rows zero. Returns send [rows_max, H] bf16."""
+    _need(hidden, "hidden", torch.bfloat16, (problem.N, problem.H), layout.device)
+    if send is None:
+        send = torch.empty((problem.rows_max, problem.H), dtype=torch.bfloat16, device=hidden.device)
+    _need(send, "send", torch.bfloat16, (problem.rows_max, problem.H), layout.device)
+    p = problem.c_struct()
+    L = layout.c_struct()
+    _native.check("moe_permute",
+                  _native.lib().moe_permute(ctypes.byref(p), ctypes.byref(L), _ptr(hidden), _ptr(send),
+                                            _stream(stream)))
+    return send
+
+
+def moe_combine(problem: Problem, layout: Layout, expert_out: torch.Tensor, topk_probs: Optional[torch.Tensor],
+                out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out[t] = bf16(fp32 fma chain over ascending kept j of p[t,j] * expert_out[dest_row[t,j]])."""
+    _need(expert_out, "expert_out", torch.bfloat16, (problem.rows_max, problem.H), layout.device)
+    if topk_probs is not None:
+        _need(topk_probs, "topk_probs", torch.float32, (problem.N, problem.k), layout.device)
+    if out is None:
+        out = torch.empty((problem.N, problem.H), dtype=torch.bfloat16, device=expert_out.device)
+    _need(out, "out", torch.bfloat16, (problem.N, problem.H), layout.device)
+    p = problem.c_struct()
+    L = layout.c_struct()
+    _native.check("moe_combine",
+                  _native.lib().moe_combine(ctypes.byref(p), ctypes.byref(L), _ptr(expert_out), _ptr(topk_probs),
+                                            _ptr(out), _stream(stream)))
+    return out
+
+
+def moe_permute_backward(problem: Problem, layout: Layout, grad_send: torch.Tensor,
+                         grad_hidden: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """grad_hidden[t] = bf16(fp32 sum over ascending kept j of grad_send[dest_row[t,j]])."""
+    _need(grad_send, "grad_send", torch.bfloat16, (problem.rows_max, problem.H), layout.device)
+    if grad_hidden is None:
+        grad_hidden = torch.empty((problem.N, problem.H), dtype=torch.bfloat16, device=grad_send.device)
+    _need(grad_hidden, "grad_hidden", torch.bfloat16, (problem.N, problem.H), layout.device)
+    p = problem.c_struct()
+    L = layout.c_struct()
+    _native.check("moe_permute_backward",
+                  _native.lib().moe_permute_backward(ctypes.byref(p), ctypes.byref(L), _ptr(grad_send),
+                                                     _ptr(grad_hidden), _stream(stream)))
+    return grad_hidden
+
+
+def moe_combine_backward(problem: Problem, layout: Layout, grad_out: torch.Tensor, expert_out: torch.Tensor,
+                         topk_probs: torch.Tensor, grad_expert_out: Optional[torch.Tensor] = None,
+                         grad_probs: Optional[torch.Tensor] = None, stream=None):
+    """Returns (grad_expert_out [rows_max,H] bf16, grad_probs [N,k] fp32)."""
+    _need(grad_out, "grad_out", torch.bfloat16, (problem.N, problem.H), layout.device)
+    _need(expert_out, "expert_out", torch.bfloat16, (problem.rows_max, problem.H), layout.device)
+    _need(topk_probs, "topk_probs", torch.float32, (problem.N, problem.k), layout.device)
+    if grad_expert_out is None:
+        grad_expert_out = torch.empty((problem.rows_max, problem.H), dtype=torch.bfloat16, device=grad_out.device)
+    if grad_probs is None:
+        grad_probs = torch.empty((problem.N, problem.k), dtype=torch.float32, device=grad_out.device)
+    _need(grad_expert_out, "grad_expert_out", torch.bfloat16, (problem.rows_max, problem.H), layout.device)
+    _need(grad_probs, "grad_probs", torch.float32, (problem.N, problem.k), layout.device)
+    p = problem.c_struct()
+    L = layout.c_struct()
+    _native.check("moe_combine_backward",
+                  _native.lib().moe_combine_backward(ctypes.byref(p), ctypes.byref(L), _ptr(grad_out),
+                                                     _ptr(expert_out), _ptr(topk_probs), _ptr(grad_expert_out),
+                                                     _ptr(grad_probs), _stream(stream)))
+    return grad_expert_out, grad_probs

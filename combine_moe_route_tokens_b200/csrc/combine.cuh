@@ -1,0 +1,282 @@
+// combine.cuh — the combine gather-reduce and both backward passes.
+//
+// DeepSpeed EP page, restore_combined: weighted expert outputs are added back
+// per token one top-k slot at a time in ascending slot order, so the
+// accumulation order is fixed. Megatron MoE page, combine. Megatron MORI
+// page: backward passes use receiver-side indices and probs.
+//
+// Combine: one thread per 16-byte column chunk (8 bf16) of one token. All k
+// source rows of the chunk are loaded up front (k independent 16-byte
+// streaming loads in flight per thread), then accumulated in fp32 with one
+// fmaf per kept slot in ascending j from +0, and rounded once to bf16
+// (cvt.rn.bf16x2). No atomics: every output element has one writer. A warp
+// covers 512 contiguous bytes of each source row.
+//
+// Combine backward: one CTA per token walks the row in 16-byte chunks,
+// writes grad_y[dest_row[t,j]] = bf16(fp32(p[t,j] * g)) and accumulates the
+// per-slot dot products <g, y[dest_row[t,j]]> in fp32, reduced across the CTA
+// in a fixed order (deterministic). Extra CTAs zero the pad rows of grad_y.
+#pragma once
+
+#include <cstdint>
+
+#include "moe_rt.h"
+#include "permute.cuh"
+#include "ptx.cuh"
+
+namespace moert {
+
+constexpr int COMBINE_THREADS = 128;
+constexpr int COMBINE_BWD_THREADS = 128;
+constexpr int COMBINE_MAX_K = 32;
+
+struct CombineArgs {
+    const uint4 *y;          // [rows_max, V]
+    const int32_t *dest_row; // [N, k]
+    const float *probs;      // [N, k] or null (unit weights)
+    uint4 *out;              // [N, V]
+    uint32_t *status;
+    int64_t N;
+    int64_t rows_max;
+    int32_t k;
+    int32_t V;       // 16-byte chunks per row (H / 8)
+    int32_t nchunks; // CTAs per token
+};
+
+__device__ __forceinline__ void fma8(float (&acc)[8], float p, const uint4 &y)
+{
+    acc[0] = __fmaf_rn(p, bf16_lo(y.x), acc[0]);
+    acc[1] = __fmaf_rn(p, bf16_hi(y.x), acc[1]);
+    acc[2] = __fmaf_rn(p, bf16_lo(y.y), acc[2]);
+    acc[3] = __fmaf_rn(p, bf16_hi(y.y), acc[3]);
+    acc[4] = __fmaf_rn(p, bf16_lo(y.z), acc[4]);
+    acc[5] = __fmaf_rn(p, bf16_hi(y.z), acc[5]);
+    acc[6] = __fmaf_rn(p, bf16_lo(y.w), acc[6]);
+    acc[7] = __fmaf_rn(p, bf16_hi(y.w), acc[7]);
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&acc)[8])
+{
+    return make_uint4(pack_bf16x2_rn(acc[0], acc[1]), pack_bf16x2_rn(acc[2], acc[3]),
+                      pack_bf16x2_rn(acc[4], acc[5]), pack_bf16x2_rn(acc[6], acc[7]));
+}
+
+// Slot metadata of token t: lane j < k holds dest_row[t,j] and its weight.
+__device__ __forceinline__ void load_slot_meta(const int32_t *dest_row, const float *probs, int64_t t, int k,
+                                               int64_t rows_max, uint32_t *status, int32_t &d, float &p)
+{
+    const int lane = threadIdx.x & 31;
+    d = -1;
+    p = 0.0f;
+    if (lane < k) {
+        d = __ldg(dest_row + t * k + lane);
+        p = probs != nullptr ? __ldg(probs + t * k + lane) : 1.0f;
+        if (d < -1 || d >= rows_max) {
+            atomicOr(status, MOE_DEV_ROW_RANGE);
+            d = -1;
+        }
+    }
+}
+
+template <int K> // K > 0: top-k fixed at compile time; K == 0: runtime k <= 32
+__global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(CombineArgs a)
+{
+    const int64_t t = blockIdx.x / a.nchunks;
+    const int c = static_cast<int>(blockIdx.x - t * a.nchunks);
+    const int v = c * blockDim.x + threadIdx.x;
+    const int k = K > 0 ? K : a.k;
+
+    int32_t d;
+    float p;
+    load_slot_meta(a.dest_row, a.probs, t, k, a.rows_max, a.status, d, p);
+
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+        acc[e] = 0.0f;
+
+    if constexpr (K > 0) {
+        int32_t dj[K];
+        float pj[K];
+        uint4 yj[K];
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+            dj[j] = __shfl_sync(0xffffffffu, d, j);
+            pj[j] = __shfl_sync(0xffffffffu, p, j);
+        }
+        if (v >= a.V)
+            return;
+#pragma unroll
+        for (int j = 0; j < K; ++j)
+            if (dj[j] >= 0)
+                yj[j] = ld_stream_u4(a.y + static_cast<int64_t>(dj[j]) * a.V + v);
+#pragma unroll
+        for (int j = 0; j < K; ++j)
+            if (dj[j] >= 0)
+                fma8(acc, pj[j], yj[j]);
+    } else {
+        const bool active = v < a.V;
+        for (int j0 = 0; j0 < k; j0 += 4) {
+            int32_t dj[4];
+            float pj[4];
+            uint4 yj[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                dj[u] = __shfl_sync(0xffffffffu, d, (j0 + u) & 31);
+                pj[u] = __shfl_sync(0xffffffffu, p, (j0 + u) & 31);
+                if (j0 + u >= k || !active)
+                    dj[u] = -1;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (dj[u] >= 0)
+                    yj[u] = ld_stream_u4(a.y + static_cast<int64_t>(dj[u]) * a.V + v);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (dj[u] >= 0)
+                    fma8(acc, pj[u], yj[u]);
+        }
+        if (!active)
+            return;
+    }
+    st_u4(a.out + t * a.V + v, pack8(acc));
+}
+
+struct CombineBwdArgs {
+    const uint4 *grad_out;   // [N, V]
+    const uint4 *y;          // [rows_max, V]
+    const int32_t *dest_row; // [N, k]
+    const float *probs;      // [N, k]
+    const uint8_t *pad_mask; // [rows_max]
+    uint4 *grad_y;           // [rows_max, V]
+    float *grad_probs;       // [N, k]
+    uint32_t *status;
+    int64_t N;
+    int64_t rows_max;
+    int32_t k;
+    int32_t V;
+    int32_t zero_blocks; // trailing CTAs that zero pad rows of grad_y
+};
+
+__device__ __forceinline__ float dot8(float s, const uint4 &g, const uint4 &y)
+{
+    s = __fmaf_rn(bf16_lo(g.x), bf16_lo(y.x), s);
+    s = __fmaf_rn(bf16_hi(g.x), bf16_hi(y.x), s);
+    s = __fmaf_rn(bf16_lo(g.y), bf16_lo(y.y), s);
+    s = __fmaf_rn(bf16_hi(g.y), bf16_hi(y.y), s);
+    s = __fmaf_rn(bf16_lo(g.z), bf16_lo(y.z), s);
+    s = __fmaf_rn(bf16_hi(g.z), bf16_hi(y.z), s);
+    s = __fmaf_rn(bf16_lo(g.w), bf16_lo(y.w), s);
+    s = __fmaf_rn(bf16_hi(g.w), bf16_hi(y.w), s);
+    return s;
+}
+
+__device__ __forceinline__ uint4 scale8(float p, const uint4 &g)
+{
+    return make_uint4(pack_bf16x2_rn(__fmul_rn(p, bf16_lo(g.x)), __fmul_rn(p, bf16_hi(g.x))),
+                      pack_bf16x2_rn(__fmul_rn(p, bf16_lo(g.y)), __fmul_rn(p, bf16_hi(g.y))),
+                      pack_bf16x2_rn(__fmul_rn(p, bf16_lo(g.z)), __fmul_rn(p, bf16_hi(g.z))),
+                      pack_bf16x2_rn(__fmul_rn(p, bf16_lo(g.w)), __fmul_rn(p, bf16_hi(g.w))));
+}
+
+// Deterministic CTA-wide sum: warp butterfly, then warps in index order.
+__device__ __forceinline__ float cta_sum_fixed(float v, float *s_red)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncthreads();
+    if (lane == 0)
+        s_red[warp] = v;
+    __syncthreads();
+    float total = 0.0f;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w)
+        total += s_red[w];
+    return total;
+}
+
+template <int K>
+__global__ void __launch_bounds__(COMBINE_BWD_THREADS) combine_backward_kernel(CombineBwdArgs a)
+{
+    __shared__ float s_red[COMBINE_BWD_THREADS / 32];
+    __shared__ float s_part[COMBINE_BWD_THREADS / 32][K > 0 ? K : 1];
+    if (blockIdx.x >= a.N) {
+        const int64_t workers = static_cast<int64_t>(a.zero_blocks) * (COMBINE_BWD_THREADS / 32);
+        const int64_t worker = (blockIdx.x - a.N) * (COMBINE_BWD_THREADS / 32) + (threadIdx.x >> 5);
+        zero_pad_rows_warp(reinterpret_cast<uint8_t *>(a.grad_y), a.pad_mask, a.rows_max,
+                           static_cast<uint32_t>(a.V) * 16u, worker, workers);
+        return;
+    }
+    const int64_t t = blockIdx.x;
+    const int k = K > 0 ? K : a.k;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int32_t d;
+    float p;
+    load_slot_meta(a.dest_row, a.probs, t, k, a.rows_max, a.status, d, p);
+    const uint4 *g_row = a.grad_out + t * a.V;
+
+    if constexpr (K > 0) {
+        int32_t dj[K];
+        float pj[K];
+        float part[K];
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+            dj[j] = __shfl_sync(0xffffffffu, d, j);
+            pj[j] = __shfl_sync(0xffffffffu, p, j);
+            part[j] = 0.0f;
+        }
+        for (int v = threadIdx.x; v < a.V; v += COMBINE_BWD_THREADS) {
+            const uint4 g = ld_stream_u4(g_row + v);
+            uint4 yj[K];
+#pragma unroll
+            for (int j = 0; j < K; ++j)
+                if (dj[j] >= 0)
+                    yj[j] = ld_stream_u4(a.y + static_cast<int64_t>(dj[j]) * a.V + v);
+#pragma unroll
+            for (int j = 0; j < K; ++j)
+                if (dj[j] >= 0) {
+                    st_u4(a.grad_y + static_cast<int64_t>(dj[j]) * a.V + v, scale8(pj[j], g));
+                    part[j] = dot8(part[j], g, yj[j]);
+                }
+        }
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                part[j] += __shfl_xor_sync(0xffffffffu, part[j], o);
+        }
+        if (lane == 0) {
+#pragma unroll
+            for (int j = 0; j < K; ++j)
+                s_part[warp][j] = part[j];
+        }
+        __syncthreads();
+        if (threadIdx.x < K) { // lane j of warp 0 holds slot j's own dest_row in d
+            const int j = threadIdx.x;
+            float total = 0.0f;
+            for (int w = 0; w < COMBINE_BWD_THREADS / 32; ++w)
+                total += s_part[w][j];
+            a.grad_probs[t * K + j] = d >= 0 ? total : 0.0f;
+        }
+    } else {
+        for (int j = 0; j < k; ++j) {
+            const int32_t dj = __shfl_sync(0xffffffffu, d, j);
+            const float pj = __shfl_sync(0xffffffffu, p, j);
+            float part = 0.0f;
+            if (dj >= 0) {
+                for (int v = threadIdx.x; v < a.V; v += COMBINE_BWD_THREADS) {
+                    const uint4 g = __ldg(g_row + v);
+                    const uint4 y = ld_stream_u4(a.y + static_cast<int64_t>(dj) * a.V + v);
+                    st_u4(a.grad_y + static_cast<int64_t>(dj) * a.V + v, scale8(pj, g));
+                    part = dot8(part, g, y);
+                }
+            }
+            const float total = cta_sum_fixed(part, s_red);
+            if (threadIdx.x == 0)
+                a.grad_probs[t * k + j] = dj >= 0 ? total : 0.0f;
+        }
+    }
+}
+
+} // namespace moert

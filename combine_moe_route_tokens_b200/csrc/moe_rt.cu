@@ -1,0 +1,479 @@
+// moe_rt.cu — host side of libmoert.so: argument checks, launch
+// configuration and the extern "C" entry points declared in moe_rt.h.
+//
+// Every entry point validates on the host, then enqueues its kernel(s) on the
+// caller's stream and returns; nothing here synchronises with the device or
+// reads device memory. The only host state is a per-device cache of
+// attributes (SM count, shared-memory limit) and kernel attribute setup.
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "moe_rt.h"
+
+#include "ptx.cuh"
+#include "route.cuh"
+#include "layout.cuh"
+#include "permute.cuh"
+#include "combine.cuh"
+
+namespace {
+
+using namespace moert;
+
+constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;     // 1 s: every device-side wait gives up after this
+constexpr uint64_t TEST_WAIT_LIMIT_NS = 10000000ull;  // 10 ms for MOE_FLAG_TEST_BARRIER_TIMEOUT
+constexpr size_t WS_BARRIER_BYTES = 256;
+
+struct DeviceInfo {
+    int sms = 0;
+    int smem_optin = 0;
+    bool ready = false;
+};
+
+constexpr int MAX_DEVICES = 64;
+DeviceInfo g_devices[MAX_DEVICES];
+std::mutex g_mutex;
+
+int device_info(DeviceInfo *out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES)
+        return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo &d = g_devices[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        cudaError_t e = cudaFuncSetAttribute(layout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             d.smem_optin - 16 * 1024);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     d.smem_optin - 1024);
+        if (e != cudaSuccess)
+            return MOE_ERR_CUDA;
+        d.ready = true;
+    }
+    *out = d;
+    return MOE_OK;
+}
+
+int launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Derived sizes of a validated problem.
+struct Dims {
+    int64_t NK = 0;
+    int64_t rows_max = 0;
+    int32_t E = 0, E_loc = 0, M = 0, S = 0;
+};
+
+int check_problem(const moe_problem_t *p, Dims *d)
+{
+    if (p == nullptr)
+        return MOE_ERR_INVALID;
+    if (p->N < 0 || p->H <= 0 || (p->H & 7) != 0 || p->k < 1 || p->E_log < 1 || p->R < 1 || p->capacity < 0 ||
+        p->num_replicas < 0)
+        return MOE_ERR_INVALID;
+    if (p->E_log % p->R != 0 || p->num_replicas % p->R != 0 || p->num_replicas > p->E_log)
+        return MOE_ERR_INVALID;
+    if ((p->flags & ~MOE_FLAG_TEST_BARRIER_TIMEOUT) != 0)
+        return MOE_ERR_INVALID;
+    const int64_t NK = p->N * static_cast<int64_t>(p->k);
+    if (p->N > (int64_t(1) << 40) || NK > INT32_MAX)
+        return MOE_ERR_INVALID;
+    const int64_t E = static_cast<int64_t>(p->E_log) + p->num_replicas;
+    const int64_t rows_max = p->capacity > 0 ? E * p->capacity : NK;
+    if (rows_max > INT32_MAX)
+        return MOE_ERR_INVALID;
+    if (p->k > COMBINE_MAX_K || p->E_log > LAYOUT_MAX_E_LOG)
+        return MOE_ERR_UNSUPPORTED;
+    if (p->num_replicas > 0 && p->R > LAYOUT_MAX_PLACEMENT_RANKS)
+        return MOE_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(p->H) * 2 > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    d->NK = NK;
+    d->rows_max = rows_max;
+    d->E = static_cast<int32_t>(E);
+    d->E_loc = static_cast<int32_t>(E / p->R);
+    d->M = p->E_log / p->R;
+    d->S = p->num_replicas / p->R;
+    return MOE_OK;
+}
+
+// Per-assignment outputs may be NULL only when there are no assignments, per-row
+// outputs only when there are no rows.
+int check_layout(const moe_layout_t *l, const Dims &d, bool need_rows)
+{
+    if (l == nullptr || l->status == nullptr)
+        return MOE_ERR_INVALID;
+    if (d.NK > 0 && l->dest_row == nullptr)
+        return MOE_ERR_INVALID;
+    if (need_rows && d.rows_max > 0 && l->pad_mask == nullptr)
+        return MOE_ERR_INVALID;
+    return MOE_OK;
+}
+
+struct LayoutGrid {
+    int32_t G;
+    int32_t sub;
+};
+
+LayoutGrid layout_grid(int64_t NK)
+{
+    int64_t G = (NK + LAYOUT_ITEMS_PER_BLOCK - 1) / LAYOUT_ITEMS_PER_BLOCK;
+    G = G < 1 ? 1 : (G > LAYOUT_MAX_BLOCKS ? LAYOUT_MAX_BLOCKS : G);
+    int64_t sub = (NK + G * LAYOUT_WARPS - 1) / (G * LAYOUT_WARPS);
+    sub = ((sub + 31) / 32) * 32;
+    if (sub < 32)
+        sub = 32;
+    G = (NK + LAYOUT_WARPS * sub - 1) / (LAYOUT_WARPS * sub);
+    if (G < 1)
+        G = 1;
+    return {static_cast<int32_t>(G), static_cast<int32_t>(sub)};
+}
+
+size_t layout_workspace_bytes(int32_t E_log)
+{
+    return WS_BARRIER_BYTES + static_cast<size_t>(LAYOUT_MAX_BLOCKS) * (static_cast<size_t>(E_log) + 1) * 4;
+}
+
+} // namespace
+
+extern "C" {
+
+int moe_abi_version(void) { return MOE_RT_ABI_VERSION; }
+
+const char *moe_status_string(int code)
+{
+    switch (code) {
+    case MOE_OK:
+        return "ok";
+    case MOE_ERR_INVALID:
+        return "invalid argument (size, NULL pointer, alignment or inconsistent problem)";
+    case MOE_ERR_UNSUPPORTED:
+        return "valid problem beyond the kernels' limits";
+    case MOE_ERR_CUDA:
+        return "CUDA runtime call or kernel launch failed";
+    case static_cast<int>(MOE_DEV_EXPERT_RANGE):
+        return "device: expert id outside [-1, E_log) skipped";
+    case static_cast<int>(MOE_DEV_TIMEOUT):
+        return "device: bounded wait ran out";
+    case static_cast<int>(MOE_DEV_ROW_RANGE):
+        return "device: destination row outside [-1, rows_max) skipped";
+    default:
+        return "unknown status";
+    }
+}
+
+int64_t moe_rows_max(const moe_problem_t *problem)
+{
+    Dims d;
+    const int rc = check_problem(problem, &d);
+    return rc != MOE_OK ? rc : d.rows_max;
+}
+
+int moe_layout_workspace_bytes(const moe_problem_t *problem, size_t *bytes)
+{
+    Dims d;
+    const int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    if (bytes == nullptr)
+        return MOE_ERR_INVALID;
+    *bytes = layout_workspace_bytes(problem->E_log);
+    return MOE_OK;
+}
+
+int moe_route_topk(const float *logits, const uint8_t *token_mask, int64_t N, int32_t E, int32_t k,
+                   int32_t *topk_idx, float *topk_probs, void *stream)
+{
+    if (N < 0 || E < 1 || k < 1 || k > E)
+        return MOE_ERR_INVALID;
+    if (k > 32 || E > 1024)
+        return MOE_ERR_UNSUPPORTED;
+    if (N == 0)
+        return MOE_OK;
+    if (logits == nullptr || topk_idx == nullptr || topk_probs == nullptr)
+        return MOE_ERR_INVALID;
+    if (N > (int64_t(1) << 40))
+        return MOE_ERR_INVALID;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t blocks64 = (N + ROUTE_WARPS_PER_BLOCK - 1) / ROUTE_WARPS_PER_BLOCK;
+    if (blocks64 > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    const dim3 grid(static_cast<unsigned>(blocks64)), block(ROUTE_WARPS_PER_BLOCK * 32);
+    const int vpl = (E + 31) / 32;
+    if (vpl <= 1)
+        route_topk_kernel<1><<<grid, block, 0, s>>>(logits, token_mask, N, E, k, topk_idx, topk_probs);
+    else if (vpl <= 2)
+        route_topk_kernel<2><<<grid, block, 0, s>>>(logits, token_mask, N, E, k, topk_idx, topk_probs);
+    else if (vpl <= 4)
+        route_topk_kernel<4><<<grid, block, 0, s>>>(logits, token_mask, N, E, k, topk_idx, topk_probs);
+    else if (vpl <= 8)
+        route_topk_kernel<8><<<grid, block, 0, s>>>(logits, token_mask, N, E, k, topk_idx, topk_probs);
+    else if (vpl <= 16)
+        route_topk_kernel<16><<<grid, block, 0, s>>>(logits, token_mask, N, E, k, topk_idx, topk_probs);
+    else
+        route_topk_kernel<32><<<grid, block, 0, s>>>(logits, token_mask, N, E, k, topk_idx, topk_probs);
+    return launch_status();
+}
+
+int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, const float *topk_probs,
+                        const moe_layout_t *layout, void *workspace, size_t workspace_bytes, void *stream)
+{
+    Dims d;
+    int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    const moe_layout_t *l = layout;
+    if (l == nullptr || l->status == nullptr || l->counts_logical == nullptr || l->placement == nullptr ||
+        l->counts_raw == nullptr || l->tokens_per_expert == nullptr || l->expert_offsets == nullptr ||
+        l->input_splits == nullptr || l->output_splits == nullptr || l->rank_offsets == nullptr ||
+        l->counters == nullptr || l->num_rows == nullptr)
+        return MOE_ERR_INVALID;
+    if (d.NK > 0 && (topk_idx == nullptr || l->phys_idx == nullptr || l->ordinal == nullptr ||
+                     l->dest_row == nullptr || l->drop_mask == nullptr))
+        return MOE_ERR_INVALID;
+    if (d.rows_max > 0 && (l->row_token == nullptr || l->row_slot == nullptr || l->row_local_expert == nullptr ||
+                           l->row_prob == nullptr || l->pad_mask == nullptr))
+        return MOE_ERR_INVALID;
+    if (workspace == nullptr || workspace_bytes < layout_workspace_bytes(problem->E_log) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return MOE_ERR_INVALID;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev)) != MOE_OK)
+        return rc;
+    const LayoutGrid lg = layout_grid(d.NK);
+    if (lg.G > dev.sms)
+        return MOE_ERR_UNSUPPORTED;
+    const size_t smem = layout_smem_words(problem->E_log, d.E) * 4;
+    if (smem > static_cast<size_t>(dev.smem_optin - 16 * 1024))
+        return MOE_ERR_UNSUPPORTED;
+
+    LayoutArgs a;
+    a.topk_idx = topk_idx;
+    a.topk_probs = topk_probs;
+    a.NK = d.NK;
+    a.rows_max = d.rows_max;
+    a.k = problem->k;
+    a.E_log = problem->E_log;
+    a.E = d.E;
+    a.R = problem->R;
+    a.E_loc = d.E_loc;
+    a.M = d.M;
+    a.S = d.S;
+    a.num_replicas = problem->num_replicas;
+    a.C = problem->capacity;
+    a.sub = lg.sub;
+    a.G = lg.G;
+    a.ws_barrier = static_cast<uint32_t *>(workspace);
+    a.ws_counts = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + WS_BARRIER_BYTES);
+    const bool test_timeout = (problem->flags & MOE_FLAG_TEST_BARRIER_TIMEOUT) != 0;
+    a.barrier_limit_ns = test_timeout ? TEST_WAIT_LIMIT_NS : WAIT_LIMIT_NS;
+    a.barrier_extra = test_timeout ? 1u : 0u;
+    a.out = *l;
+
+    void *args[] = {&a};
+    const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(layout_kernel), dim3(lg.G),
+                                                      dim3(LAYOUT_THREADS), args, smem,
+                                                      static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
+
+int moe_permute(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *hidden, uint16_t *send,
+                void *stream)
+{
+    Dims d;
+    int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    if ((rc = check_layout(layout, d, true)) != MOE_OK)
+        return rc;
+    if ((problem->N > 0 && (hidden == nullptr || !aligned16(hidden))) ||
+        (d.rows_max > 0 && (send == nullptr || !aligned16(send))))
+        return MOE_ERR_INVALID;
+    if (problem->N == 0 && d.rows_max == 0)
+        return MOE_OK;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev)) != MOE_OK)
+        return rc;
+
+    PermuteArgs a;
+    a.hidden = reinterpret_cast<const uint8_t *>(hidden);
+    a.send = reinterpret_cast<uint8_t *>(send);
+    a.dest_row = layout->dest_row;
+    a.pad_mask = layout->pad_mask;
+    a.status = layout->status;
+    a.N = problem->N;
+    a.rows_max = d.rows_max;
+    a.k = problem->k;
+    a.row_bytes = static_cast<uint32_t>(problem->H) * 2u;
+    a.seg_bytes = a.row_bytes < PERMUTE_SEG_BYTES ? a.row_bytes : PERMUTE_SEG_BYTES;
+    a.nseg = static_cast<int32_t>((a.row_bytes + a.seg_bytes - 1) / a.seg_bytes);
+    a.stages = PERMUTE_MAX_STAGES;
+    a.wait_limit_ns = WAIT_LIMIT_NS;
+    const size_t smem = static_cast<size_t>(a.stages) * a.seg_bytes;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, permute_kernel, 32, smem) != cudaSuccess ||
+        per_sm < 1)
+        return MOE_ERR_CUDA;
+    const int64_t units = problem->N * a.nseg;
+    int64_t grid = static_cast<int64_t>(dev.sms) * per_sm;
+    const int64_t want = units > 0 ? units : 1;
+    if (grid > want)
+        grid = want;
+    // the pad-row pass uses the same CTAs; keep at least a full wave for it
+    if (units < static_cast<int64_t>(dev.sms) * per_sm && d.rows_max > units)
+        grid = static_cast<int64_t>(dev.sms) * per_sm;
+    permute_kernel<<<static_cast<unsigned>(grid), 32, smem, static_cast<cudaStream_t>(stream)>>>(a);
+    return launch_status();
+}
+
+namespace {
+
+int launch_combine(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *y, const float *probs,
+                   uint16_t *out, void *stream)
+{
+    Dims d;
+    int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    if ((rc = check_layout(layout, d, false)) != MOE_OK)
+        return rc;
+    if (problem->N == 0)
+        return MOE_OK;
+    if (out == nullptr || !aligned16(out) || (d.rows_max > 0 && (y == nullptr || !aligned16(y))))
+        return MOE_ERR_INVALID;
+    CombineArgs a;
+    a.y = reinterpret_cast<const uint4 *>(y);
+    a.dest_row = layout->dest_row;
+    a.probs = probs;
+    a.out = reinterpret_cast<uint4 *>(out);
+    a.status = layout->status;
+    a.N = problem->N;
+    a.rows_max = d.rows_max;
+    a.k = problem->k;
+    a.V = problem->H / 8;
+    const int threads = a.V >= COMBINE_THREADS ? COMBINE_THREADS : ((a.V + 31) / 32) * 32;
+    a.nchunks = (a.V + threads - 1) / threads;
+    const int64_t blocks = problem->N * a.nchunks;
+    if (blocks > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const dim3 grid(static_cast<unsigned>(blocks)), block(threads);
+    switch (problem->k) {
+    case 1:
+        combine_kernel<1><<<grid, block, 0, s>>>(a);
+        break;
+    case 2:
+        combine_kernel<2><<<grid, block, 0, s>>>(a);
+        break;
+    case 4:
+        combine_kernel<4><<<grid, block, 0, s>>>(a);
+        break;
+    case 6:
+        combine_kernel<6><<<grid, block, 0, s>>>(a);
+        break;
+    case 8:
+        combine_kernel<8><<<grid, block, 0, s>>>(a);
+        break;
+    default:
+        combine_kernel<0><<<grid, block, 0, s>>>(a);
+        break;
+    }
+    return launch_status();
+}
+
+} // namespace
+
+int moe_combine(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *expert_out,
+                const float *topk_probs, uint16_t *out, void *stream)
+{
+    return launch_combine(problem, layout, expert_out, topk_probs, out, stream);
+}
+
+int moe_permute_backward(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *grad_send,
+                         uint16_t *grad_hidden, void *stream)
+{
+    return launch_combine(problem, layout, grad_send, nullptr, grad_hidden, stream);
+}
+
+int moe_combine_backward(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *grad_out,
+                         const uint16_t *expert_out, const float *topk_probs, uint16_t *grad_expert_out,
+                         float *grad_probs, void *stream)
+{
+    Dims d;
+    int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    if ((rc = check_layout(layout, d, true)) != MOE_OK)
+        return rc;
+    if (problem->N > 0 && (grad_out == nullptr || !aligned16(grad_out) || topk_probs == nullptr ||
+                           grad_probs == nullptr))
+        return MOE_ERR_INVALID;
+    if (d.rows_max > 0 && (expert_out == nullptr || !aligned16(expert_out) || grad_expert_out == nullptr ||
+                           !aligned16(grad_expert_out)))
+        return MOE_ERR_INVALID;
+    if (problem->N == 0 && d.rows_max == 0)
+        return MOE_OK;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev)) != MOE_OK)
+        return rc;
+    CombineBwdArgs a;
+    a.grad_out = reinterpret_cast<const uint4 *>(grad_out);
+    a.y = reinterpret_cast<const uint4 *>(expert_out);
+    a.dest_row = layout->dest_row;
+    a.probs = topk_probs;
+    a.pad_mask = layout->pad_mask;
+    a.grad_y = reinterpret_cast<uint4 *>(grad_expert_out);
+    a.grad_probs = grad_probs;
+    a.status = layout->status;
+    a.N = problem->N;
+    a.rows_max = d.rows_max;
+    a.k = problem->k;
+    a.V = problem->H / 8;
+    int64_t zb = (d.rows_max + 63) / 64;
+    const int64_t zmax = static_cast<int64_t>(dev.sms) * 2;
+    a.zero_blocks = static_cast<int32_t>(zb > zmax ? zmax : zb);
+    const int64_t blocks = problem->N + a.zero_blocks;
+    if (blocks > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const dim3 grid(static_cast<unsigned>(blocks)), block(COMBINE_BWD_THREADS);
+    switch (problem->k) {
+    case 1:
+        combine_backward_kernel<1><<<grid, block, 0, s>>>(a);
+        break;
+    case 2:
+        combine_backward_kernel<2><<<grid, block, 0, s>>>(a);
+        break;
+    case 4:
+        combine_backward_kernel<4><<<grid, block, 0, s>>>(a);
+        break;
+    case 6:
+        combine_backward_kernel<6><<<grid, block, 0, s>>>(a);
+        break;
+    case 8:
+        combine_backward_kernel<8><<<grid, block, 0, s>>>(a);
+        break;
+    default:
+        combine_backward_kernel<0><<<grid, block, 0, s>>>(a);
+        break;
+    }
+    return launch_status();
+}
+
+} // extern "C"

@@ -1,0 +1,235 @@
+/*
+ * moe_rt.h — C ABI of libmoert.so: MoE token dispatch and combine on one
+ * B200 (sm_100a), expert-parallel ranks simulated as contiguous partitions
+ * of the send buffer.
+ *
+ * Sources (page titles; sections named inline below):
+ *   [Megatron MORI]  "Add MORI as a Token Dispatcher" (ROCm/Megatron-LM PR #135)
+ *   [UltraEP]        "Integrate UltraEP Runtime for MoE EP Load Balancing" (InternLM/xtuner PR #2050)
+ *   [Megatron MoE]   "Megatron MoE 实现" (MoELayer.forward: route, dispatch, experts, combine)
+ *   [mscclpp HT]     mscclpp python/ page, high-throughput dispatch/combine summary
+ *   [DeepSpeed EP]   deepspeed/moe/ep_tp_dispatch.py (route-full / partition-dispatch helpers)
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Memory.  Every pointer argument is DEVICE memory owned by the caller, except
+ *   `problem` and `layout`, which are host structs read during the call only.
+ *   The library allocates nothing and keeps no state between calls. Tensors
+ *   are dense row-major; bf16 tensors are passed as uint16_t bit patterns.
+ *   hidden / send / expert-output / gradient buffers must be 16-byte aligned.
+ * Streams.  `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *   Every call only enqueues work on it: no host synchronisation, no host
+ *   read of device data ([Megatron MORI]: sync-free counts and padded buffers).
+ * Sizes.  Buffers have fixed upper-bound sizes ([Megatron MORI]: work on the
+ *   full [max_tokens, ...] padded buffers and mask the tail). rows_max =
+ *   E*capacity when capacity > 0, else N*k. N*k and rows_max must be < 2^31.
+ * Returns.  MOE_OK or a negative host-detected error; on error nothing is
+ *   enqueued. Device-detected problems are OR-ed into *layout->status as
+ *   MOE_DEV_* bits; read them when convenient (no call waits for them).
+ * Concurrency.  A layout / workspace pair backs one dispatch at a time
+ *   ([Megatron MORI] review thread: one staging region per op means two calls
+ *   of the same op must not be in flight together). Reusing the layout for
+ *   combine and both backward calls is intended ([mscclpp HT]: cached
+ *   dispatch via previous_handle).
+ */
+#ifndef MOE_RT_H
+#define MOE_RT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_RT_ABI_VERSION 1
+
+/* Every entry point is exported; everything else in the library is hidden. */
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+/* Host-detected return codes (nothing was enqueued). */
+#define MOE_OK 0
+#define MOE_ERR_INVALID (-1)     /* bad size, NULL required pointer, misaligned buffer, inconsistent problem */
+#define MOE_ERR_UNSUPPORTED (-2) /* valid but beyond the kernels' limits (see each call) */
+#define MOE_ERR_CUDA (-3)        /* a CUDA runtime call or launch failed */
+
+/* Device-detected status bits, OR-ed into *layout->status. */
+#define MOE_DEV_EXPERT_RANGE 0x1u /* a topk id outside [-1, E_log): the entry was skipped as if -1 */
+#define MOE_DEV_TIMEOUT 0x2u      /* a bounded device wait ran out; outputs of that call are invalid */
+#define MOE_DEV_ROW_RANGE 0x4u    /* a dest_row outside [-1, rows_max): that row was skipped */
+
+/* moe_problem_t.flags */
+#define MOE_FLAG_NONE 0u
+/* Test hook: the layout's grid barrier waits for one arrival that never comes,
+ * with a ~10 ms limit, so the timeout path can be exercised without hanging. */
+#define MOE_FLAG_TEST_BARRIER_TIMEOUT 0x80000000u
+
+/* The problem statement ([DeepSpeed EP] RoutedAssignmentPayload; it follows the
+ * pages' shapes: hidden [N,H] bf16, topk ids [N,k] int32, probs [N,k] fp32). */
+typedef struct {
+    int64_t N;            /* tokens (>= 0) */
+    int32_t H;            /* hidden size, a positive multiple of 8 (16-byte rows) */
+    int32_t k;            /* top-k, 1..32 */
+    int32_t E_log;        /* logical experts (router width), 1..2048, divisible by R */
+    int32_t num_replicas; /* UltraEP replica slots in total (0 = no reroute), divisible by R, <= E_log */
+    int32_t R;            /* simulated EP ranks, >= 1 */
+    int32_t capacity;     /* per-expert capacity C (0 = unlimited) */
+    uint32_t flags;       /* MOE_FLAG_* */
+} moe_problem_t;
+
+/*
+ * Outputs of moe_dispatch_layout, all device buffers of the sizes shown
+ * (E = E_log + num_replicas physical experts, E_loc = E / R per rank).
+ * Physical numbering: rank r owns experts [r*E_loc, (r+1)*E_loc); with replicas
+ * the first E_log/R of them are the masters of logical experts
+ * r*E_log/R + i, the rest are replica slots.
+ */
+typedef struct {
+    /* per assignment a = t*k + j, [N*k] */
+    int32_t *phys_idx;  /* physical expert, -1 for a -1 (or skipped) id */
+    int32_t *ordinal;   /* stable rank among earlier assignments to the same physical expert, -1 as above */
+    int32_t *dest_row;  /* send-buffer row, -1 if the id is -1 or the assignment was dropped */
+    uint8_t *drop_mask; /* 1 = over capacity */
+    /* per logical expert, [E_log] */
+    int32_t *counts_logical; /* router histogram before reroute */
+    int32_t *placement;      /* physical replica slot of a hot expert, else -1 */
+    /* per physical expert */
+    int32_t *counts_raw;        /* [E] assignments before capacity */
+    int32_t *tokens_per_expert; /* [E] rows filled: min(counts_raw, C), or counts_raw when C = 0 */
+    int32_t *expert_offsets;    /* [E+1] first row of each expert (e*C when C > 0) */
+    /* per rank */
+    int32_t *input_splits;  /* [R] rows destined to rank r (pad rows included when C > 0) */
+    int32_t *output_splits; /* [R] equal to input_splits on one GPU */
+    int32_t *rank_offsets;  /* [R+1] first row of each rank */
+    /* scalars */
+    int32_t *counters; /* [8] assignments_total, kept, dropped, padded, split_sum_in, split_sum_out, num_rows, error */
+    int32_t *num_rows; /* [1] expert_offsets[E] */
+    uint32_t *status;  /* [1] MOE_DEV_* bits; the caller zeroes it, calls only OR into it */
+    /* per send-buffer row, [rows_max] */
+    int32_t *row_token;        /* source token, -1 in pad / tail rows */
+    int32_t *row_slot;         /* top-k slot j, -1 in pad / tail rows */
+    int32_t *row_local_expert; /* expert id local to the row's rank, -1 in pad / tail rows */
+    float *row_prob;           /* receiver-side prob p[t,j], 0 in pad / tail rows */
+    uint8_t *pad_mask;         /* 1 = the row holds no assignment */
+    /* optional DeepEP-contract view, [R*N*k] or NULL */
+    int32_t *local_topk; /* [r][t][j]: local id if (t,j) is kept on rank r, else -1 */
+} moe_layout_t;
+
+/* ABI version of the loaded library (MOE_RT_ABI_VERSION it was built with). */
+MOE_API int moe_abi_version(void);
+
+/* Static text for a return code or a single MOE_DEV_* bit. Never NULL. */
+MOE_API const char *moe_status_string(int code);
+
+/*
+ * Number of send-buffer rows (the first dimension of send / expert_out /
+ * row_* buffers): E*capacity if capacity > 0, else N*k. Host only.
+ * Returns a negative MOE_ERR_* if the problem is invalid.
+ */
+MOE_API int64_t moe_rows_max(const moe_problem_t *problem);
+
+/*
+ * Bytes of device scratch moe_dispatch_layout needs (per-block histograms and
+ * a grid barrier). Host only. The scratch must be zero-filled before its first
+ * use; afterwards every call leaves it ready for the next one, except a call
+ * that reported MOE_DEV_TIMEOUT, after which it must be zero-filled again.
+ * Returns MOE_OK and sets *bytes, or a negative MOE_ERR_*.
+ */
+MOE_API int moe_layout_workspace_bytes(const moe_problem_t *problem, size_t *bytes);
+
+/*
+ * Router: softmax over E fp32 logits and top-k
+ * ([Megatron MoE] MoELayer.router_and_preprocess; [Megatron MORI] router.py:
+ * padding tokens do not take part in routing).
+ *   logits      [N, E] fp32, device
+ *   token_mask  [N] uint8 or NULL; a token with mask != 0 gets ids -1, probs 0
+ *   topk_idx    [N, k] int32 out: the k largest logits, descending; equal
+ *               logits to the lower expert id
+ *   topk_probs  [N, k] fp32 out: exp(l - max) / sum_e exp(l - max) over all E
+ *               (no renormalisation over the k chosen), CUDA expf
+ * Limits: 1 <= k <= min(E, 32), E <= 1024 (MOE_ERR_UNSUPPORTED beyond).
+ */
+MOE_API int moe_route_topk(const float *logits, const uint8_t *token_mask, int64_t N, int32_t E, int32_t k,
+                   int32_t *topk_idx, float *topk_probs, void *stream);
+
+/*
+ * Dispatch layout: optional UltraEP reroute, histogram, stable ordinals,
+ * capacity drop / pad, exclusive scan, rank splits, row maps and the local
+ * view, in one cooperative launch.
+ *   [UltraEP]: hot-expert replicas from the layer's actual load, tokens
+ *     rerouted logical -> physical; router semantics stay logical.
+ *   [DeepSpeed EP] assignment_ordinals_by_expert: stable ordinals per expert;
+ *     RoutedAssignmentPayload capacity_slots / drop_mask / pad_mask;
+ *     _recompute_input_splits / partition_assignments: splits and counters.
+ *   [Megatron MORI]: local ids with -1 sentinels, receiver-side probs, tails
+ *     masked 0 / -1 / 0, fixed-size scatter instead of bincount (no host sync).
+ * Readings where the pages are silent: ordinals follow the flattened [N,k]
+ * order; drops are first-come; hot experts = the num_replicas largest
+ * logical counts (ties to the lower id), placed greedily on the least-loaded
+ * other rank with a free replica slot (own rank only if no other is free);
+ * a hot expert's logical ordinal o goes to the master if o is even, to the
+ * replica if odd (physical ordinal o/2).
+ *   topk_idx    [N, k] int32, ids in [-1, E_log); others are skipped (MOE_DEV_EXPERT_RANGE)
+ *   topk_probs  [N, k] fp32 or NULL (row_prob then 0)
+ *   layout      every pointer except local_topk must be non-NULL
+ *   workspace   moe_layout_workspace_bytes() bytes, zero-filled before first use
+ * Limits: E_log <= 2048, k <= 32, R <= 64 when num_replicas > 0.
+ */
+MOE_API int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, const float *topk_probs,
+                        const moe_layout_t *layout, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Permute ([Megatron MoE] dispatch_postprocess; [Megatron MORI] permute fused
+ * into the dispatch node): send[dest_row[t,j]] = hidden[t] for every kept
+ * (t,j); rows with pad_mask = 1 are zero-filled. Byte copy, bit-exact.
+ * Reads layout->dest_row and layout->pad_mask.
+ *   hidden [N, H] bf16; send [rows_max, H] bf16 (must not overlap hidden)
+ */
+MOE_API int moe_permute(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *hidden, uint16_t *send,
+                void *stream);
+
+/*
+ * Combine ([DeepSpeed EP] restore_combined: weighted rows added back one
+ * top-k slot at a time in ascending slot order; [Megatron MoE] combine):
+ *   out[t,h] = bf16_rn( fp32 chain acc = fmaf(p[t,j], y[dest_row[t,j], h], acc)
+ *                       over ascending j with dest_row >= 0, from acc = +0 )
+ * Deterministic, no atomics, bit-exact with the CPU definition.
+ *   expert_out [rows_max, H] bf16; topk_probs [N, k] fp32 or NULL (unit
+ *   weights); out [N, H] bf16. Reads layout->dest_row.
+ */
+MOE_API int moe_combine(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *expert_out,
+                const float *topk_probs, uint16_t *out, void *stream);
+
+/*
+ * Backward of permute ([Megatron MORI]: dispatch backward sums the row
+ * gradients back per token with receiver-side indices): combine with unit
+ * weights, grad_hidden[t] = bf16_rn( fp32 sum over ascending kept j of
+ * grad_send[dest_row[t,j]] ).
+ *   grad_send [rows_max, H] bf16; grad_hidden [N, H] bf16
+ */
+MOE_API int moe_permute_backward(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *grad_send,
+                         uint16_t *grad_hidden, void *stream);
+
+/*
+ * Backward of combine ([Megatron MORI]: combine backward with receiver-side
+ * probs):
+ *   grad_expert_out[dest_row[t,j]] = bf16_rn( fp32(p[t,j] * grad_out[t]) ); pad rows 0
+ *   grad_probs[t,j] = fp32 sum_h grad_out[t,h] * expert_out[dest_row[t,j],h]; 0 if no row
+ * grad_probs is a deterministic fp32 tree reduction (not bit-equal to a
+ * sequential sum; within the fp32 summation error bound).
+ *   grad_out [N,H] bf16; expert_out [rows_max,H] bf16; topk_probs [N,k] fp32;
+ *   grad_expert_out [rows_max,H] bf16; grad_probs [N,k] fp32.
+ *   Reads layout->dest_row and layout->pad_mask.
+ */
+MOE_API int moe_combine_backward(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *grad_out,
+                         const uint16_t *expert_out, const float *topk_probs, uint16_t *grad_expert_out,
+                         float *grad_probs, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_RT_H */

@@ -1,0 +1,319 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Bar: bit-exact for every integer, mask, row-map and copied output, for the
+combine / permute-backward outputs (fixed fp32 fma order, one bf16 rounding)
+and for grad_expert_out (one fp32 product, one rounding). Router probs and
+grad_probs are within bounds derived from their fp32 arithmetic (router:
+tests/gpu_util.py; grad_probs: the fp32 summation bound gamma_H * sum|g*y|).
+
+All five workloads run at their full sizes, with the same launch
+configuration the benchmark uses. Inputs come from ``synthetic``; the oracle
+route output feeds both sides so that layout/combine parity never depends on
+expf rounding.
+"""
+
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import combine_moe_route_tokens_b200 as moe
+import oracle
+from synthetic import bf16_bits_from_f32, get_workload, make_inputs
+from synthetic.workloads import make_token_mask
+
+from gpu_util import dev, host, require_cuda, route_prob_tolerance
+
+pytestmark = pytest.mark.gpu
+
+WORKLOAD_NAMES = ["tiny", "ht", "qwen3", "capacity", "ultraep"]
+LAYOUT_KEYS = [
+    "phys_idx", "ordinal", "dest_row", "drop_mask", "counts_logical", "placement", "counts_raw",
+    "tokens_per_expert", "expert_offsets", "input_splits", "output_splits", "rank_offsets", "counters",
+    "num_rows", "row_token", "row_slot", "row_local_expert", "row_prob", "pad_mask", "local_topk",
+]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    require_cuda()
+    moe.load_library()
+
+
+_cache = {}
+
+
+def workload_case(name):
+    """Inputs and the oracle's route + layout for a workload (cached per module)."""
+    if name not in _cache:
+        w = get_workload(name)
+        d = make_inputs(w, grad=True)
+        idx, probs = oracle.route_topk(d["logits"], w.k)
+        L = oracle.layout(idx, probs, E_log=w.E_log, R=w.R, C=w.capacity, num_replicas=w.num_replicas)
+        _cache.clear()
+        _cache[name] = (w, d, idx, probs, L)
+    return _cache[name]
+
+
+def problem_of(w, N=None):
+    return moe.Problem(N=w.N if N is None else N, H=w.H, k=w.k, E_log=w.E_log, R=w.R, capacity=w.capacity,
+                       num_replicas=w.num_replicas)
+
+
+def assert_layout_equal(G, L):
+    for key in LAYOUT_KEYS:
+        got = host(G[key]).reshape(-1)
+        exp = np.asarray(L[key]).reshape(-1)
+        if key == "row_prob":
+            assert np.array_equal(got.view(np.uint32), exp.astype(np.float32).view(np.uint32)), key
+        else:
+            assert np.array_equal(got.astype(np.int64), exp.astype(np.int64)), key
+
+
+@pytest.mark.parametrize("name", WORKLOAD_NAMES)
+def test_route(name):
+    w, d, idx, probs, _ = workload_case(name)
+    gi, gp = moe.moe_route_topk(dev(d["logits"]), w.k)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(gi), idx)
+    tol = route_prob_tolerance(d["logits"], idx) * probs.astype(np.float64)
+    assert np.all(np.abs(host(gp).astype(np.float64) - probs.astype(np.float64)) <= tol)
+
+
+@pytest.mark.parametrize("name", WORKLOAD_NAMES)
+def test_layout(name):
+    w, d, idx, probs, L = workload_case(name)
+    G = moe.moe_dispatch_layout(problem_of(w), dev(idx), dev(probs))
+    torch.cuda.synchronize()
+    assert_layout_equal(G, L)
+    assert G.status() == 0
+
+
+@pytest.mark.parametrize("name", WORKLOAD_NAMES)
+def test_permute_combine(name):
+    w, d, idx, probs, L = workload_case(name)
+    p = problem_of(w)
+    G = moe.moe_dispatch_layout(p, dev(idx), dev(probs))
+    send = moe.moe_permute(p, G, dev(d["hidden"]))
+    send_h = host(send)
+    exp_send = oracle.permute(d["hidden"], L["dest_row"], L["rows_max"])
+    assert np.array_equal(send_h, exp_send)
+    # identity experts: y = send
+    out = moe.moe_combine(p, G, send, dev(probs))
+    assert np.array_equal(host(out), oracle.combine(exp_send, L["dest_row"], probs))
+    out1 = moe.moe_combine(p, G, send, None)
+    assert np.array_equal(host(out1), oracle.combine(exp_send, L["dest_row"], None))
+    assert G.status() == 0
+
+
+@pytest.mark.parametrize("name", WORKLOAD_NAMES)
+def test_backward(name):
+    w, d, idx, probs, L = workload_case(name)
+    p = problem_of(w)
+    G = moe.moe_dispatch_layout(p, dev(idx), dev(probs))
+    y = oracle.permute(d["hidden"], L["dest_row"], L["rows_max"])  # identity-expert outputs
+    gy, gp = moe.moe_combine_backward(p, G, dev(d["grad_out"]), dev(y), dev(probs))
+    exp_gy, exp_gp = oracle.combine_backward(d["grad_out"], y, L["dest_row"], L["row_token"], L["row_prob"])
+    assert np.array_equal(host(gy), exp_gy)
+    # grad_probs: fp32 accumulation in some fixed order vs the oracle's double sum
+    gf = d["grad_out"].astype(np.uint32) << 16
+    g = gf.view(np.float32).astype(np.float64)
+    yf = (y.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    dest = L["dest_row"]
+    S = np.zeros_like(exp_gp, dtype=np.float64)
+    for j in range(w.k):
+        rows = np.maximum(dest[:, j], 0)
+        S[:, j] = np.einsum("nh,nh->n", np.abs(g), np.abs(yf[rows]))
+    u = 2.0 ** -24
+    gamma = w.H * u / (1 - w.H * u)
+    got = host(gp).astype(np.float64)
+    assert np.all(np.abs(got - exp_gp.astype(np.float64)) <= gamma * S + 2 * u * np.abs(exp_gp) + 1e-30)
+    assert np.all(got[dest < 0] == 0)
+    # permute backward = unit-weight combine of grad_send (here: the grads just produced)
+    gh = moe.moe_permute_backward(p, G, gy)
+    assert np.array_equal(host(gh), oracle.permute_backward(exp_gy, L["dest_row"]))
+    assert G.status() == 0
+
+
+def test_layout_is_deterministic_and_reusable():
+    w, d, idx, probs, L = workload_case("qwen3")
+    p = problem_of(w)
+    G = moe.Layout.allocate(p)
+    for _ in range(3):  # the workspace's barrier state is left ready for the next call
+        moe.moe_dispatch_layout(p, dev(idx), dev(probs), layout=G)
+        torch.cuda.synchronize()
+        assert_layout_equal(G, L)
+
+
+# ---------------------------------------------------------------- edge cases
+
+
+def _small_case(N, H, k, E_log, R, C=0, reps=0, neg=0.0, seed=0, zipf=None, bad=0):
+    rng = np.random.default_rng(seed)
+    if zipf:
+        idx = (rng.zipf(zipf, size=(N, k)) % E_log).astype(np.int32)
+    else:
+        idx = rng.integers(0, E_log, size=(N, k)).astype(np.int32)
+    if neg:
+        idx[rng.random((N, k)) < neg] = -1
+    if bad:
+        flat = idx.reshape(-1)
+        pos = rng.choice(flat.size, size=min(bad, flat.size), replace=False)
+        flat[pos] = np.where(rng.random(len(pos)) < 0.5, E_log + 3, -7)
+    probs = rng.random((N, k)).astype(np.float32)
+    hidden = bf16_bits_from_f32(rng.standard_normal((N, H)).astype(np.float32))
+    return idx, probs, hidden
+
+
+EDGE_CASES = [
+    # N, H, k, E_log, R, C, reps, neg, zipf
+    (1, 8, 1, 1, 1, 0, 0, 0.0, None),
+    (3, 24, 3, 5, 1, 0, 0, 0.0, None),  # generic-k kernels, ragged row (3 x 16 B)
+    (37, 264, 6, 12, 3, 0, 0, 0.2, None),
+    (1000, 1032, 12, 40, 4, 0, 0, 0.1, 1.3),  # k beyond the specialised set
+    (5000, 520, 2, 64, 4, 90, 0, 0.05, 1.5),  # capacity with drops and pads
+    (4099, 136, 8, 128, 8, 0, 8, 0.0, 1.2),  # reroute, ragged block tail
+    (2048, 64, 4, 32, 2, 40, 4, 0.1, 1.4),  # reroute + capacity
+    (777, 16, 8, 2048, 1, 0, 0, 0.0, None),  # widest router supported
+    (300, 20000, 2, 8, 2, 0, 0, 0.0, None),  # row of 40000 B: two TMA segments
+    (70000, 8, 1, 4, 2, 0, 0, 0.0, None),  # many blocks, tiny rows
+]
+
+
+@pytest.mark.parametrize("case", EDGE_CASES, ids=[f"N{c[0]}_H{c[1]}_k{c[2]}_E{c[3]}" for c in EDGE_CASES])
+def test_edge_cases_full_path(case):
+    N, H, k, E_log, R, C, reps, neg, zipf = case
+    idx, probs, hidden = _small_case(N, H, k, E_log, R, C, reps, neg, seed=N, zipf=zipf)
+    L = oracle.layout(idx, probs, E_log=E_log, R=R, C=C, num_replicas=reps)
+    p = moe.Problem(N=N, H=H, k=k, E_log=E_log, R=R, capacity=C, num_replicas=reps)
+    G = moe.moe_dispatch_layout(p, dev(idx), dev(probs))
+    torch.cuda.synchronize()
+    assert_layout_equal(G, L)
+    send = moe.moe_permute(p, G, dev(hidden))
+    exp_send = oracle.permute(hidden, L["dest_row"], L["rows_max"])
+    assert np.array_equal(host(send), exp_send)
+    assert np.array_equal(host(moe.moe_combine(p, G, send, dev(probs))),
+                          oracle.combine(exp_send, L["dest_row"], probs))
+    rng = np.random.default_rng(1)
+    g = bf16_bits_from_f32(rng.standard_normal((N, H)).astype(np.float32))
+    gy, gp = moe.moe_combine_backward(p, G, dev(g), send, dev(probs))
+    exp_gy, exp_gp = oracle.combine_backward(g, exp_send, L["dest_row"], L["row_token"], L["row_prob"])
+    assert np.array_equal(host(gy), exp_gy)
+    assert np.allclose(host(gp), exp_gp, rtol=1e-4, atol=1e-4 * np.sqrt(H))
+    assert np.array_equal(host(moe.moe_permute_backward(p, G, gy)), oracle.permute_backward(exp_gy, L["dest_row"]))
+    assert G.status() == 0
+
+
+@pytest.mark.parametrize("C", [0, 5])
+def test_empty_batch(C):
+    p = moe.Problem(N=0, H=16, k=2, E_log=4, R=2, capacity=C)
+    idx = torch.zeros((0, 2), dtype=torch.int32, device="cuda")
+    G = moe.moe_dispatch_layout(p, idx, None)
+    send = moe.moe_permute(p, G, torch.zeros((0, 16), dtype=torch.bfloat16, device="cuda"))
+    out = moe.moe_combine(p, G, send, None)
+    torch.cuda.synchronize()
+    L = oracle.layout(np.zeros((0, 2), np.int32), None, E_log=4, R=2, C=C)
+    assert_layout_equal(G, L)
+    assert out.shape == (0, 16) and send.shape == (L["rows_max"], 16)
+    assert torch.all(send == 0)
+
+
+def test_padding_tokens_via_route_mask():
+    w = dataclasses.replace(get_workload("tiny"), N=300)
+    d = make_inputs(w)
+    mask = make_token_mask(w, 0.3)
+    gi, gp = moe.moe_route_topk(dev(d["logits"]), w.k, token_mask=dev(mask))
+    idx, probs = oracle.route_topk(d["logits"], w.k, token_mask=mask)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(gi), idx)
+    assert np.all(host(gp)[mask == 1] == 0)
+    p = problem_of(w)
+    G = moe.moe_dispatch_layout(p, dev(idx), dev(probs))
+    L = oracle.layout(idx, probs, E_log=w.E_log, R=w.R)
+    torch.cuda.synchronize()
+    assert_layout_equal(G, L)
+    assert int(host(G["num_rows"])[0]) < w.N * w.k  # a tail of pad rows
+    send = moe.moe_permute(p, G, dev(d["hidden"]))
+    assert np.array_equal(host(send), oracle.permute(d["hidden"], L["dest_row"], L["rows_max"]))
+
+
+def test_out_of_range_ids_flagged_and_skipped():
+    idx, probs, hidden = _small_case(500, 64, 4, 16, 4, bad=37, seed=3)
+    p = moe.Problem(N=500, H=64, k=4, E_log=16, R=4)
+    G = moe.moe_dispatch_layout(p, dev(idx), dev(probs))
+    L = oracle.layout(idx, probs, E_log=16, R=4)
+    torch.cuda.synchronize()
+    assert L["counters"][7] == 1
+    assert G.status() == moe.MOE_DEV_EXPERT_RANGE
+    got = host(G["counters"])
+    assert got[7] == moe.MOE_DEV_EXPERT_RANGE
+    L["counters"][7] = moe.MOE_DEV_EXPERT_RANGE  # the device reports the bit, the oracle a flag
+    assert_layout_equal(G, L)
+
+
+def test_outputs_stay_inside_their_buffers():
+    """Canary rows after every row-indexed output must be untouched."""
+    idx, probs, hidden = _small_case(600, 72, 4, 16, 4, C=100, neg=0.1, zipf=1.4, seed=9)
+    p = moe.Problem(N=600, H=72, k=4, E_log=16, R=4, capacity=100)
+    RM = p.rows_max
+    guard = 17
+    G = moe.Layout.allocate(p)
+    for key in ("row_token", "row_slot", "row_local_expert", "row_prob", "pad_mask"):
+        big = torch.full((RM + guard,), 0x5A, dtype=G[key].dtype, device="cuda")
+        G.tensors[key] = big[:RM]
+        G.tensors[key + "_guard"] = big
+    moe.moe_dispatch_layout(p, dev(idx), dev(probs), layout=G)
+    send_big = torch.full((RM + guard, 72), 1.5, dtype=torch.bfloat16, device="cuda")
+    moe.moe_permute(p, G, dev(hidden), send=send_big[:RM])
+    out_big = torch.full((600 + guard, 72), -2.0, dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine(p, G, send_big[:RM], dev(probs), out=out_big[:600])
+    gy_big = torch.full((RM + guard, 72), 3.0, dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine_backward(p, G, out_big[:600].clone(), send_big[:RM], dev(probs), grad_expert_out=gy_big[:RM])
+    torch.cuda.synchronize()
+    for key in ("row_token", "row_slot", "row_local_expert", "row_prob", "pad_mask"):
+        tail = G.tensors[key + "_guard"][RM:]
+        assert torch.all(tail == torch.full_like(tail, 0x5A)), key
+    assert torch.all(send_big[RM:] == 1.5) and torch.all(out_big[600:] == -2.0) and torch.all(gy_big[RM:] == 3.0)
+
+
+def test_barrier_timeout_reports_and_recovers():
+    """The layout's grid barrier gives up after its limit and says so; the context stays usable."""
+    idx, probs, hidden = _small_case(4000, 16, 2, 8, 2, seed=4)
+    p_bad = moe.Problem(N=4000, H=16, k=2, E_log=8, R=2, flags=moe.MOE_FLAG_TEST_BARRIER_TIMEOUT)
+    G = moe.moe_dispatch_layout(p_bad, dev(idx), dev(probs))
+    torch.cuda.synchronize()
+    assert G.status() & moe.MOE_DEV_TIMEOUT
+    # after a timeout the workspace is zeroed, then a normal call works
+    p = dataclasses.replace(p_bad, flags=0)
+    G2 = moe.Layout.allocate(p)
+    moe.moe_dispatch_layout(p, dev(idx), dev(probs), layout=G2)
+    torch.cuda.synchronize()
+    assert G2.status() == 0
+    assert_layout_equal(G2, oracle.layout(idx, probs, E_log=8, R=2))
+
+
+def test_misaligned_tensor_rejected_by_library():
+    p = moe.Problem(N=4, H=8, k=2, E_log=4, R=2)
+    idx = torch.zeros((4, 2), dtype=torch.int32, device="cuda")
+    G = moe.moe_dispatch_layout(p, idx, None)
+    base = torch.zeros(4 * 8 + 1, dtype=torch.bfloat16, device="cuda")
+    hidden = base[1:].view(4, 8)  # 2-byte offset
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_permute(p, G, hidden)
+    assert ei.value.code == -1
+
+
+def test_streams_are_respected():
+    w, d, idx, probs, L = workload_case("tiny")
+    p = problem_of(w)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        ii, pp = dev(idx), dev(probs)
+        hid = dev(d["hidden"])
+        G = moe.moe_dispatch_layout(p, ii, pp)
+        send = moe.moe_permute(p, G, hid)
+        out = moe.moe_combine(p, G, send, pp)
+    s.synchronize()
+    exp_send = oracle.permute(d["hidden"], L["dest_row"], L["rows_max"])
+    assert np.array_equal(host(out), oracle.combine(exp_send, L["dest_row"], probs))
