@@ -26,7 +26,7 @@
 
 namespace moert {
 
-constexpr int COMBINE_THREADS = 128;
+constexpr int COMBINE_THREADS = 256; // widest CTA; the host picks 32..256 to split the row evenly
 constexpr int COMBINE_BWD_THREADS = 128;
 constexpr int COMBINE_MAX_K = 32;
 
@@ -81,6 +81,8 @@ __device__ __forceinline__ void load_slot_meta(const int32_t *dest_row, const fl
 template <int K> // K > 0: top-k fixed at compile time; K == 0: runtime k <= 32
 __global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(CombineArgs a)
 {
+    pdl_trigger();
+    pdl_wait();
     const int64_t t = blockIdx.x / a.nchunks;
     const int c = static_cast<int>(blockIdx.x - t * a.nchunks);
     const int v = c * blockDim.x + threadIdx.x;
@@ -201,11 +203,12 @@ __global__ void __launch_bounds__(COMBINE_BWD_THREADS) combine_backward_kernel(C
 {
     __shared__ float s_red[COMBINE_BWD_THREADS / 32];
     __shared__ float s_part[COMBINE_BWD_THREADS / 32][K > 0 ? K : 1];
+    pdl_trigger();
+    pdl_wait();
     if (blockIdx.x >= a.N) {
         const int64_t workers = static_cast<int64_t>(a.zero_blocks) * (COMBINE_BWD_THREADS / 32);
         const int64_t worker = (blockIdx.x - a.N) * (COMBINE_BWD_THREADS / 32) + (threadIdx.x >> 5);
-        zero_pad_rows_warp(reinterpret_cast<uint8_t *>(a.grad_y), a.pad_mask, a.rows_max,
-                           static_cast<uint32_t>(a.V) * 16u, worker, workers);
+        zero_pad_rows_warp(a.grad_y, a.pad_mask, a.rows_max, a.V, worker, workers);
         return;
     }
     const int64_t t = blockIdx.x;

@@ -1,22 +1,23 @@
 // layout.cuh — the dispatch layout in one cooperative launch.
 //
 // Steps (page citations in moe_rt.h, moe_dispatch_layout):
-//   phase 1  per-warp histograms of the logical ids of a contiguous slice of
-//            the flattened [N,k] assignments (warp-aggregated with
-//            __match_any_sync, one shared-memory add per distinct expert),
-//            turned into per-warp exclusive prefixes and a per-block total
-//            published to the workspace;
-//   barrier  bounded grid barrier (co-residency guaranteed by the
-//            cooperative launch);
-//   phase 2  every block reads all block totals and so knows, per logical
-//            expert, the total count and the count in earlier blocks; it
-//            derives the hot-expert placement, physical counts, capacity,
-//            the exclusive scan and the rank splits (block 0 publishes them),
-//            then re-walks its slice: the stable logical ordinal of an
-//            assignment is  earlier blocks + earlier warps + earlier
-//            iterations of its warp + earlier lanes with the same id, and the
-//            physical ordinal, drop flag and destination row follow in closed
-//            form. Finally the pad / tail rows of the row maps are filled.
+//   phase 1  each warp loads its contiguous slice of the flattened [N,k]
+//            assignments (ids and probs, kept in registers), ranks every
+//            assignment among the earlier ones of its warp with the same id
+//            (__match_any_sync + popc, one shared-memory counter update per
+//            distinct id), then the block turns its per-warp counts into
+//            per-warp exclusive prefixes and publishes its per-expert total;
+//   barrier  bounded grid barrier (acquire/release atomics; co-residency is
+//            guaranteed by the cooperative launch);
+//   phase 2  every block reads all block totals in one batch of loads, so it
+//            knows per logical expert the total count and the count in
+//            earlier blocks; it derives the hot-expert placement, physical
+//            counts, capacity, the exclusive scan and the rank splits (block 0
+//            publishes them); then, with no further global reads, it writes
+//            every per-assignment and per-row output: the stable logical
+//            ordinal is  earlier blocks + earlier warps + earlier items of the
+//            same warp, and the physical ordinal, drop flag and row follow in
+//            closed form. Finally the pad / tail rows of the row maps.
 //
 // Closed forms used by phase 2 (equal to counting physical ordinals
 // directly, as the CPU definition does): a hot expert's assignment with
@@ -36,7 +37,9 @@ constexpr int LAYOUT_THREADS = 512;
 constexpr int LAYOUT_WARPS = LAYOUT_THREADS / 32;
 constexpr int LAYOUT_MAX_BLOCKS = 128;
 constexpr int LAYOUT_MAX_E_LOG = 2048;
-constexpr int LAYOUT_ITEMS_PER_BLOCK = 1024; // target slice per block before the block cap
+constexpr int LAYOUT_MAX_PLACEMENT_RANKS = 64;
+constexpr int LAYOUT_MAX_IPL = 8; // assignments per lane held in registers
+constexpr int LAYOUT_ITEMS_PER_BLOCK = 512; // target slice per block before the block cap
 
 struct LayoutArgs {
     const int32_t *topk_idx;
@@ -46,50 +49,62 @@ struct LayoutArgs {
     int32_t k, E_log, E, R, E_loc, M, S, num_replicas, C;
     int32_t sub; // assignments per warp slice, a multiple of 32
     int32_t G;   // blocks
-    int32_t *ws_counts;   // [G][E_log + 1]: per-block logical totals, last column = error bits
-    uint32_t *ws_barrier; // [2]: arrival count, generation
+    int32_t *ws_counts;   // [G][E_log]: per-block logical totals
+    uint32_t *ws_barrier; // [3]: arrival count, generation, error bits of this call
     uint64_t barrier_limit_ns;
     uint32_t barrier_extra; // test hook: extra arrivals the barrier waits for
     moe_layout_t out;
 };
 
-// Dynamic shared memory layout, in 32-bit words.
+// Dynamic shared memory, in 32-bit words.
 __host__ __device__ inline size_t layout_smem_words(int E_log, int E)
 {
-    return static_cast<size_t>(LAYOUT_WARPS) * E_log // per-warp counters
+    return static_cast<size_t>(LAYOUT_WARPS) * E_log // per-warp counters, then prefixes
            + 3 * static_cast<size_t>(E_log)          // block prefix, totals, placement
            + 2 * static_cast<size_t>(E) + 1;         // physical counts, offsets
 }
 
-constexpr int LAYOUT_MAX_PLACEMENT_RANKS = 64;
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
 
-// Bounded grid barrier with a generation counter; the state words are left
-// ready for the next launch (count back to 0) unless the wait ran out.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_u32(uint32_t *p, uint32_t v)
+{
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void red_release_add_u32(uint32_t *p, uint32_t v)
+{
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Bounded grid barrier with a generation word. The arrival count goes back to
+// 0 for the next launch unless the wait ran out.
 __device__ __forceinline__ bool layout_grid_barrier(uint32_t *bar, uint32_t target, uint64_t limit_ns)
 {
     __shared__ int s_ok;
     __syncthreads();
     if (threadIdx.x == 0) {
-        volatile uint32_t *vgen = bar + 1;
-        const uint32_t gen = *vgen;
-        __threadfence();
-        const uint32_t arrived = atomicAdd(bar, 1u);
+        const uint32_t gen = ld_acquire_u32(bar + 1);
+        const uint32_t arrived = atom_add_acq_rel_u32(bar, 1u);
         int ok = 1;
         if (arrived == target - 1) {
             atomicExch(bar, 0u);
-            __threadfence();
-            atomicAdd(bar + 1, 1u);
+            red_release_add_u32(bar + 1, 1u);
         } else {
             const uint64_t t0 = global_timer_ns();
-            while (*vgen == gen) {
-                __nanosleep(100);
+            while (ld_acquire_u32(bar + 1) == gen) {
                 if (global_timer_ns() - t0 > limit_ns) {
                     ok = 0;
                     break;
                 }
             }
         }
-        __threadfence();
         s_ok = ok;
     }
     __syncthreads();
@@ -103,100 +118,102 @@ __device__ __forceinline__ uint32_t lanemask_lt()
     return m;
 }
 
-// Hot set and greedy placement for the reroute, computed identically by every
-// block from the logical totals. Warp 0 ranks the experts by (count desc, id
-// asc) with num_replicas rounds of a warp arg-max; lane 0 then places them.
-__device__ void layout_placement(const LayoutArgs &a, const int32_t *s_cnt, int32_t *s_repl, int64_t *s_load,
-                                 int32_t *s_free, int32_t *s_hot)
+// Hot set and greedy placement for the reroute (warp 0; every block computes
+// the same result from the same totals). Hot experts: num_replicas rounds of
+// a warp arg-max over (count desc, id asc). Placement, per hot expert in that
+// order: the least-loaded rank (lowest id on ties) among the ranks other than
+// the master's that still have a free replica slot, else the master's own
+// rank; then floor(c/2) of load moves from the master's rank to it.
+__device__ void layout_placement(const LayoutArgs &a, const int32_t *s_cnt, int32_t *s_repl, int32_t *s_hot)
 {
     const int lane = threadIdx.x & 31;
     if (threadIdx.x >= 32)
         return;
-    for (int r = lane; r < a.R; r += 32) {
-        int64_t l = 0;
-        for (int i = 0; i < a.M; ++i)
-            l += s_cnt[r * a.M + i];
-        s_load[r] = l;
-        s_free[r] = a.S;
-    }
     uint64_t taken = 0; // bit u: expert lane + 32u already chosen (E_log <= 2048)
     for (int h = 0; h < a.num_replicas; ++h) {
-        uint64_t best = 0;
+        uint32_t best = 0;
+        int be = -1;
         for (int u = 0, e = lane; e < a.E_log; ++u, e += 32) {
-            if ((taken >> u) & 1ull)
-                continue;
-            const uint64_t key =
-                (static_cast<uint64_t>(static_cast<uint32_t>(s_cnt[e])) << 32) | static_cast<uint32_t>(~e);
-            best = key > best ? key : best;
+            const uint32_t c = static_cast<uint32_t>(s_cnt[e]) + 1u; // +1: 0 marks "none"
+            if (!((taken >> u) & 1ull) && c > best) {
+                best = c;
+                be = e;
+            }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
-            best = other > best ? other : best;
-        }
-        const int e = static_cast<int>(~static_cast<uint32_t>(best));
+        const uint32_t wmax = __reduce_max_sync(0xffffffffu, best);
+        const uint32_t cand = (best == wmax && be >= 0) ? ~static_cast<uint32_t>(be) : 0u;
+        const int e = static_cast<int>(~__reduce_max_sync(0xffffffffu, cand));
         if ((e & 31) == lane)
             taken |= 1ull << (e >> 5);
         if (lane == 0)
             s_hot[h] = e;
     }
     __syncwarp();
-    if (lane == 0) {
-        for (int h = 0; h < a.num_replicas; ++h) {
-            const int e = s_hot[h];
-            const int home = e / a.M;
-            int best = -1;
-            for (int r = 0; r < a.R; ++r)
-                if (r != home && s_free[r] > 0 && (best < 0 || s_load[r] < s_load[best]))
-                    best = r;
-            if (best < 0)
-                best = home;
-            const int slot = a.S - s_free[best];
-            s_free[best] -= 1;
-            s_repl[e] = best * a.E_loc + a.M + slot;
-            const int64_t moved = s_cnt[e] / 2;
-            s_load[home] -= moved;
-            s_load[best] += moved;
+    // lane owns ranks lane and lane + 32
+    uint32_t load0 = 0, load1 = 0;
+    int free0 = a.S, free1 = a.S;
+    if (lane < a.R)
+        for (int i = 0; i < a.M; ++i)
+            load0 += static_cast<uint32_t>(s_cnt[lane * a.M + i]);
+    if (lane + 32 < a.R)
+        for (int i = 0; i < a.M; ++i)
+            load1 += static_cast<uint32_t>(s_cnt[(lane + 32) * a.M + i]);
+    for (int h = 0; h < a.num_replicas; ++h) {
+        const int e = s_hot[h];
+        const int home = e / a.M;
+        const uint32_t c0 = (lane < a.R && free0 > 0 && lane != home) ? load0 : 0xFFFFFFFFu;
+        const uint32_t c1 = (lane + 32 < a.R && free1 > 0 && lane + 32 != home) ? load1 : 0xFFFFFFFFu;
+        const uint32_t m = __reduce_min_sync(0xffffffffu, min(c0, c1));
+        int best;
+        if (m == 0xFFFFFFFFu) {
+            best = home;
+        } else {
+            const uint32_t r0 = c0 == m ? static_cast<uint32_t>(lane) : 0xFFFFFFFFu;
+            const uint32_t r1 = c1 == m ? static_cast<uint32_t>(lane + 32) : 0xFFFFFFFFu;
+            best = static_cast<int>(__reduce_min_sync(0xffffffffu, min(r0, r1)));
         }
+        const int owner_free = __shfl_sync(0xffffffffu, best < 32 ? free0 : free1, best & 31);
+        const int slot = a.S - owner_free;
+        const uint32_t moved = static_cast<uint32_t>(s_cnt[e]) / 2u;
+        if (lane == (best & 31)) {
+            if (best < 32) {
+                free0 -= 1;
+                load0 += moved;
+            } else {
+                free1 -= 1;
+                load1 += moved;
+            }
+        }
+        if (lane == (home & 31)) {
+            if (home < 32)
+                load0 -= moved;
+            else
+                load1 -= moved;
+        }
+        if (lane == 0)
+            s_repl[e] = best * a.E_loc + a.M + slot;
     }
 }
 
-// Sum of one int32 per thread over the block (all threads must call it).
-__device__ __forceinline__ int32_t layout_block_sum(int32_t v, int32_t *s_scratch)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        v += __shfl_xor_sync(0xffffffffu, v, o);
-    __syncthreads();
-    if (lane == 0)
-        s_scratch[warp] = v;
-    __syncthreads();
-    int32_t total = 0;
-#pragma unroll
-    for (int w = 0; w < LAYOUT_WARPS; ++w)
-        total += s_scratch[w];
-    return total;
-}
-
+template <int IPL> // IPL > 0: each lane keeps IPL assignments in registers (sub = 32 * IPL); 0: any sub
 __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
 {
     extern __shared__ __align__(16) uint32_t layout_smem[];
     const int E_log = a.E_log, E = a.E;
-    uint32_t *wcnt = layout_smem;                                            // [WARPS][E_log]
+    uint32_t *wcnt = layout_smem;                                                // [WARPS][E_log]
     int32_t *s_pre = reinterpret_cast<int32_t *>(wcnt + LAYOUT_WARPS * E_log); // [E_log]
-    int32_t *s_cnt = s_pre + E_log;                                   // [E_log]
-    int32_t *s_repl = s_cnt + E_log;                                  // [E_log]
-    int32_t *s_raw = s_repl + E_log;                                  // [E]
-    int32_t *s_off = s_raw + E;                                       // [E+1]
-    __shared__ int64_t s_load[LAYOUT_MAX_PLACEMENT_RANKS];
-    __shared__ int32_t s_free[LAYOUT_MAX_PLACEMENT_RANKS];
+    int32_t *s_cnt = s_pre + E_log;                                            // [E_log]
+    int32_t *s_repl = s_cnt + E_log;                                           // [E_log]
+    int32_t *s_raw = s_repl + E_log;                                           // [E]
+    int32_t *s_off = s_raw + E;                                                // [E+1]
     __shared__ int32_t s_hot[LAYOUT_MAX_E_LOG];
-    __shared__ int32_t s_scratch[LAYOUT_WARPS];
+    __shared__ int32_t s_part[2][LAYOUT_THREADS];
+    __shared__ int32_t s_wsum[3][LAYOUT_WARPS];
     __shared__ uint32_t s_err;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.x;
+    const uint32_t lt = lanemask_lt();
 
     for (int i = tid; i < LAYOUT_WARPS * E_log; i += LAYOUT_THREADS)
         wcnt[i] = 0;
@@ -205,40 +222,73 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
     __syncthreads();
 
     const int64_t base = (static_cast<int64_t>(b) * LAYOUT_WARPS + warp) * a.sub;
+    uint32_t *my_cnt = wcnt + warp * E_log;
+    pdl_trigger();
+    pdl_wait(); // inputs and the workspace may have been written by the previous kernel
 
-    // ---- phase 1: per-warp histograms
+    // ---- phase 1: load the slice, rank within the warp, per-warp counts
+    constexpr int NR = IPL > 0 ? IPL : 1;
+    int32_t ids[NR];
+    float prs[NR];
+    int32_t wrank[NR]; // rank among earlier assignments of this warp with the same id
     uint32_t err = 0;
-    for (int it = 0; it < a.sub; it += 32) {
-        const int64_t i = base + it + lane;
-        int e = -1;
+    auto load_item = [&](int64_t i, int32_t &e, float &p) {
+        e = -1;
+        p = 0.0f;
         if (i < a.NK) {
             e = __ldg(a.topk_idx + i);
+            if (a.topk_probs != nullptr)
+                p = __ldg(a.topk_probs + i);
             if (e < -1 || e >= E_log) {
                 err |= MOE_DEV_EXPERT_RANGE;
                 e = -1;
             }
         }
+    };
+    // Rank of id e among the earlier items of this warp (counter value before
+    // this round + earlier lanes with the same id); advances the counter.
+    auto rank_item = [&](int32_t e) -> int32_t {
         const uint32_t peers = __match_any_sync(0xffffffffu, e);
+        const uint32_t before = e >= 0 ? my_cnt[e] : 0u;
+        __syncwarp();
         if (e >= 0 && lane == __ffs(peers) - 1)
-            wcnt[warp * E_log + e] += __popc(peers);
+            my_cnt[e] = before + __popc(peers);
         __syncwarp(); // the next update of this counter may come from another lane
+        return static_cast<int32_t>(before + __popc(peers & lt));
+    };
+    if constexpr (IPL > 0) {
+#pragma unroll
+        for (int u = 0; u < IPL; ++u)
+            load_item(base + u * 32 + lane, ids[u], prs[u]);
+#pragma unroll
+        for (int u = 0; u < IPL; ++u)
+            wrank[u] = rank_item(ids[u]);
+    } else {
+        for (int it = 0; it < a.sub; it += 32) {
+            load_item(base + it + lane, ids[0], prs[0]);
+            (void)rank_item(ids[0]);
+        }
     }
     err = __reduce_or_sync(0xffffffffu, err);
     if (lane == 0 && err)
         atomicOr(&s_err, err);
     __syncthreads();
+    // per-warp counts -> exclusive prefix over warps; block total to the workspace
     for (int e = tid; e < E_log; e += LAYOUT_THREADS) {
+        uint32_t c[LAYOUT_WARPS];
+#pragma unroll
+        for (int w = 0; w < LAYOUT_WARPS; ++w)
+            c[w] = wcnt[w * E_log + e];
         uint32_t run = 0;
 #pragma unroll
         for (int w = 0; w < LAYOUT_WARPS; ++w) {
-            const uint32_t c = wcnt[w * E_log + e];
             wcnt[w * E_log + e] = run;
-            run += c;
+            run += c[w];
         }
-        a.ws_counts[static_cast<int64_t>(b) * (E_log + 1) + e] = static_cast<int32_t>(run);
+        a.ws_counts[static_cast<int64_t>(b) * E_log + e] = static_cast<int32_t>(run);
     }
-    if (tid == 0)
-        a.ws_counts[static_cast<int64_t>(b) * (E_log + 1) + E_log] = static_cast<int32_t>(s_err);
+    if (tid == 0 && s_err != 0)
+        atomicOr(a.ws_barrier + 2, s_err);
 
     if (!layout_grid_barrier(a.ws_barrier, static_cast<uint32_t>(a.G) + a.barrier_extra, a.barrier_limit_ns)) {
         if (tid == 0)
@@ -246,32 +296,63 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
         return;
     }
 
-    // ---- phase 2a: block prefix and totals per logical expert
-    for (int e = tid; e < E_log; e += LAYOUT_THREADS) {
-        int32_t pre = 0, tot = 0;
-        for (int bb = 0; bb < a.G; ++bb) {
-            const int32_t c = __ldcg(a.ws_counts + static_cast<int64_t>(bb) * (E_log + 1) + e);
-            pre += bb < b ? c : 0;
-            tot += c;
+    // ---- phase 2a: block prefix and totals per logical expert. P threads
+    // share an expert; each sums every P-th block with all its loads in flight.
+    {
+        const int P = E_log >= LAYOUT_THREADS ? 1 : min(32, LAYOUT_THREADS / E_log);
+        for (int item = tid; item < E_log * P; item += LAYOUT_THREADS) {
+            const int e = item % E_log, part = item / E_log;
+            int32_t pre = 0, tot = 0;
+            for (int bb0 = part; bb0 < a.G; bb0 += 32 * P) {
+                int32_t c[32];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const int bb = bb0 + u * P;
+                    c[u] = bb < a.G ? __ldcg(a.ws_counts + static_cast<int64_t>(bb) * E_log + e) : 0;
+                }
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    tot += c[u];
+                    pre += (bb0 + u * P < b) ? c[u] : 0;
+                }
+            }
+            if (P == 1) {
+                s_pre[e] = pre;
+                s_cnt[e] = tot;
+                s_repl[e] = -1;
+            } else { // E_log * P <= LAYOUT_THREADS: item indexes the scratch in bounds
+                s_part[0][item] = pre;
+                s_part[1][item] = tot;
+            }
         }
-        s_pre[e] = pre;
-        s_cnt[e] = tot;
-        s_repl[e] = -1;
+        if (b == 0 && tid == LAYOUT_THREADS - 1) {
+            // every block OR-ed its error bits in before the barrier; block 0 reports and clears them
+            s_err = __ldcg(a.ws_barrier + 2);
+            a.ws_barrier[2] = 0;
+        }
+        __syncthreads();
+        if (P > 1) {
+            for (int e = tid; e < E_log; e += LAYOUT_THREADS) {
+                int32_t pre = 0, tot = 0;
+                for (int part = 0; part < P; ++part) {
+                    pre += s_part[0][part * E_log + e];
+                    tot += s_part[1][part * E_log + e];
+                }
+                s_pre[e] = pre;
+                s_cnt[e] = tot;
+                s_repl[e] = -1;
+            }
+            __syncthreads();
+        }
     }
-    if (tid == 0) {
-        uint32_t all = 0;
-        for (int bb = 0; bb < a.G; ++bb)
-            all |= static_cast<uint32_t>(__ldcg(a.ws_counts + static_cast<int64_t>(bb) * (E_log + 1) + E_log));
-        s_err = all;
-    }
-    __syncthreads();
 
     // ---- phase 2b: hot experts and placement
-    if (a.num_replicas > 0)
-        layout_placement(a, s_cnt, s_repl, s_load, s_free, s_hot);
-    __syncthreads();
+    if (a.num_replicas > 0) {
+        layout_placement(a, s_cnt, s_repl, s_hot);
+        __syncthreads();
+    }
 
-    // ---- phase 2c: physical counts, scan, splits
+    // ---- phase 2c: physical counts, scan of the rows each expert owns, totals
     for (int q = tid; q < E; q += LAYOUT_THREADS) {
         const int r = q / a.E_loc, i = q - r * a.E_loc;
         int32_t c = 0;
@@ -290,19 +371,21 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
                 s_raw[s_repl[e]] = s_cnt[e] / 2;
         __syncthreads();
     }
-    // exclusive scan of the rows each expert owns (C rows each when capped)
+    int32_t total_valid, total_kept;
     {
         constexpr int PER = 8; // E <= 4096 = LAYOUT_THREADS * PER
         const int q0 = tid * PER;
-        int32_t v[PER];
-        int32_t sum = 0;
+        int32_t rows[PER];
+        int32_t sum = 0, valid = 0, kept = 0;
 #pragma unroll
         for (int u = 0; u < PER; ++u) {
             const int q = q0 + u;
-            v[u] = q < E ? (a.C > 0 ? a.C : s_raw[q]) : 0;
-            sum += v[u];
+            const int32_t raw = q < E ? s_raw[q] : 0;
+            rows[u] = q < E ? (a.C > 0 ? a.C : raw) : 0;
+            sum += rows[u];
+            valid += raw;
+            kept += a.C > 0 ? min(raw, a.C) : raw;
         }
-        // warp inclusive scan of the per-thread sums
         int32_t inc = sum;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -310,31 +393,38 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
             if (lane >= o)
                 inc += n;
         }
-        __shared__ int32_t s_warp_tot[LAYOUT_WARPS];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            valid += __shfl_xor_sync(0xffffffffu, valid, o);
+            kept += __shfl_xor_sync(0xffffffffu, kept, o);
+        }
         if (lane == 31)
-            s_warp_tot[warp] = inc;
+            s_wsum[0][warp] = inc;
+        if (lane == 0) {
+            s_wsum[1][warp] = valid;
+            s_wsum[2][warp] = kept;
+        }
         __syncthreads();
         int32_t wpre = 0;
-        for (int w = 0; w < warp; ++w)
-            wpre += s_warp_tot[w];
+        total_valid = 0;
+        total_kept = 0;
+#pragma unroll
+        for (int w = 0; w < LAYOUT_WARPS; ++w) {
+            wpre += w < warp ? s_wsum[0][w] : 0;
+            total_valid += s_wsum[1][w];
+            total_kept += s_wsum[2][w];
+        }
         int32_t run = wpre + inc - sum;
 #pragma unroll
         for (int u = 0; u < PER; ++u) {
             const int q = q0 + u;
             if (q < E)
                 s_off[q] = run;
-            run += v[u];
+            run += rows[u];
         }
         if (tid == LAYOUT_THREADS - 1)
             s_off[E] = run;
     }
-    int32_t my_valid = 0, my_kept = 0;
-    for (int e = tid; e < E_log; e += LAYOUT_THREADS)
-        my_valid += s_cnt[e];
-    for (int q = tid; q < E; q += LAYOUT_THREADS)
-        my_kept += a.C > 0 ? min(s_raw[q], a.C) : s_raw[q];
-    const int32_t total_valid = layout_block_sum(my_valid, s_scratch);
-    const int32_t total_kept = layout_block_sum(my_kept, s_scratch);
     __syncthreads();
 
     const moe_layout_t &o = a.out;
@@ -371,28 +461,13 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
         }
     }
 
-    // ---- phase 2d: per-assignment pass over this warp's slice
-    const uint32_t lt = lanemask_lt();
-    for (int it = 0; it < a.sub; it += 32) {
-        const int64_t i = base + it + lane;
-        int e = -1;
-        if (i < a.NK) {
-            e = __ldg(a.topk_idx + i);
-            if (e < -1 || e >= E_log)
-                e = -1;
-        }
-        const uint32_t peers = __match_any_sync(0xffffffffu, e);
-        const uint32_t wbase = e >= 0 ? wcnt[warp * E_log + e] : 0u;
-        __syncwarp();
-        if (e >= 0 && lane == __ffs(peers) - 1)
-            wcnt[warp * E_log + e] = wbase + __popc(peers);
-        __syncwarp();
-        if (i >= a.NK)
-            continue;
+    // ---- phase 2d: per-assignment outputs. `in_block` = rank of the assignment
+    // among the earlier ones of its block with the same logical id.
+    auto emit = [&](int64_t i, int32_t e, float p, int32_t in_block) {
         int32_t q = -1, ord = -1, dest = -1;
         uint8_t drop = 0;
         if (e >= 0) {
-            const int32_t lo = s_pre[e] + static_cast<int32_t>(wbase) + __popc(peers & lt);
+            const int32_t lo = s_pre[e] + in_block;
             const int32_t master = (e / a.M) * a.E_loc + (e % a.M);
             const int32_t repl = s_repl[e];
             if (repl >= 0) {
@@ -414,37 +489,73 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
         o.ordinal[i] = ord;
         o.drop_mask[i] = drop;
         o.dest_row[i] = dest;
-        if (dest >= 0) {
-            const int32_t t = static_cast<int32_t>(i / a.k);
+        if (dest >= 0) { // scattered: the rest of the row maps is written row by row below
+            const int32_t t = static_cast<int32_t>(i) / a.k;
             o.row_token[dest] = t;
-            o.row_slot[dest] = static_cast<int32_t>(i - static_cast<int64_t>(t) * a.k);
-            o.row_prob[dest] = a.topk_probs != nullptr ? __ldg(a.topk_probs + i) : 0.0f;
-            o.row_local_expert[dest] = q % a.E_loc;
-            o.pad_mask[dest] = 0;
+            o.row_slot[dest] = static_cast<int32_t>(i) - t * a.k;
+            o.row_prob[dest] = p;
         }
         if (o.local_topk != nullptr) {
             const int owner = dest >= 0 ? q / a.E_loc : -1;
             for (int r = 0; r < a.R; ++r)
                 o.local_topk[static_cast<int64_t>(r) * a.NK + i] = (r == owner) ? q - r * a.E_loc : -1;
         }
+    };
+    if constexpr (IPL > 0) {
+        // wcnt now holds the exclusive prefix over earlier warps and is not modified any more
+#pragma unroll
+        for (int u = 0; u < IPL; ++u) {
+            const int64_t i = base + u * 32 + lane;
+            if (i < a.NK)
+                emit(i, ids[u], prs[u], ids[u] >= 0 ? static_cast<int32_t>(my_cnt[ids[u]]) + wrank[u] : 0);
+        }
+    } else {
+        // slices too long for registers: reload and rank again; the counters now
+        // start from the warp's exclusive prefix, so the rank includes it
+        for (int it = 0; it < a.sub; it += 32) {
+            const int64_t i = base + it + lane;
+            int32_t e;
+            float p;
+            load_item(i, e, p);
+            const int32_t in_block = rank_item(e);
+            if (i < a.NK)
+                emit(i, e, p, in_block);
+        }
     }
 
-    // ---- phase 2e: pad rows (capacity slots left empty) and the tail
+    // ---- phase 2e: per-row outputs that depend on the row index only, written
+    // in row order: the owning expert (capacity slot, or a binary search of the
+    // offsets), pad_mask, the rank-local expert id, and 0 / -1 / 0 in pad rows.
     const int64_t stride = static_cast<int64_t>(a.G) * LAYOUT_THREADS;
-    const int64_t start = a.C > 0 ? 0 : s_off[E];
-    for (int64_t row = start + static_cast<int64_t>(b) * LAYOUT_THREADS + tid; row < a.rows_max; row += stride) {
-        bool pad = true;
+    const int32_t num_rows = s_off[E];
+    for (int64_t row = static_cast<int64_t>(b) * LAYOUT_THREADS + tid; row < a.rows_max; row += stride) {
+        int32_t q;
+        bool pad;
         if (a.C > 0) {
-            const int32_t q = static_cast<int32_t>(row / a.C);
+            q = static_cast<int32_t>(row / a.C);
             const int32_t slot = static_cast<int32_t>(row - static_cast<int64_t>(q) * a.C);
             pad = slot >= min(s_raw[q], a.C);
+        } else if (row >= num_rows) {
+            q = -1;
+            pad = true;
+        } else {
+            int32_t lo = 0, hi = E; // last q with s_off[q] <= row
+            while (hi - lo > 1) {
+                const int32_t mid = (lo + hi) >> 1;
+                if (s_off[mid] <= row)
+                    lo = mid;
+                else
+                    hi = mid;
+            }
+            q = lo;
+            pad = false;
         }
+        o.pad_mask[row] = pad ? 1 : 0;
+        o.row_local_expert[row] = pad ? -1 : q - (q / a.E_loc) * a.E_loc;
         if (pad) {
             o.row_token[row] = -1;
             o.row_slot[row] = -1;
-            o.row_local_expert[row] = -1;
             o.row_prob[row] = 0.0f;
-            o.pad_mask[row] = 1;
         }
     }
 }

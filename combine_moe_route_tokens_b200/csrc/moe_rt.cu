@@ -10,6 +10,7 @@
 
 #include <cstdint>
 #include <cstdio>
+#include <atomic>
 #include <mutex>
 
 #include "moe_rt.h"
@@ -27,6 +28,72 @@ using namespace moert;
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;     // 1 s: every device-side wait gives up after this
 constexpr uint64_t TEST_WAIT_LIMIT_NS = 10000000ull;  // 10 ms for MOE_FLAG_TEST_BARRIER_TIMEOUT
 constexpr size_t WS_BARRIER_BYTES = 256;
+
+using LayoutKernel = void (*)(LayoutArgs);
+
+LayoutKernel layout_kernel_for(int ipl)
+{
+    switch (ipl) {
+    case 1:
+        return layout_kernel<1>;
+    case 2:
+        return layout_kernel<2>;
+    case 4:
+        return layout_kernel<4>;
+    case 8:
+        return layout_kernel<8>;
+    default:
+        return layout_kernel<0>;
+    }
+}
+
+// Programmatic dependent launch is used unless the driver refuses it for a
+// kind of launch; then that kind falls back to ordinary stream order.
+std::atomic<bool> g_pdl_plain{true};
+std::atomic<bool> g_pdl_coop{true};
+
+// Every kernel goes through cudaLaunchKernelEx with programmatic stream
+// serialization, so its launch overlaps the tail of the previous kernel in the
+// stream (each kernel calls pdl_wait() before reading anything); cooperative
+// kernels add the cooperative attribute.
+template <typename... KArgs, typename... Args>
+int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, void *stream, bool cooperative,
+           Args... args)
+{
+    std::atomic<bool> &pdl_ok = cooperative ? g_pdl_coop : g_pdl_plain;
+    cudaLaunchAttribute attrs[2];
+    unsigned n = 0;
+    if (cooperative) {
+        attrs[n].id = cudaLaunchAttributeCooperative;
+        attrs[n].val.cooperative = 1;
+        ++n;
+    }
+    const unsigned n_base = n;
+    if (pdl_ok.load(std::memory_order_relaxed)) {
+        attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attrs[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cfg.attrs = attrs;
+    cfg.numAttrs = n;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    if (e != cudaSuccess && n > n_base) {
+        (void)cudaGetLastError();
+        pdl_ok.store(false, std::memory_order_relaxed);
+        cfg.numAttrs = n_base;
+        e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    }
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
 
 struct DeviceInfo {
     int sms = 0;
@@ -49,22 +116,17 @@ int device_info(DeviceInfo *out)
         if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
             return MOE_ERR_CUDA;
-        cudaError_t e = cudaFuncSetAttribute(layout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             d.smem_optin - 16 * 1024);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     d.smem_optin - 1024);
+        cudaError_t e = cudaSuccess;
+        for (int ipl : {0, 1, 2, 4, 8})
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(layout_kernel_for(ipl), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         d.smem_optin - 16 * 1024);
         if (e != cudaSuccess)
             return MOE_ERR_CUDA;
         d.ready = true;
     }
     *out = d;
     return MOE_OK;
-}
-
-int launch_status()
-{
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -123,27 +185,38 @@ int check_layout(const moe_layout_t *l, const Dims &d, bool need_rows)
 }
 
 struct LayoutGrid {
-    int32_t G;
-    int32_t sub;
+    int32_t G;   // blocks
+    int32_t sub; // assignments per warp slice
+    int32_t ipl; // assignments per lane kept in registers (1, 2, 4, 8), or 0 for longer slices
 };
 
+// About LAYOUT_ITEMS_PER_BLOCK assignments per block, at most LAYOUT_MAX_BLOCKS
+// blocks; slices of up to 8 items per lane stay in registers.
 LayoutGrid layout_grid(int64_t NK)
 {
     int64_t G = (NK + LAYOUT_ITEMS_PER_BLOCK - 1) / LAYOUT_ITEMS_PER_BLOCK;
     G = G < 1 ? 1 : (G > LAYOUT_MAX_BLOCKS ? LAYOUT_MAX_BLOCKS : G);
-    int64_t sub = (NK + G * LAYOUT_WARPS - 1) / (G * LAYOUT_WARPS);
-    sub = ((sub + 31) / 32) * 32;
-    if (sub < 32)
-        sub = 32;
+    int64_t ipl = (NK + G * LAYOUT_THREADS - 1) / (G * LAYOUT_THREADS);
+    if (ipl < 1)
+        ipl = 1;
+    int32_t kind = 0;
+    if (ipl <= LAYOUT_MAX_IPL) {
+        int64_t p2 = 1;
+        while (p2 < ipl)
+            p2 <<= 1;
+        ipl = p2;
+        kind = static_cast<int32_t>(ipl);
+    }
+    const int64_t sub = 32 * ipl;
     G = (NK + LAYOUT_WARPS * sub - 1) / (LAYOUT_WARPS * sub);
     if (G < 1)
         G = 1;
-    return {static_cast<int32_t>(G), static_cast<int32_t>(sub)};
+    return {static_cast<int32_t>(G), static_cast<int32_t>(sub), kind};
 }
 
 size_t layout_workspace_bytes(int32_t E_log)
 {
-    return WS_BARRIER_BYTES + static_cast<size_t>(LAYOUT_MAX_BLOCKS) * (static_cast<size_t>(E_log) + 1) * 4;
+    return WS_BARRIER_BYTES + static_cast<size_t>(LAYOUT_MAX_BLOCKS) * static_cast<size_t>(E_log) * 4;
 }
 
 } // namespace
@@ -206,25 +279,25 @@ int moe_route_topk(const float *logits, const uint8_t *token_mask, int64_t N, in
         return MOE_ERR_INVALID;
     if (N > (int64_t(1) << 40))
         return MOE_ERR_INVALID;
-    const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t blocks64 = (N + ROUTE_WARPS_PER_BLOCK - 1) / ROUTE_WARPS_PER_BLOCK;
     if (blocks64 > INT32_MAX)
         return MOE_ERR_UNSUPPORTED;
     const dim3 grid(static_cast<unsigned>(blocks64)), block(ROUTE_WARPS_PER_BLOCK * 32);
     const int vpl = (E + 31) / 32;
+    auto go = [&](auto kernel) {
+        return launch(kernel, grid, block, 0, stream, false, logits, token_mask, N, E, k, topk_idx, topk_probs);
+    };
     if (vpl <= 1)
-        route_topk_kernel<1><<<grid, block, 0, s>>>(logits, token_mask, N, E, k, topk_idx, topk_probs);
-    else if (vpl <= 2)
-        route_topk_kernel<2><<<grid, block, 0, s>>>(logits, token_mask, N, E, k, topk_idx, topk_probs);
-    else if (vpl <= 4)
-        route_topk_kernel<4><<<grid, block, 0, s>>>(logits, token_mask, N, E, k, topk_idx, topk_probs);
-    else if (vpl <= 8)
-        route_topk_kernel<8><<<grid, block, 0, s>>>(logits, token_mask, N, E, k, topk_idx, topk_probs);
-    else if (vpl <= 16)
-        route_topk_kernel<16><<<grid, block, 0, s>>>(logits, token_mask, N, E, k, topk_idx, topk_probs);
-    else
-        route_topk_kernel<32><<<grid, block, 0, s>>>(logits, token_mask, N, E, k, topk_idx, topk_probs);
-    return launch_status();
+        return go(route_topk_kernel<1>);
+    if (vpl <= 2)
+        return go(route_topk_kernel<2>);
+    if (vpl <= 4)
+        return go(route_topk_kernel<4>);
+    if (vpl <= 8)
+        return go(route_topk_kernel<8>);
+    if (vpl <= 16)
+        return go(route_topk_kernel<16>);
+    return go(route_topk_kernel<32>);
 }
 
 int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, const float *topk_probs,
@@ -282,15 +355,7 @@ int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, c
     a.barrier_extra = test_timeout ? 1u : 0u;
     a.out = *l;
 
-    void *args[] = {&a};
-    const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(layout_kernel), dim3(lg.G),
-                                                      dim3(LAYOUT_THREADS), args, smem,
-                                                      static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) {
-        (void)cudaGetLastError();
-        return MOE_ERR_CUDA;
-    }
-    return MOE_OK;
+    return launch(layout_kernel_for(lg.ipl), dim3(lg.G), dim3(LAYOUT_THREADS), smem, stream, true, a);
 }
 
 int moe_permute(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *hidden, uint16_t *send,
@@ -312,34 +377,25 @@ int moe_permute(const moe_problem_t *problem, const moe_layout_t *layout, const 
         return rc;
 
     PermuteArgs a;
-    a.hidden = reinterpret_cast<const uint8_t *>(hidden);
-    a.send = reinterpret_cast<uint8_t *>(send);
+    a.hidden = reinterpret_cast<const uint4 *>(hidden);
+    a.send = reinterpret_cast<uint4 *>(send);
     a.dest_row = layout->dest_row;
     a.pad_mask = layout->pad_mask;
     a.status = layout->status;
     a.N = problem->N;
     a.rows_max = d.rows_max;
     a.k = problem->k;
-    a.row_bytes = static_cast<uint32_t>(problem->H) * 2u;
-    a.seg_bytes = a.row_bytes < PERMUTE_SEG_BYTES ? a.row_bytes : PERMUTE_SEG_BYTES;
-    a.nseg = static_cast<int32_t>((a.row_bytes + a.seg_bytes - 1) / a.seg_bytes);
-    a.stages = PERMUTE_MAX_STAGES;
-    a.wait_limit_ns = WAIT_LIMIT_NS;
-    const size_t smem = static_cast<size_t>(a.stages) * a.seg_bytes;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, permute_kernel, 32, smem) != cudaSuccess ||
-        per_sm < 1)
-        return MOE_ERR_CUDA;
-    const int64_t units = problem->N * a.nseg;
-    int64_t grid = static_cast<int64_t>(dev.sms) * per_sm;
-    const int64_t want = units > 0 ? units : 1;
-    if (grid > want)
-        grid = want;
-    // the pad-row pass uses the same CTAs; keep at least a full wave for it
-    if (units < static_cast<int64_t>(dev.sms) * per_sm && d.rows_max > units)
-        grid = static_cast<int64_t>(dev.sms) * per_sm;
-    permute_kernel<<<static_cast<unsigned>(grid), 32, smem, static_cast<cudaStream_t>(stream)>>>(a);
-    return launch_status();
+    a.V = problem->H / 8;
+    a.group = a.V <= 32 * PERMUTE_CHUNKS ? 32 : (a.V <= 64 * PERMUTE_CHUNKS ? 64 : PERMUTE_THREADS);
+    a.pieces = (a.V + a.group * PERMUTE_CHUNKS - 1) / (a.group * PERMUTE_CHUNKS);
+    // pad-row workers: one warp checks 32 rows per pass, at most four CTAs per SM
+    const int64_t zb = (d.rows_max + PERMUTE_THREADS - 1) / PERMUTE_THREADS;
+    a.zero_blocks = static_cast<int32_t>(zb < 4 * dev.sms ? zb : 4 * dev.sms);
+    const int64_t groups = PERMUTE_THREADS / a.group;
+    const int64_t blocks = a.zero_blocks + (problem->N * a.pieces + groups - 1) / groups;
+    if (blocks > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    return launch(permute_kernel, dim3(static_cast<unsigned>(blocks)), dim3(PERMUTE_THREADS), 0, stream, false, a);
 }
 
 namespace {
@@ -367,34 +423,28 @@ int launch_combine(const moe_problem_t *problem, const moe_layout_t *layout, con
     a.rows_max = d.rows_max;
     a.k = problem->k;
     a.V = problem->H / 8;
-    const int threads = a.V >= COMBINE_THREADS ? COMBINE_THREADS : ((a.V + 31) / 32) * 32;
+    // the widest CTA (up to 256 threads) that splits the row into equal parts
+    const int v32 = ((a.V + 31) / 32) * 32;
+    const int threads = v32 % 256 == 0 ? 256 : (v32 % 128 == 0 ? 128 : (v32 % 64 == 0 ? 64 : 32));
     a.nchunks = (a.V + threads - 1) / threads;
     const int64_t blocks = problem->N * a.nchunks;
     if (blocks > INT32_MAX)
         return MOE_ERR_UNSUPPORTED;
-    const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const dim3 grid(static_cast<unsigned>(blocks)), block(threads);
     switch (problem->k) {
     case 1:
-        combine_kernel<1><<<grid, block, 0, s>>>(a);
-        break;
+        return launch(combine_kernel<1>, grid, block, 0, stream, false, a);
     case 2:
-        combine_kernel<2><<<grid, block, 0, s>>>(a);
-        break;
+        return launch(combine_kernel<2>, grid, block, 0, stream, false, a);
     case 4:
-        combine_kernel<4><<<grid, block, 0, s>>>(a);
-        break;
+        return launch(combine_kernel<4>, grid, block, 0, stream, false, a);
     case 6:
-        combine_kernel<6><<<grid, block, 0, s>>>(a);
-        break;
+        return launch(combine_kernel<6>, grid, block, 0, stream, false, a);
     case 8:
-        combine_kernel<8><<<grid, block, 0, s>>>(a);
-        break;
+        return launch(combine_kernel<8>, grid, block, 0, stream, false, a);
     default:
-        combine_kernel<0><<<grid, block, 0, s>>>(a);
-        break;
+        return launch(combine_kernel<0>, grid, block, 0, stream, false, a);
     }
-    return launch_status();
 }
 
 } // namespace
@@ -451,29 +501,21 @@ int moe_combine_backward(const moe_problem_t *problem, const moe_layout_t *layou
     const int64_t blocks = problem->N + a.zero_blocks;
     if (blocks > INT32_MAX)
         return MOE_ERR_UNSUPPORTED;
-    const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const dim3 grid(static_cast<unsigned>(blocks)), block(COMBINE_BWD_THREADS);
     switch (problem->k) {
     case 1:
-        combine_backward_kernel<1><<<grid, block, 0, s>>>(a);
-        break;
+        return launch(combine_backward_kernel<1>, grid, block, 0, stream, false, a);
     case 2:
-        combine_backward_kernel<2><<<grid, block, 0, s>>>(a);
-        break;
+        return launch(combine_backward_kernel<2>, grid, block, 0, stream, false, a);
     case 4:
-        combine_backward_kernel<4><<<grid, block, 0, s>>>(a);
-        break;
+        return launch(combine_backward_kernel<4>, grid, block, 0, stream, false, a);
     case 6:
-        combine_backward_kernel<6><<<grid, block, 0, s>>>(a);
-        break;
+        return launch(combine_backward_kernel<6>, grid, block, 0, stream, false, a);
     case 8:
-        combine_backward_kernel<8><<<grid, block, 0, s>>>(a);
-        break;
+        return launch(combine_backward_kernel<8>, grid, block, 0, stream, false, a);
     default:
-        combine_backward_kernel<0><<<grid, block, 0, s>>>(a);
-        break;
+        return launch(combine_backward_kernel<0>, grid, block, 0, stream, false, a);
     }
-    return launch_status();
 }
 
 } // extern "C"

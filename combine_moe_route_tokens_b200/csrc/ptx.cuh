@@ -1,16 +1,11 @@
-// ptx.cuh — thin inline-PTX wrappers for sm_100a: mbarriers, bulk (TMA)
-// copies between global and shared memory, cache-hinted vector loads and the
-// global timer used to bound every device-side wait.
+// ptx.cuh — thin inline-PTX wrappers for sm_100a: programmatic dependent
+// launch, cache-hinted vector loads, bf16 packing and the global timer used to
+// bound every device-side wait.
 #pragma once
 
 #include <cstdint>
 
 namespace moert {
-
-__device__ __forceinline__ uint32_t smem_addr(const void *p)
-{
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
 
 __device__ __forceinline__ uint64_t global_timer_ns()
 {
@@ -19,98 +14,22 @@ __device__ __forceinline__ uint64_t global_timer_ns()
     return t;
 }
 
-// ---------------------------------------------------------------- mbarrier --
+// --------------------------------------------- programmatic dependent launch --
+// A kernel launched with programmatic stream serialization may start before
+// the previous kernel in the stream has finished. pdl_wait() blocks until that
+// kernel has completed and its memory is visible; every kernel here calls it
+// before its first read of data a predecessor may have written (without the
+// launch attribute it returns at once). pdl_trigger() lets the next kernel in
+// the stream be launched once every CTA of this one has started.
 
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t arrivals)
+__device__ __forceinline__ void pdl_wait()
 {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(arrivals) : "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-// Makes barrier initialisation visible to the async proxy (the TMA unit).
-__device__ __forceinline__ void fence_mbar_init()
+__device__ __forceinline__ void pdl_trigger()
 {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
-{
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    return done != 0;
-}
-
-// Waits for the barrier phase with the given parity; gives up after
-// `limit_ns` and returns false.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t limit_ns)
-{
-    if (mbar_try_wait(bar, parity))
-        return true;
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > limit_ns)
-            return false;
-    }
-    return true;
-}
-
-// ------------------------------------------------------ bulk (TMA) copies --
-// Non-tensor bulk copies: both addresses 16-byte aligned, size a multiple of 16.
-
-// global -> shared, completion counted in bytes on `bar`.
-__device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gmem_src, uint32_t bytes, uint64_t *bar,
-                                         uint64_t policy)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
-            smem_addr(smem_dst)),
-        "l"(gmem_src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
-        : "memory");
-}
-
-// shared -> global, tracked by the issuing thread's bulk groups.
-__device__ __forceinline__ void bulk_s2g(void *gmem_dst, const void *smem_src, uint32_t bytes)
-{
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem_dst),
-                 "r"(smem_addr(smem_src)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit()
-{
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// At most N committed groups may still be reading shared memory.
-template <int N>
-__device__ __forceinline__ void bulk_wait_read()
-{
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-
-// Every committed group has completed (writes performed).
-__device__ __forceinline__ void bulk_wait_all()
-{
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
-// L2 eviction-priority policies for cache-hinted copies.
-__device__ __forceinline__ uint64_t policy_evict_first()
-{
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ------------------------------------------------------------ vector I/O ----

@@ -96,7 +96,7 @@ def test_unsupported_problems(lib, kw):
 
 def test_workspace_size(lib):
     p = moe.Problem(N=4096, H=7168, k=8, E_log=256, R=4)
-    assert p.workspace_bytes == 256 + 128 * 257 * 4
+    assert p.workspace_bytes == 256 + 128 * 256 * 4
 
 
 def test_layout_requires_outputs_and_workspace(lib):

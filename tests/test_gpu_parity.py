@@ -176,8 +176,10 @@ EDGE_CASES = [
     (4099, 136, 8, 128, 8, 0, 8, 0.0, 1.2),  # reroute, ragged block tail
     (2048, 64, 4, 32, 2, 40, 4, 0.1, 1.4),  # reroute + capacity
     (777, 16, 8, 2048, 1, 0, 0, 0.0, None),  # widest router supported
-    (300, 20000, 2, 8, 2, 0, 0, 0.0, None),  # row of 40000 B: two TMA segments
+    (300, 20000, 2, 8, 2, 0, 0, 0.0, None),  # row of 40000 B: three 16 KB pieces, the last ragged
     (70000, 8, 1, 4, 2, 0, 0, 0.0, None),  # many blocks, tiny rows
+    (36000, 8, 8, 256, 8, 0, 8, 0.0, 1.2),  # 288k assignments: 8 per lane in registers, reroute
+    (75000, 8, 8, 64, 4, 0, 0, 0.05, 1.2),  # 600k assignments: slices too long for registers
 ]
 
 
@@ -317,3 +319,26 @@ def test_streams_are_respected():
     s.synchronize()
     exp_send = oracle.permute(d["hidden"], L["dest_row"], L["rows_max"])
     assert np.array_equal(host(out), oracle.combine(exp_send, L["dest_row"], probs))
+
+
+ROUTE_CASES = [(5, 5), (8, 1), (33, 7), (100, 8), (256, 8), (256, 32), (600, 12), (1000, 2), (1024, 32)]
+
+
+@pytest.mark.parametrize("E,k", ROUTE_CASES, ids=[f"E{e}_k{k}" for e, k in ROUTE_CASES])
+@pytest.mark.parametrize("kind", ["normal", "ties", "signed_zero"])
+def test_route_edge_cases(E, k, kind):
+    rng = np.random.default_rng(E * 100 + k)
+    N = 257
+    if kind == "normal":
+        logits = (rng.standard_normal((N, E)) * 4).astype(np.float32)
+    elif kind == "ties":
+        logits = rng.integers(-2, 3, size=(N, E)).astype(np.float32)
+    else:
+        logits = np.where(rng.random((N, E)) < 0.5, np.float32(0.0), np.float32(-0.0)).astype(np.float32)
+        logits[:, ::7] = 0.5
+    gi, gp = moe.moe_route_topk(dev(logits), k)
+    idx, probs = oracle.route_topk(logits, k)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(gi), idx)
+    tol = route_prob_tolerance(logits, idx) * probs.astype(np.float64)
+    assert np.all(np.abs(host(gp).astype(np.float64) - probs.astype(np.float64)) <= tol)
