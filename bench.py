@@ -54,6 +54,23 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """The maximum of a per-rank value over all ranks (the value itself without a process group)."""
+    import torch
+    import torch.distributed as tdist
+
+    if not (tdist.is_available() and tdist.is_initialized()) or tdist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_inputs(w, rank: int) -> dict:
+    """Each data-parallel rank processes its own batch: the workload's recipe with seed + rank."""
+    return make_inputs(w, grad=w.backward, seed_offset=rank)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -253,7 +270,7 @@ def run_ours(args, ws, rank, local):
     moe.load_library()
 
     w = get_workload(args.workload)
-    host = make_inputs(w, grad=w.backward, seed_offset=rank)
+    host = rank_inputs(w, rank)
     set_bytes = sum(v.nbytes for v in host.values())
     nsets = max(2, min(8, math.ceil(2 * L2_BYTES / set_bytes)))
     # one generated batch; the other sets are token-rotated copies of it (same distribution,
@@ -315,10 +332,7 @@ def run_ours(args, ws, rank, local):
     status = step.layout.status()
     if status != 0:
         raise RuntimeError(f"device status {status:#x} after the timed steps")
-    if ws > 1:
-        t = torch.tensor([elapsed_ms], device=device, dtype=torch.float64)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, device)
 
     # end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
@@ -350,11 +364,7 @@ def run_ours(args, ws, rank, local):
         e1.record(step.stream)
         torch.cuda.synchronize()
         barrier()
-        e_ms = e0.elapsed_time(e1)
-        if ws > 1:
-            t = torch.tensor([e_ms], device=device, dtype=torch.float64)
-            tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e0.elapsed_time(e1), device)
         e2e = {
             "value": w.N * args.steps * ws / (e_ms / 1e3),
             "unit": "tokens/s",
