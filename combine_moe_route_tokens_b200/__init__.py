@@ -51,6 +51,7 @@ __all__ = [
     "MoeError",
     "moe_route_topk",
     "moe_dispatch_layout",
+    "moe_dispatch_layout_noalloc",
     "moe_permute",
     "moe_combine",
     "moe_permute_backward",
@@ -252,6 +253,29 @@ def moe_dispatch_layout(problem: Problem, topk_idx: torch.Tensor, topk_probs: Op
     rc = _native.lib().moe_dispatch_layout(ctypes.byref(p), _ptr(topk_idx), _ptr(topk_probs), ctypes.byref(L),
                                            _ptr(layout.workspace), layout.workspace.numel(), _stream(stream))
     _native.check("moe_dispatch_layout", rc)
+    return layout
+
+
+def moe_dispatch_layout_noalloc(problem: Problem, topk_idx: torch.Tensor, topk_probs: Optional[torch.Tensor],
+                                layout: Layout, stream=None) -> Layout:
+    """moe_dispatch_layout for callers that cannot allocate device scratch.
+
+    The library keeps the scratch in a fixed device array (E_log up to
+    MOE_NOALLOC_MAX_E_LOG); ``layout.workspace`` is not used. Calls share that
+    array, so calls running at the same time on different streams race; keep
+    them on one stream. The first call on a device must not happen during
+    stream capture.
+    """
+    _need(topk_idx, "topk_idx", torch.int32, (problem.N, problem.k))
+    if topk_probs is not None:
+        _need(topk_probs, "topk_probs", torch.float32, (problem.N, problem.k), topk_idx.device)
+    if layout.problem != problem:
+        raise ValueError("layout was allocated for a different problem")
+    p = problem.c_struct()
+    L = layout.c_struct()
+    rc = _native.lib().moe_dispatch_layout_noalloc(ctypes.byref(p), _ptr(topk_idx), _ptr(topk_probs),
+                                                   ctypes.byref(L), _stream(stream))
+    _native.check("moe_dispatch_layout_noalloc", rc)
     return layout
 
 

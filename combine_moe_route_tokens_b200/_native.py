@@ -21,6 +21,8 @@ MOE_OK = 0
 MOE_ERR_INVALID = -1
 MOE_ERR_UNSUPPORTED = -2
 MOE_ERR_CUDA = -3
+MOE_ERR_SCRATCH_LIMIT = -4
+MOE_NOALLOC_MAX_E_LOG = 512
 
 MOE_DEV_EXPERT_RANGE = 0x1
 MOE_DEV_TIMEOUT = 0x2
@@ -93,6 +95,7 @@ _SIGNATURES = {
     "moe_layout_workspace_bytes": (ctypes.c_int, [_PP, ctypes.POINTER(ctypes.c_size_t)]),
     "moe_route_topk": (ctypes.c_int, [_VP, _VP, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _VP, _VP, _VP]),
     "moe_dispatch_layout": (ctypes.c_int, [_PP, _VP, _VP, _PL, _VP, ctypes.c_size_t, _VP]),
+    "moe_dispatch_layout_noalloc": (ctypes.c_int, [_PP, _VP, _VP, _PL, _VP]),
     "moe_permute": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP]),
     "moe_combine": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP]),
     "moe_permute_backward": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP]),

@@ -236,6 +236,8 @@ const char *moe_status_string(int code)
         return "valid problem beyond the kernels' limits";
     case MOE_ERR_CUDA:
         return "CUDA runtime call or kernel launch failed";
+    case MOE_ERR_SCRATCH_LIMIT:
+        return "problem needs more scratch than the library's fixed array holds (E_log above MOE_NOALLOC_MAX_E_LOG)";
     case static_cast<int>(MOE_DEV_EXPERT_RANGE):
         return "device: expert id outside [-1, E_log) skipped";
     case static_cast<int>(MOE_DEV_TIMEOUT):
@@ -519,3 +521,88 @@ int moe_combine_backward(const moe_problem_t *problem, const moe_layout_t *layou
 }
 
 } // extern "C"
+
+// ------------------------------------------------ layout without allocation --
+// moe_dispatch_layout_noalloc: the same layout, with its scratch in a
+// fixed device array of this library instead of a caller-provided workspace,
+// for callers that cannot allocate device memory.
+
+namespace {
+
+static_assert(MOE_NOALLOC_SCRATCH_BYTES ==
+                  WS_BARRIER_BYTES + static_cast<size_t>(LAYOUT_MAX_BLOCKS) * MOE_NOALLOC_MAX_E_LOG * 4,
+              "fixed scratch must hold the barrier words and LAYOUT_MAX_BLOCKS rows of per-expert counts");
+
+// Held by every device that loads the library, for the life of the process.
+static __device__ __align__(256) unsigned char g_layout_scratch[MOE_NOALLOC_SCRATCH_BYTES];
+
+struct ScratchAddress {
+    void *ptr = nullptr;
+    bool ready = false;
+};
+ScratchAddress g_scratch_address[MAX_DEVICES];
+std::mutex g_scratch_mutex;
+
+// Device address of g_layout_scratch on the current device, looked up once per
+// device (in host code the symbol is only a stand-in, not a device address).
+int scratch_address(void **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES)
+        return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    ScratchAddress &s = g_scratch_address[dev];
+    if (!s.ready) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_layout_scratch) != cudaSuccess || p == nullptr) {
+            (void)cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+        s.ptr = p;
+        s.ready = true;
+    }
+    *out = s.ptr;
+    return MOE_OK;
+}
+
+} // namespace
+
+extern "C" int moe_dispatch_layout_noalloc(const moe_problem_t *problem, const int32_t *topk_idx,
+                                           const float *topk_probs, const moe_layout_t *layout, void *stream)
+{
+    Dims d;
+    int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    if (problem->E_log > MOE_NOALLOC_MAX_E_LOG)
+        return MOE_ERR_SCRATCH_LIMIT;
+    // the argument checks of moe_dispatch_layout, made before anything is enqueued here
+    const moe_layout_t *l = layout;
+    if (l == nullptr || l->status == nullptr || l->counts_logical == nullptr || l->placement == nullptr ||
+        l->counts_raw == nullptr || l->tokens_per_expert == nullptr || l->expert_offsets == nullptr ||
+        l->input_splits == nullptr || l->output_splits == nullptr || l->rank_offsets == nullptr ||
+        l->counters == nullptr || l->num_rows == nullptr)
+        return MOE_ERR_INVALID;
+    if (d.NK > 0 && (topk_idx == nullptr || l->phys_idx == nullptr || l->ordinal == nullptr ||
+                     l->dest_row == nullptr || l->drop_mask == nullptr))
+        return MOE_ERR_INVALID;
+    if (d.rows_max > 0 && (l->row_token == nullptr || l->row_slot == nullptr || l->row_local_expert == nullptr ||
+                           l->row_prob == nullptr || l->pad_mask == nullptr))
+        return MOE_ERR_INVALID;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev)) != MOE_OK)
+        return rc;
+    if (layout_grid(d.NK).G > dev.sms)
+        return MOE_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    if ((rc = scratch_address(&scratch)) != MOE_OK)
+        return rc;
+    // The grid barrier's arrival count and the error word must start at zero; a
+    // previous call that timed out may have left them set. The per-block counts
+    // are rewritten by every call before they are read.
+    if (cudaMemsetAsync(scratch, 0, WS_BARRIER_BYTES, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    return moe_dispatch_layout(problem, topk_idx, topk_probs, layout, scratch, MOE_NOALLOC_SCRATCH_BYTES, stream);
+}

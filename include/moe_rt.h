@@ -56,6 +56,7 @@ extern "C" {
 #define MOE_ERR_INVALID (-1)     /* bad size, NULL required pointer, misaligned buffer, inconsistent problem */
 #define MOE_ERR_UNSUPPORTED (-2) /* valid but beyond the kernels' limits (see each call) */
 #define MOE_ERR_CUDA (-3)        /* a CUDA runtime call or launch failed */
+#define MOE_ERR_SCRATCH_LIMIT (-4) /* moe_dispatch_layout_noalloc: E_log above MOE_NOALLOC_MAX_E_LOG */
 
 /* Device-detected status bits, OR-ed into *layout->status. */
 #define MOE_DEV_EXPERT_RANGE 0x1u /* a topk id outside [-1, E_log): the entry was skipped as if -1 */
@@ -181,6 +182,36 @@ MOE_API int moe_route_topk(const float *logits, const uint8_t *token_mask, int64
  */
 MOE_API int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, const float *topk_probs,
                         const moe_layout_t *layout, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Dispatch layout for callers that cannot allocate device memory. The pages
+ * have no counterpart of this entry point; it exists for the library's users.
+ *
+ * Some callers have no way to obtain device scratch: a C or Fortran host
+ * program without an allocator of its own, a plugin running inside a host
+ * application that owns every allocation, or a hot loop that must not touch
+ * cudaMalloc (it can synchronise the device and fail under memory pressure).
+ * This call computes exactly what moe_dispatch_layout computes, with the same
+ * arguments except the workspace: its scratch is a fixed array inside the
+ * library, MOE_NOALLOC_SCRATCH_BYTES bytes that every GPU which loads the
+ * library keeps until the process exits. It calls no allocator.
+ *
+ * Limits and rules:
+ *  - E_log <= MOE_NOALLOC_MAX_E_LOG, else MOE_ERR_SCRATCH_LIMIT and nothing is enqueued;
+ *    every other argument rule of moe_dispatch_layout applies.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current). Make that first call before any stream
+ *    capture begins.
+ *  - All calls share the one array and it keeps what the last call left there.
+ *    Each call first clears, in stream order, the words that must start at zero,
+ *    so a call that ran out of time (MOE_DEV_TIMEOUT) does not affect the next.
+ *    Calls whose executions overlap on the GPU (for example on two streams)
+ *    race on the array and give wrong results: order them on one stream.
+ */
+#define MOE_NOALLOC_MAX_E_LOG 512
+#define MOE_NOALLOC_SCRATCH_BYTES (256 + 128 * MOE_NOALLOC_MAX_E_LOG * 4)
+MOE_API int moe_dispatch_layout_noalloc(const moe_problem_t *problem, const int32_t *topk_idx,
+                                        const float *topk_probs, const moe_layout_t *layout, void *stream);
 
 /*
  * Permute ([Megatron MoE] dispatch_postprocess; [Megatron MORI] permute fused
