@@ -184,7 +184,7 @@ class Step:
         self.torch = torch
         self.lib = native.lib()
         p = moe.Problem(N=w.N, H=w.H, k=w.k, E_log=w.E_log, R=w.R, capacity=w.capacity,
-                        num_replicas=w.num_replicas)
+                        num_replicas=w.num_replicas, row_align=w.row_align)
         self.problem = p
         self.layout = moe.Layout.allocate(p, device)
         self.sets = sets
@@ -442,7 +442,7 @@ def oracle_step(oracle, w, d):
     """The whole path on the CPU oracle for the batch in ``d``."""
     idx, probs = oracle.route_topk(d["logits"], w.k)
     L = oracle.layout(idx, probs, E_log=w.E_log, R=w.R, C=w.capacity, num_replicas=w.num_replicas,
-                      local_topk=True)
+                      align=w.row_align, local_topk=True)
     send = oracle.permute(d["hidden"], L["dest_row"], L["rows_max"])
     out = oracle.combine(send, L["dest_row"], probs)
     if w.backward:

@@ -83,6 +83,7 @@ class Problem:
     capacity: int = 0
     num_replicas: int = 0
     flags: int = MOE_FLAG_NONE
+    row_align: int = 0
 
     @property
     def E(self) -> int:
@@ -102,6 +103,7 @@ class Problem:
             R=self.R,
             capacity=self.capacity,
             flags=self.flags,
+            row_align=self.row_align,
         )
 
     @property

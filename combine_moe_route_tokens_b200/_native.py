@@ -31,7 +31,7 @@ MOE_DEV_ROW_RANGE = 0x4
 MOE_FLAG_NONE = 0
 MOE_FLAG_TEST_BARRIER_TIMEOUT = 0x80000000
 
-ABI_VERSION = 1
+ABI_VERSION = 2
 
 
 class MoeProblem(ctypes.Structure):
@@ -44,6 +44,7 @@ class MoeProblem(ctypes.Structure):
         ("R", ctypes.c_int32),
         ("capacity", ctypes.c_int32),
         ("flags", ctypes.c_uint32),
+        ("row_align", ctypes.c_int32),
     ]
 
 

@@ -47,6 +47,7 @@ struct LayoutArgs {
     int64_t NK;
     int64_t rows_max;
     int32_t k, E_log, E, R, E_loc, M, S, num_replicas, C;
+    int32_t A; // row alignment (1 = none)
     int32_t sub; // assignments per warp slice, a multiple of 32
     int32_t G;   // blocks
     int32_t *ws_counts;   // [G][E_log]: per-block logical totals
@@ -352,7 +353,8 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
         __syncthreads();
     }
 
-    // ---- phase 2c: physical counts, scan of the rows each expert owns, totals
+    // ---- phase 2c: physical counts, scan of the rows each expert owns (C, or its
+    // count rounded up to the row alignment), totals
     for (int q = tid; q < E; q += LAYOUT_THREADS) {
         const int r = q / a.E_loc, i = q - r * a.E_loc;
         int32_t c = 0;
@@ -381,7 +383,7 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
         for (int u = 0; u < PER; ++u) {
             const int q = q0 + u;
             const int32_t raw = q < E ? s_raw[q] : 0;
-            rows[u] = q < E ? (a.C > 0 ? a.C : raw) : 0;
+            rows[u] = q < E ? (a.C > 0 ? a.C : ((raw + a.A - 1) / a.A) * a.A) : 0;
             sum += rows[u];
             valid += raw;
             kept += a.C > 0 ? min(raw, a.C) : raw;
@@ -548,7 +550,7 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
                     hi = mid;
             }
             q = lo;
-            pad = false;
+            pad = row - s_off[q] >= s_raw[q]; // alignment pad after the expert's tokens
         }
         o.pad_mask[row] = pad ? 1 : 0;
         o.row_local_expert[row] = pad ? -1 : q - (q / a.E_loc) * a.E_loc;

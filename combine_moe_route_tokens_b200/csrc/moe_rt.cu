@@ -136,6 +136,7 @@ struct Dims {
     int64_t NK = 0;
     int64_t rows_max = 0;
     int32_t E = 0, E_loc = 0, M = 0, S = 0;
+    int32_t A = 1; // row alignment
 };
 
 int check_problem(const moe_problem_t *p, Dims *d)
@@ -149,11 +150,16 @@ int check_problem(const moe_problem_t *p, Dims *d)
         return MOE_ERR_INVALID;
     if ((p->flags & ~MOE_FLAG_TEST_BARRIER_TIMEOUT) != 0)
         return MOE_ERR_INVALID;
+    if (p->row_align < 0)
+        return MOE_ERR_INVALID;
+    const int64_t A = p->row_align > 1 ? p->row_align : 1;
+    if (p->capacity > 0 && p->capacity % A != 0)
+        return MOE_ERR_INVALID;
     const int64_t NK = p->N * static_cast<int64_t>(p->k);
     if (p->N > (int64_t(1) << 40) || NK > INT32_MAX)
         return MOE_ERR_INVALID;
     const int64_t E = static_cast<int64_t>(p->E_log) + p->num_replicas;
-    const int64_t rows_max = p->capacity > 0 ? E * p->capacity : NK;
+    const int64_t rows_max = p->capacity > 0 ? E * p->capacity : NK + E * (A - 1);
     if (rows_max > INT32_MAX)
         return MOE_ERR_INVALID;
     if (p->k > COMBINE_MAX_K || p->E_log > LAYOUT_MAX_E_LOG)
@@ -168,6 +174,7 @@ int check_problem(const moe_problem_t *p, Dims *d)
     d->E_loc = static_cast<int32_t>(E / p->R);
     d->M = p->E_log / p->R;
     d->S = p->num_replicas / p->R;
+    d->A = static_cast<int32_t>(A);
     return MOE_OK;
 }
 
@@ -348,6 +355,7 @@ int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, c
     a.S = d.S;
     a.num_replicas = problem->num_replicas;
     a.C = problem->capacity;
+    a.A = d.A;
     a.sub = lg.sub;
     a.G = lg.G;
     a.ws_barrier = static_cast<uint32_t *>(workspace);

@@ -22,7 +22,8 @@
  *   read of device data ([Megatron MORI]: sync-free counts and padded buffers).
  * Sizes.  Buffers have fixed upper-bound sizes ([Megatron MORI]: work on the
  *   full [max_tokens, ...] padded buffers and mask the tail). rows_max =
- *   E*capacity when capacity > 0, else N*k. N*k and rows_max must be < 2^31.
+ *   E*capacity when capacity > 0, else N*k + E*(row_align - 1) (N*k without
+ *   alignment). N*k and rows_max must be < 2^31.
  * Returns.  MOE_OK or a negative host-detected error; on error nothing is
  *   enqueued. Device-detected problems are OR-ed into *layout->status as
  *   MOE_DEV_* bits; read them when convenient (no call waits for them).
@@ -42,7 +43,7 @@
 extern "C" {
 #endif
 
-#define MOE_RT_ABI_VERSION 1
+#define MOE_RT_ABI_VERSION 2
 
 /* Every entry point is exported; everything else in the library is hidden. */
 #if defined(__GNUC__)
@@ -80,6 +81,9 @@ typedef struct {
     int32_t R;            /* simulated EP ranks, >= 1 */
     int32_t capacity;     /* per-expert capacity C (0 = unlimited) */
     uint32_t flags;       /* MOE_FLAG_* */
+    int32_t row_align;    /* 0 or 1 = none; A > 1: each expert's rows are padded up to a multiple of A
+                             ([Megatron MORI]: router padding for FP8 grouped GEMMs). With a capacity,
+                             C must be a multiple of A. */
 } moe_problem_t;
 
 /*
@@ -101,7 +105,8 @@ typedef struct {
     /* per physical expert */
     int32_t *counts_raw;        /* [E] assignments before capacity */
     int32_t *tokens_per_expert; /* [E] rows filled: min(counts_raw, C), or counts_raw when C = 0 */
-    int32_t *expert_offsets;    /* [E+1] first row of each expert (e*C when C > 0) */
+    int32_t *expert_offsets;    /* [E+1] first row of each expert (e*C when C > 0); an expert owns
+                                   C rows, or tokens_per_expert rounded up to a multiple of row_align */
     /* per rank */
     int32_t *input_splits;  /* [R] rows destined to rank r (pad rows included when C > 0) */
     int32_t *output_splits; /* [R] equal to input_splits on one GPU */
@@ -115,7 +120,7 @@ typedef struct {
     int32_t *row_slot;         /* top-k slot j, -1 in pad / tail rows */
     int32_t *row_local_expert; /* expert id local to the row's rank, -1 in pad / tail rows */
     float *row_prob;           /* receiver-side prob p[t,j], 0 in pad / tail rows */
-    uint8_t *pad_mask;         /* 1 = the row holds no assignment */
+    uint8_t *pad_mask;         /* 1 = the row holds no assignment (capacity or alignment pad, or tail) */
     /* optional DeepEP-contract view, [R*N*k] or NULL */
     int32_t *local_topk; /* [r][t][j]: local id if (t,j) is kept on rank r, else -1 */
 } moe_layout_t;
@@ -128,7 +133,7 @@ MOE_API const char *moe_status_string(int code);
 
 /*
  * Number of send-buffer rows (the first dimension of send / expert_out /
- * row_* buffers): E*capacity if capacity > 0, else N*k. Host only.
+ * row_* buffers): E*capacity if capacity > 0, else N*k + E*(row_align - 1). Host only.
  * Returns a negative MOE_ERR_* if the problem is invalid.
  */
 MOE_API int64_t moe_rows_max(const moe_problem_t *problem);

@@ -44,19 +44,24 @@ float oracle_f32_from_bf16(uint16_t h)
 
 int32_t oracle_num_experts(const oracle_problem *p) { return p->E_log + p->num_replicas; }
 
+static int32_t oracle_align(const oracle_problem *p) { return p->align > 1 ? p->align : 1; }
+
 int64_t oracle_rows_max(const oracle_problem *p)
 {
     /* Sync-free padded buffers ([Megatron MORI], the commit that drops the
      * recv_num_token host sync): the send buffer always has its upper-bound
-     * size. With a capacity it is E*C slots, otherwise one row per assignment. */
+     * size. With a capacity it is E*C slots, otherwise one row per assignment
+     * plus, with row alignment, at most align-1 pad rows per expert. */
     if (p->C > 0)
         return (int64_t)oracle_num_experts(p) * p->C;
-    return p->N * p->k;
+    return p->N * p->k + (int64_t)oracle_num_experts(p) * (oracle_align(p) - 1);
 }
 
 int oracle_problem_valid(const oracle_problem *p)
 {
-    if (p->N < 0 || p->k < 1 || p->E_log < 1 || p->R < 1 || p->C < 0 || p->num_replicas < 0)
+    if (p->N < 0 || p->k < 1 || p->E_log < 1 || p->R < 1 || p->C < 0 || p->num_replicas < 0 || p->align < 0)
+        return 0;
+    if (p->C > 0 && p->C % oracle_align(p) != 0)
         return 0;
     if (p->E_log % p->R != 0 || p->num_replicas % p->R != 0 || p->num_replicas > p->E_log)
         return 0;
@@ -270,10 +275,17 @@ int oracle_layout(const oracle_problem *p, const int32_t *topk_idx, const float 
         }
     }
 
-    /* 5. exclusive scan and splits. With a capacity every expert owns C rows. */
+    /* 5. exclusive scan and splits. With a capacity every expert owns C rows;
+     *    otherwise its token count, rounded up to a multiple of the row
+     *    alignment ([Megatron MORI]: router padding for FP8 grouped GEMMs). */
+    const int32_t A = oracle_align(p);
     o->expert_offsets[0] = 0;
-    for (int32_t e = 0; e < E; ++e)
-        o->expert_offsets[e + 1] = o->expert_offsets[e] + (C > 0 ? C : o->tokens_per_expert[e]);
+    for (int32_t e = 0; e < E; ++e) {
+        int32_t rows = C > 0 ? C : o->tokens_per_expert[e];
+        while (rows % A != 0)
+            ++rows;
+        o->expert_offsets[e + 1] = o->expert_offsets[e] + rows;
+    }
     *o->num_rows = o->expert_offsets[E];
     int64_t split_sum = 0;
     for (int32_t r = 0; r < R; ++r) {

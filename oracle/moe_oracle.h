@@ -32,6 +32,7 @@ typedef struct {
     int32_t num_replicas; /* replica slots in total; 0 = no reroute */
     int32_t R;            /* simulated expert-parallel ranks */
     int32_t C;            /* per-expert capacity; 0 = unlimited */
+    int32_t align;        /* rows per expert rounded up to a multiple of align; 0 or 1 = none */
 } oracle_problem;
 
 /* Every output of the dispatch layout. Arrays are caller-allocated:

@@ -69,6 +69,7 @@ class _Problem(ctypes.Structure):
         ("num_replicas", ctypes.c_int32),
         ("R", ctypes.c_int32),
         ("C", ctypes.c_int32),
+        ("align", ctypes.c_int32),
     ]
 
 
@@ -152,15 +153,17 @@ def _c(a, dtype) -> np.ndarray:
     return np.ascontiguousarray(a, dtype=dtype)
 
 
-def _problem(N, k, E_log, R, C=0, num_replicas=0) -> _Problem:
-    p = _Problem(N=int(N), k=int(k), E_log=int(E_log), num_replicas=int(num_replicas), R=int(R), C=int(C))
+def _problem(N, k, E_log, R, C=0, num_replicas=0, align=0) -> _Problem:
+    p = _Problem(N=int(N), k=int(k), E_log=int(E_log), num_replicas=int(num_replicas), R=int(R), C=int(C),
+                 align=int(align))
     if not _lib().oracle_problem_valid(ctypes.byref(p)):
-        raise ValueError(f"invalid problem N={N} k={k} E_log={E_log} R={R} C={C} replicas={num_replicas}")
+        raise ValueError(f"invalid problem N={N} k={k} E_log={E_log} R={R} C={C} replicas={num_replicas} "
+                         f"align={align}")
     return p
 
 
-def rows_max(N, k, E_log, R, C=0, num_replicas=0) -> int:
-    return int(_lib().oracle_rows_max(ctypes.byref(_problem(N, k, E_log, R, C, num_replicas))))
+def rows_max(N, k, E_log, R, C=0, num_replicas=0, align=0) -> int:
+    return int(_lib().oracle_rows_max(ctypes.byref(_problem(N, k, E_log, R, C, num_replicas, align))))
 
 
 def num_experts(E_log, num_replicas=0) -> int:
@@ -185,11 +188,11 @@ def route_topk(logits: np.ndarray, k: int, token_mask: Optional[np.ndarray] = No
 
 
 def layout(topk_idx: np.ndarray, topk_probs: Optional[np.ndarray], *, E_log: int, R: int, C: int = 0,
-           num_replicas: int = 0, local_topk: bool = True) -> dict:
+           num_replicas: int = 0, align: int = 0, local_topk: bool = True) -> dict:
     """Every dispatch-layout output as a dict of numpy arrays (see moe_oracle.c)."""
     topk_idx = _c(topk_idx, np.int32)
     N, k = topk_idx.shape
-    p = _problem(N, k, E_log, R, C, num_replicas)
+    p = _problem(N, k, E_log, R, C, num_replicas, align)
     lib = _lib()
     E = E_log + num_replicas
     NK = N * k

@@ -12,6 +12,8 @@ Shapes follow the pages' problem statements:
 * ``ultraep``   — N=8192, H=7168, 256 logical experts, top-8, 8 ranks, the 8
                   hottest experts get one replica slot each (264 physical), Zipf(1.2)
                   skew; forward and backward.
+* ``ht_align16`` — the ``ht`` shape and inputs with every expert's rows padded up to
+                  a multiple of 16 (grouped-GEMM / FP8 alignment).
 
 Recipe: logits are N(0,1) float32 plus, where a workload is skewed, a per-expert
 bias ``-s ln(rank+1)`` over a seeded ranking of the experts; hidden states and
@@ -48,6 +50,7 @@ class Workload:
     zipf_s: Optional[float] = None
     num_replicas: int = 0
     backward: bool = False
+    row_align: int = 0
     seed: int = 0x5EED0000
     note: str = field(default="", compare=False)
 
@@ -77,6 +80,7 @@ class Workload:
             zipf_s=self.zipf_s,
             num_replicas=self.num_replicas,
             backward=self.backward,
+            row_align=self.row_align,
             seed=self.seed,
             note=self.note,
         )
@@ -98,6 +102,8 @@ class Workload:
             d["replicas"] = self.num_replicas
         if self.backward:
             d["backward"] = True
+        if self.row_align > 1:
+            d["row_align"] = self.row_align
         return d
 
 
@@ -130,6 +136,9 @@ WORKLOADS = {
             backward=True,
             seed=0x5EED0005,
         ),
+        # the 4096-token / e256 / top-8 shape with every expert's rows padded to a
+        # multiple of 16 (grouped-GEMM / FP8 alignment); not one of the five configs
+        Workload("ht_align16", N=4096, H=7168, E_log=256, k=8, R=4, row_align=16, seed=0x5EED0002),
     ]
 }
 

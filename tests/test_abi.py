@@ -46,6 +46,8 @@ def test_abi_version_and_status_strings(lib):
         (dict(N=8192, H=7168, k=8, E_log=256, R=8, num_replicas=8), 65536),
         (dict(N=0, H=8, k=1, E_log=1, R=1), 0),
         (dict(N=0, H=8, k=2, E_log=4, R=2, capacity=3), 12),
+        (dict(N=4096, H=7168, k=8, E_log=256, R=4, row_align=16), 32768 + 256 * 15),
+        (dict(N=10, H=8, k=2, E_log=4, R=2, capacity=32, row_align=16), 128),
     ],
 )
 def test_rows_max(lib, kw, rows):
@@ -65,6 +67,8 @@ def test_rows_max(lib, kw, rows):
         dict(N=4, H=8, k=1, E_log=4, R=1, capacity=-1),
         dict(N=2**31, H=8, k=2, E_log=4, R=1),  # N*k overflows int32
         dict(N=4, H=8, k=1, E_log=4, R=1, flags=0x1),  # unknown flag
+        dict(N=4, H=8, k=1, E_log=4, R=1, row_align=-2),
+        dict(N=4, H=8, k=1, E_log=4, R=1, capacity=10, row_align=4),  # capacity not a multiple of the alignment
     ],
 )
 def test_invalid_problems_rejected(lib, kw):

@@ -27,7 +27,7 @@ from gpu_util import dev, host, require_cuda, route_prob_tolerance
 
 pytestmark = pytest.mark.gpu
 
-WORKLOAD_NAMES = ["tiny", "ht", "qwen3", "capacity", "ultraep"]
+WORKLOAD_NAMES = ["tiny", "ht", "qwen3", "capacity", "ultraep", "ht_align16"]
 LAYOUT_KEYS = [
     "phys_idx", "ordinal", "dest_row", "drop_mask", "counts_logical", "placement", "counts_raw",
     "tokens_per_expert", "expert_offsets", "input_splits", "output_splits", "rank_offsets", "counters",
@@ -50,7 +50,8 @@ def workload_case(name):
         w = get_workload(name)
         d = make_inputs(w, grad=True)
         idx, probs = oracle.route_topk(d["logits"], w.k)
-        L = oracle.layout(idx, probs, E_log=w.E_log, R=w.R, C=w.capacity, num_replicas=w.num_replicas)
+        L = oracle.layout(idx, probs, E_log=w.E_log, R=w.R, C=w.capacity, num_replicas=w.num_replicas,
+                          align=w.row_align)
         _cache.clear()
         _cache[name] = (w, d, idx, probs, L)
     return _cache[name]
@@ -58,7 +59,7 @@ def workload_case(name):
 
 def problem_of(w, N=None):
     return moe.Problem(N=w.N if N is None else N, H=w.H, k=w.k, E_log=w.E_log, R=w.R, capacity=w.capacity,
-                       num_replicas=w.num_replicas)
+                       num_replicas=w.num_replicas, row_align=w.row_align)
 
 
 def assert_layout_equal(G, L):
@@ -181,14 +182,24 @@ EDGE_CASES = [
     (36000, 8, 8, 256, 8, 0, 8, 0.0, 1.2),  # 288k assignments: 8 per lane in registers, reroute
     (75000, 8, 8, 64, 4, 0, 0, 0.05, 1.2),  # 600k assignments: slices too long for registers
 ]
+ALIGN_CASES = [
+    # N, H, k, E_log, R, C, reps, neg, zipf, align
+    (1000, 72, 4, 24, 4, 0, 0, 0.05, 1.4, 16),
+    (3000, 40, 2, 16, 2, 256, 0, 0.1, 1.5, 128),  # capacity and alignment
+    (2049, 24, 8, 64, 8, 0, 8, 0.0, 1.2, 8),  # reroute and alignment
+    (5, 8, 2, 4, 2, 0, 0, 0.0, None, 1000),  # alignment far above the counts
+]
 
 
-@pytest.mark.parametrize("case", EDGE_CASES, ids=[f"N{c[0]}_H{c[1]}_k{c[2]}_E{c[3]}" for c in EDGE_CASES])
+@pytest.mark.parametrize("case", EDGE_CASES + ALIGN_CASES,
+                         ids=[f"N{c[0]}_H{c[1]}_k{c[2]}_E{c[3]}" + (f"_A{c[9]}" if len(c) > 9 else "")
+                              for c in EDGE_CASES + ALIGN_CASES])
 def test_edge_cases_full_path(case):
-    N, H, k, E_log, R, C, reps, neg, zipf = case
+    N, H, k, E_log, R, C, reps, neg, zipf = case[:9]
+    A = case[9] if len(case) > 9 else 0
     idx, probs, hidden = _small_case(N, H, k, E_log, R, C, reps, neg, seed=N, zipf=zipf)
-    L = oracle.layout(idx, probs, E_log=E_log, R=R, C=C, num_replicas=reps)
-    p = moe.Problem(N=N, H=H, k=k, E_log=E_log, R=R, capacity=C, num_replicas=reps)
+    L = oracle.layout(idx, probs, E_log=E_log, R=R, C=C, num_replicas=reps, align=A)
+    p = moe.Problem(N=N, H=H, k=k, E_log=E_log, R=R, capacity=C, num_replicas=reps, row_align=A)
     G = moe.moe_dispatch_layout(p, dev(idx), dev(probs))
     torch.cuda.synchronize()
     assert_layout_equal(G, L)

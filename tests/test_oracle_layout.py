@@ -41,9 +41,10 @@ def page_ordinals(expert_ids_flat):
     return out
 
 
-def check_invariants(L, idx, probs, E_log, R, C, num_replicas=0):
+def check_invariants(L, idx, probs, E_log, R, C, num_replicas=0, align=0):
     N, k = idx.shape
     E = E_log + num_replicas
+    A = max(align, 1)
     E_loc = E // R
     NK = N * k
     flat = idx.reshape(-1)
@@ -53,7 +54,7 @@ def check_invariants(L, idx, probs, E_log, R, C, num_replicas=0):
     dest = L["dest_row"].reshape(-1)
     drop = L["drop_mask"].reshape(-1).astype(bool)
     rows_max = L["rows_max"]
-    assert rows_max == (E * C if C > 0 else NK)
+    assert rows_max == (E * C if C > 0 else NK + E * (A - 1))
 
     # per expert: ordinals are exactly 0..c-1, strictly increasing in flattened order
     for e in range(E):
@@ -75,7 +76,7 @@ def check_invariants(L, idx, probs, E_log, R, C, num_replicas=0):
     if C > 0:
         assert off.tolist() == [e * C for e in range(E + 1)]
     else:
-        assert off[0] == 0 and np.array_equal(np.diff(off), tpe)
+        assert off[0] == 0 and np.array_equal(np.diff(off), -(-tpe // A) * A)
     assert L["num_rows"][0] == off[E]
     sp = L["input_splits"]
     assert int(sp.sum()) == off[E]
@@ -228,3 +229,40 @@ def test_rank_major_example_by_hand(oracle_lib):
     assert L["row_local_expert"].tolist() == [0, 0, 1, 0, 1, 1]
     assert L["local_topk"][0].tolist() == [[-1, 0], [0, -1], [-1, 1]]
     assert L["local_topk"][1].tolist() == [[1, -1], [-1, 0], [1, -1]]
+
+
+@pytest.mark.parametrize("A", [2, 16, 128])
+@pytest.mark.parametrize("C", [0, 256])
+def test_row_alignment_closed_forms(oracle_lib, A, C):
+    """Megatron MORI page: routing maps padded for FP8 / grouped GEMMs. Every expert's rows
+    round up to a multiple of A; kept rows keep their order and move down by the pad rows of
+    the experts before them; the pads are exactly the tail of each expert's segment."""
+    if C % A:
+        pytest.skip("capacity must be a multiple of the alignment")
+    rng = np.random.default_rng(A + C)
+    N, k, E, R = 500, 4, 24, 4
+    idx = (rng.zipf(1.4, size=(N, k)) % E).astype(np.int32)
+    idx[rng.random((N, k)) < 0.05] = -1
+    probs = rng.random((N, k)).astype(np.float32)
+    L1 = oracle_lib.layout(idx, probs, E_log=E, R=R, C=C)
+    LA = oracle_lib.layout(idx, probs, E_log=E, R=R, C=C, align=A)
+    check_invariants(LA, idx, probs, E, R, C, align=A)
+    t = LA["tokens_per_expert"]
+    assert np.array_equal(t, L1["tokens_per_expert"])
+    rows = np.diff(LA["expert_offsets"])
+    assert np.all(rows % A == 0) and np.all(rows >= t) and np.all(rows - t < A if C == 0 else rows == C)
+    # kept rows move down by the pads of earlier experts
+    pads_before = np.concatenate([[0], np.cumsum(rows - np.diff(L1["expert_offsets"]))])
+    phys = LA["phys_idx"]
+    kept = LA["dest_row"] >= 0
+    assert np.array_equal(LA["dest_row"][kept], L1["dest_row"][kept] + pads_before[phys[kept]])
+    pad = np.ones(LA["rows_max"], bool)
+    for e in range(E):
+        pad[LA["expert_offsets"][e]: LA["expert_offsets"][e] + t[e]] = False
+    assert np.array_equal(LA["pad_mask"].astype(bool), pad)
+    assert LA["counters"][3] == LA["rows_max"] - LA["counters"][1]
+
+
+def test_row_alignment_rejects_capacity_not_multiple(oracle_lib):
+    with pytest.raises(ValueError):
+        oracle_lib.layout(np.zeros((4, 2), np.int32), None, E_log=4, R=2, C=10, align=4)
