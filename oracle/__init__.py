@@ -14,6 +14,7 @@ from .oracle import (
     layout,
     permute,
     combine,
+    restore_combined,
     permute_backward,
     combine_backward,
     bf16_from_f32,
@@ -29,6 +30,7 @@ __all__ = [
     "layout",
     "permute",
     "combine",
+    "restore_combined",
     "permute_backward",
     "combine_backward",
     "bf16_from_f32",

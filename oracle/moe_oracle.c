@@ -45,23 +45,35 @@ float oracle_f32_from_bf16(uint16_t h)
 int32_t oracle_num_experts(const oracle_problem *p) { return p->E_log + p->num_replicas; }
 
 static int32_t oracle_align(const oracle_problem *p) { return p->align > 1 ? p->align : 1; }
+static int32_t oracle_tp(const oracle_problem *p) { return p->tp_size > 1 ? p->tp_size : 1; }
+
+/* Capacity slots per expert in one TP peer's buffer: ceil(C / tp_size). */
+static int32_t oracle_local_capacity(const oracle_problem *p)
+{
+    int32_t T = oracle_tp(p);
+    return p->C > 0 ? (p->C + T - 1) / T : 0;
+}
 
 int64_t oracle_rows_max(const oracle_problem *p)
 {
     /* Sync-free padded buffers ([Megatron MORI], the commit that drops the
      * recv_num_token host sync): the send buffer always has its upper-bound
      * size. With a capacity it is E*C slots, otherwise one row per assignment
-     * plus, with row alignment, at most align-1 pad rows per expert. */
+     * plus, with row alignment, at most align-1 pad rows per expert. A TP peer
+     * holds at most ceil(c_e / tp_size) of each expert's c_e assignments. */
+    const int64_t E = oracle_num_experts(p), T = oracle_tp(p);
     if (p->C > 0)
-        return (int64_t)oracle_num_experts(p) * p->C;
-    return p->N * p->k + (int64_t)oracle_num_experts(p) * (oracle_align(p) - 1);
+        return E * oracle_local_capacity(p);
+    return (p->N * p->k + E * (T - 1)) / T + E * (oracle_align(p) - 1);
 }
 
 int oracle_problem_valid(const oracle_problem *p)
 {
     if (p->N < 0 || p->k < 1 || p->E_log < 1 || p->R < 1 || p->C < 0 || p->num_replicas < 0 || p->align < 0)
         return 0;
-    if (p->C > 0 && p->C % oracle_align(p) != 0)
+    if (p->tp_size < 0 || p->tp_rank < 0 || p->tp_rank >= oracle_tp(p))
+        return 0;
+    if (p->C > 0 && oracle_local_capacity(p) % oracle_align(p) != 0)
         return 0;
     if (p->E_log % p->R != 0 || p->num_replicas % p->R != 0 || p->num_replicas > p->E_log)
         return 0;
@@ -144,7 +156,9 @@ void oracle_route_topk(const float *logits, const uint8_t *token_mask, int64_t N
  *     tokens rerouted to the replica slot; router semantics stay logical);
  *  3. physical ordinals and counts;
  *  4. capacity: drop_mask, tokens_per_expert, pad rows ([DeepSpeed EP]
- *     RoutedAssignmentPayload.capacity_slots / drop_mask / pad_mask);
+ *     RoutedAssignmentPayload.capacity_slots / drop_mask / pad_mask), then
+ *     the optional TP folding of the active assignments ([DeepSpeed EP]
+ *     partition_assignments);
  *  5. exclusive scan into expert_offsets, per-rank input_splits / rank_offsets,
  *     output_splits = input_splits ([DeepSpeed EP] _recompute_input_splits,
  *     partition_assignments);
@@ -258,9 +272,7 @@ int oracle_layout(const oracle_problem *p, const int32_t *topk_idx, const float 
     }
 
     /* 4. capacity: an assignment whose physical ordinal reaches C is dropped. */
-    for (int32_t e = 0; e < E; ++e)
-        o->tokens_per_expert[e] = 0;
-    int64_t valid = 0, kept = 0, dropped = 0;
+    int64_t valid = 0, dropped = 0;
     for (int64_t a = 0; a < NK; ++a) {
         o->drop_mask[a] = 0;
         if (o->phys_idx[a] < 0)
@@ -269,19 +281,39 @@ int oracle_layout(const oracle_problem *p, const int32_t *topk_idx, const float 
         if (C > 0 && o->ordinal[a] >= C) {
             o->drop_mask[a] = 1;
             ++dropped;
-        } else {
-            o->tokens_per_expert[o->phys_idx[a]] += 1;
-            ++kept;
         }
     }
 
-    /* 5. exclusive scan and splits. With a capacity every expert owns C rows;
-     *    otherwise its token count, rounded up to a multiple of the row
-     *    alignment ([Megatron MORI]: router padding for FP8 grouped GEMMs). */
+    /* 4b. TP folding ([DeepSpeed EP] partition_assignments): this peer keeps the
+     *     active (valid, not dropped) assignments whose stable per-expert ordinal
+     *     is congruent to tp_rank modulo tp_size; its local ordinal is the running
+     *     count of earlier kept assignments to the same expert. Without folding
+     *     every active assignment is kept at its own ordinal. */
+    const int32_t T = oracle_tp(p);
+    int32_t *local_ordinal = (int32_t *)malloc((size_t)(NK > 0 ? NK : 1) * sizeof(int32_t));
+    for (int32_t e = 0; e < E; ++e) {
+        o->tokens_per_expert[e] = 0;
+        seen[e] = 0;
+    }
+    int64_t kept = 0;
+    for (int64_t a = 0; a < NK; ++a) {
+        int32_t q = o->phys_idx[a];
+        local_ordinal[a] = -1;
+        if (q < 0 || o->drop_mask[a] || o->ordinal[a] % T != p->tp_rank)
+            continue;
+        local_ordinal[a] = seen[q]++;
+        o->tokens_per_expert[q] += 1;
+        ++kept;
+    }
+
+    /* 5. exclusive scan and splits. With a capacity every expert owns C rows
+     *    (ceil(C / tp_size) in a TP peer's buffer); otherwise its token count,
+     *    rounded up to a multiple of the row alignment ([Megatron MORI]: router
+     *    padding for FP8 grouped GEMMs). */
     const int32_t A = oracle_align(p);
     o->expert_offsets[0] = 0;
     for (int32_t e = 0; e < E; ++e) {
-        int32_t rows = C > 0 ? C : o->tokens_per_expert[e];
+        int32_t rows = C > 0 ? oracle_local_capacity(p) : o->tokens_per_expert[e];
         while (rows % A != 0)
             ++rows;
         o->expert_offsets[e + 1] = o->expert_offsets[e] + rows;
@@ -307,11 +339,11 @@ int oracle_layout(const oracle_problem *p, const int32_t *topk_idx, const float 
     }
     for (int64_t a = 0; a < NK; ++a) {
         int32_t q = o->phys_idx[a];
-        if (q < 0 || o->drop_mask[a]) {
+        if (local_ordinal[a] < 0) {
             o->dest_row[a] = -1;
             continue;
         }
-        int32_t row = o->expert_offsets[q] + o->ordinal[a];
+        int32_t row = o->expert_offsets[q] + local_ordinal[a];
         o->dest_row[a] = row;
         o->row_token[row] = (int32_t)(a / k);
         o->row_slot[row] = (int32_t)(a % k);
@@ -325,7 +357,7 @@ int oracle_layout(const oracle_problem *p, const int32_t *topk_idx, const float 
         for (int32_t r = 0; r < R; ++r)
             for (int64_t a = 0; a < NK; ++a) {
                 int32_t q = o->phys_idx[a];
-                int keep = q >= 0 && !o->drop_mask[a] && q / E_loc == r;
+                int keep = local_ordinal[a] >= 0 && q / E_loc == r;
                 o->local_topk[(int64_t)r * NK + a] = keep ? q - r * E_loc : -1;
             }
     }
@@ -338,6 +370,7 @@ int oracle_layout(const oracle_problem *p, const int32_t *topk_idx, const float 
     o->counters[ORC_NUM_ROWS] = *o->num_rows;
     o->counters[ORC_ERROR] = error;
 
+    free(local_ordinal);
     free(seen);
     return 0;
 }
@@ -388,6 +421,31 @@ void oracle_combine(const oracle_problem *p, int32_t H, const int32_t *dest_row,
                 float w = topk_probs ? topk_probs[t * p->k + j] : 1.0f;
                 acc = fmaf(w, oracle_f32_from_bf16(expert_out[(int64_t)row * H + h]), acc);
             }
+            out[t * H + h] = oracle_bf16_from_f32(acc);
+        }
+}
+
+/*
+ * [DeepSpeed EP] restore_combined: the TP peers' weighted outputs are gathered
+ * and added back per token one top-k slot at a time in ascending slot order.
+ * On one GPU the gather is the set of peer buffers: dest_rows[q] and
+ * expert_outs[q] are peer q's row map and expert output; each assignment has a
+ * row in at most one peer. Same fp32 fused multiply-add chain as the combine.
+ */
+void oracle_restore_combined(const oracle_problem *p, int32_t H, int32_t tp_size, const int32_t *const *dest_rows,
+                             const uint16_t *const *expert_outs, const float *topk_probs, uint16_t *out)
+{
+    for (int64_t t = 0; t < p->N; ++t)
+        for (int32_t h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int32_t j = 0; j < p->k; ++j)
+                for (int32_t q = 0; q < tp_size; ++q) {
+                    int32_t row = dest_rows[q][t * p->k + j];
+                    if (row < 0)
+                        continue;
+                    float w = topk_probs ? topk_probs[t * p->k + j] : 1.0f;
+                    acc = fmaf(w, oracle_f32_from_bf16(expert_outs[q][(int64_t)row * H + h]), acc);
+                }
             out[t * H + h] = oracle_bf16_from_f32(acc);
         }
 }

@@ -33,6 +33,8 @@ typedef struct {
     int32_t R;            /* simulated expert-parallel ranks */
     int32_t C;            /* per-expert capacity; 0 = unlimited */
     int32_t align;        /* rows per expert rounded up to a multiple of align; 0 or 1 = none */
+    int32_t tp_size;      /* TP folding: peers sharing the assignments; 0 or 1 = none */
+    int32_t tp_rank;      /* this peer, 0 <= tp_rank < tp_size */
 } oracle_problem;
 
 /* Every output of the dispatch layout. Arrays are caller-allocated:
@@ -84,6 +86,9 @@ void oracle_permute(const oracle_problem *p, int32_t H, const int32_t *dest_row,
 
 void oracle_combine(const oracle_problem *p, int32_t H, const int32_t *dest_row, const uint16_t *expert_out,
                     const float *topk_probs, uint16_t *out);
+
+void oracle_restore_combined(const oracle_problem *p, int32_t H, int32_t tp_size, const int32_t *const *dest_rows,
+                             const uint16_t *const *expert_outs, const float *topk_probs, uint16_t *out);
 
 void oracle_permute_backward(const oracle_problem *p, int32_t H, const int32_t *dest_row,
                              const uint16_t *grad_send, uint16_t *grad_hidden);

@@ -70,6 +70,8 @@ class _Problem(ctypes.Structure):
         ("R", ctypes.c_int32),
         ("C", ctypes.c_int32),
         ("align", ctypes.c_int32),
+        ("tp_size", ctypes.c_int32),
+        ("tp_rank", ctypes.c_int32),
     ]
 
 
@@ -124,6 +126,9 @@ def _lib() -> ctypes.CDLL:
         lib.oracle_permute.argtypes = [ctypes.POINTER(_Problem), ctypes.c_int32, _P, ctypes.c_int64, _P, _P]
         lib.oracle_combine.restype = None
         lib.oracle_combine.argtypes = [ctypes.POINTER(_Problem), ctypes.c_int32, _P, _P, _P, _P]
+        lib.oracle_restore_combined.restype = None
+        lib.oracle_restore_combined.argtypes = [ctypes.POINTER(_Problem), ctypes.c_int32, ctypes.c_int32, _P, _P, _P,
+                                                _P]
         lib.oracle_permute_backward.restype = None
         lib.oracle_permute_backward.argtypes = [ctypes.POINTER(_Problem), ctypes.c_int32, _P, _P, _P]
         lib.oracle_combine_backward.restype = None
@@ -153,17 +158,18 @@ def _c(a, dtype) -> np.ndarray:
     return np.ascontiguousarray(a, dtype=dtype)
 
 
-def _problem(N, k, E_log, R, C=0, num_replicas=0, align=0) -> _Problem:
+def _problem(N, k, E_log, R, C=0, num_replicas=0, align=0, tp_size=0, tp_rank=0) -> _Problem:
     p = _Problem(N=int(N), k=int(k), E_log=int(E_log), num_replicas=int(num_replicas), R=int(R), C=int(C),
-                 align=int(align))
+                 align=int(align), tp_size=int(tp_size), tp_rank=int(tp_rank))
     if not _lib().oracle_problem_valid(ctypes.byref(p)):
         raise ValueError(f"invalid problem N={N} k={k} E_log={E_log} R={R} C={C} replicas={num_replicas} "
-                         f"align={align}")
+                         f"align={align} tp={tp_rank}/{tp_size}")
     return p
 
 
-def rows_max(N, k, E_log, R, C=0, num_replicas=0, align=0) -> int:
-    return int(_lib().oracle_rows_max(ctypes.byref(_problem(N, k, E_log, R, C, num_replicas, align))))
+def rows_max(N, k, E_log, R, C=0, num_replicas=0, align=0, tp_size=0, tp_rank=0) -> int:
+    p = _problem(N, k, E_log, R, C, num_replicas, align, tp_size, tp_rank)
+    return int(_lib().oracle_rows_max(ctypes.byref(p)))
 
 
 def num_experts(E_log, num_replicas=0) -> int:
@@ -188,11 +194,12 @@ def route_topk(logits: np.ndarray, k: int, token_mask: Optional[np.ndarray] = No
 
 
 def layout(topk_idx: np.ndarray, topk_probs: Optional[np.ndarray], *, E_log: int, R: int, C: int = 0,
-           num_replicas: int = 0, align: int = 0, local_topk: bool = True) -> dict:
+           num_replicas: int = 0, align: int = 0, tp_size: int = 0, tp_rank: int = 0,
+           local_topk: bool = True) -> dict:
     """Every dispatch-layout output as a dict of numpy arrays (see moe_oracle.c)."""
     topk_idx = _c(topk_idx, np.int32)
     N, k = topk_idx.shape
-    p = _problem(N, k, E_log, R, C, num_replicas, align)
+    p = _problem(N, k, E_log, R, C, num_replicas, align, tp_size, tp_rank)
     lib = _lib()
     E = E_log + num_replicas
     NK = N * k
@@ -256,6 +263,22 @@ def combine(expert_out: np.ndarray, dest_row: np.ndarray, topk_probs: Optional[n
     p = _Problem(N=N, k=k, E_log=1, num_replicas=0, R=1, C=0)
     out = np.empty((N, H), np.uint16)
     _lib().oracle_combine(ctypes.byref(p), H, _ptr(dest_row), _ptr(expert_out), _ptr(probs), _ptr(out))
+    return out
+
+
+def restore_combined(expert_outs, dest_rows, topk_probs: Optional[np.ndarray]) -> np.ndarray:
+    """Slot-ordered combine over the TP peers' buffers (one row map and expert output per peer)."""
+    expert_outs = [_c(y, np.uint16) for y in expert_outs]
+    dest_rows = [_c(d, np.int32) for d in dest_rows]
+    T = len(dest_rows)
+    N, k = dest_rows[0].shape
+    H = expert_outs[0].shape[1]
+    probs = None if topk_probs is None else _c(topk_probs, np.float32)
+    p = _Problem(N=N, k=k, E_log=1, num_replicas=0, R=1, C=0)
+    d_arr = (ctypes.c_void_p * T)(*[d.ctypes.data for d in dest_rows])
+    y_arr = (ctypes.c_void_p * T)(*[y.ctypes.data for y in expert_outs])
+    out = np.empty((N, H), np.uint16)
+    _lib().oracle_restore_combined(ctypes.byref(p), H, T, d_arr, y_arr, _ptr(probs), _ptr(out))
     return out
 
 
