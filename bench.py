@@ -177,44 +177,68 @@ class ClockSampler:
 
 
 class Step:
-    """One step of the hot path with every C-ABI argument marshalled up front."""
+    """One step of the hot path with every C-ABI argument marshalled up front.
+
+    With TP folding (workload tp_size = T > 1) the step routes once, builds the
+    layout and the send buffer of every peer in turn (all on this GPU), and
+    restores with one slot-ordered combine over the peers' buffers."""
 
     def __init__(self, w, moe, native, torch, sets, device):
         self.w = w
         self.torch = torch
         self.lib = native.lib()
-        p = moe.Problem(N=w.N, H=w.H, k=w.k, E_log=w.E_log, R=w.R, capacity=w.capacity,
-                        num_replicas=w.num_replicas, row_align=w.row_align)
+        T = max(w.tp_size, 1)
+        self.T = T
+        self.problems = [moe.Problem(N=w.N, H=w.H, k=w.k, E_log=w.E_log, R=w.R, capacity=w.capacity,
+                                     num_replicas=w.num_replicas, row_align=w.row_align,
+                                     tp_size=w.tp_size, tp_rank=r) for r in range(T)]
+        p = self.problems[0]
         self.problem = p
-        self.layout = moe.Layout.allocate(p, device)
+        self.layouts = [moe.Layout.allocate(q, device) for q in self.problems]
+        self.layout = self.layouts[0]
         self.sets = sets
         N, H, k = w.N, w.H, w.k
         RM = p.rows_max
         self.idx = torch.empty((N, k), dtype=torch.int32, device=device)
         self.probs = torch.empty((N, k), dtype=torch.float32, device=device)
-        self.send = torch.empty((RM, H), dtype=torch.bfloat16, device=device)
+        self.sends = [torch.empty((RM, H), dtype=torch.bfloat16, device=device) for _ in range(T)]
+        self.send = self.sends[0]
         self.out = torch.empty((N, H), dtype=torch.bfloat16, device=device)
         if w.backward:
             self.gy = torch.empty((RM, H), dtype=torch.bfloat16, device=device)
             self.gp = torch.empty((N, k), dtype=torch.float32, device=device)
             self.gh = torch.empty((N, H), dtype=torch.bfloat16, device=device)
-        self._p = p.c_struct()
-        self._L = self.layout.c_struct()
+        self._ps = [q.c_struct() for q in self.problems]
+        self._Ls = [L.c_struct() for L in self.layouts]
+        self._L_arr = (native.MoeLayout * T)(*self._Ls)
+        self._y_arr = (ctypes.c_void_p * T)(*[y.data_ptr() for y in self.sends])
         self.stream = torch.cuda.current_stream(device)
         self._s = ctypes.c_void_p(self.stream.cuda_stream)
         vp = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
-        P, L = ctypes.byref(self._p), ctypes.byref(self._L)
-        ws = self.layout.workspace
+        P, L = ctypes.byref(self._ps[0]), ctypes.byref(self._Ls[0])
         self.calls = []
         for s in sets:
-            c = [
-                ("route", self.lib.moe_route_topk,
-                 (vp(s["logits"]), None, N, w.E_log, k, vp(self.idx), vp(self.probs), self._s)),
-                ("layout", self.lib.moe_dispatch_layout,
-                 (P, vp(self.idx), vp(self.probs), L, vp(ws), ws.numel(), self._s)),
-                ("permute", self.lib.moe_permute, (P, L, vp(s["hidden"]), vp(self.send), self._s)),
-                ("combine", self.lib.moe_combine, (P, L, vp(self.send), vp(self.probs), vp(self.out), self._s)),
-            ]
+            c = [("route", self.lib.moe_route_topk,
+                  (vp(s["logits"]), None, N, w.E_log, k, vp(self.idx), vp(self.probs), self._s))]
+            if T == 1:
+                ws = self.layout.workspace
+                c += [
+                    ("layout", self.lib.moe_dispatch_layout,
+                     (P, vp(self.idx), vp(self.probs), L, vp(ws), ws.numel(), self._s)),
+                    ("permute", self.lib.moe_permute, (P, L, vp(s["hidden"]), vp(self.send), self._s)),
+                    ("combine", self.lib.moe_combine, (P, L, vp(self.send), vp(self.probs), vp(self.out), self._s)),
+                ]
+            else:
+                for r in range(T):
+                    Pr, Lr = ctypes.byref(self._ps[r]), ctypes.byref(self._Ls[r])
+                    ws = self.layouts[r].workspace
+                    c += [
+                        (f"layout.{r}", self.lib.moe_dispatch_layout,
+                         (Pr, vp(self.idx), vp(self.probs), Lr, vp(ws), ws.numel(), self._s)),
+                        (f"permute.{r}", self.lib.moe_permute, (Pr, Lr, vp(s["hidden"]), vp(self.sends[r]), self._s)),
+                    ]
+                c += [("restore", self.lib.moe_restore_combined,
+                       (P, self._L_arr, self._y_arr, vp(self.probs), vp(self.out), self._s))]
             if w.backward:
                 c += [
                     ("combine_backward", self.lib.moe_combine_backward,
@@ -234,23 +258,36 @@ class Step:
             if events is not None:
                 events[n][1].record(self.stream)
 
+    def status(self) -> int:
+        st = 0
+        for L in self.layouts:
+            st |= L.status()
+        return st
 
-def algorithmic_bytes(w, p, kept_rows, read_tokens):
-    """Bytes each kernel must move at least once (see the design notes).
+    def algorithmic_bytes(self) -> dict:
+        """Bytes each kernel must move at least once, from the last step's layouts.
 
-    kept_rows: send rows that hold an assignment; read_tokens: tokens with at
-    least one kept slot (only those rows of hidden must be read)."""
-    N, H, k, E = w.N, w.H, w.k, w.E_log
-    RM = p.rows_max
-    row = H * 2
-    return {
-        "route": N * E * 4 + N * k * 8,
-        "layout": N * k * 8 + N * k * (4 + 4 + 4 + 1) + RM * (4 * 4 + 1) + w.R * N * k * 4,
-        "permute": read_tokens * row + RM * row + N * k * 4 + RM,
-        "combine": kept_rows * row + N * row + N * k * 8,
-        "combine_backward": N * row + kept_rows * row + RM * row + N * k * 8 + N * k * 4,
-        "permute_backward": kept_rows * row + N * row + N * k * 4,
-    }
+        A row of hidden is read only if its token keeps a slot; every send row is
+        written (pads as zeros); the combine reads only kept rows."""
+        w, T = self.w, self.T
+        N, H, k, E = w.N, w.H, w.k, w.E_log
+        NK, row, RM = N * k, H * 2, self.problem.rows_max
+        kept = [int(L["counters"][1].item()) for L in self.layouts]
+        read = [int((L["dest_row"] >= 0).any(dim=1).sum().item()) for L in self.layouts]
+        layout_bytes = NK * 8 + NK * (4 + 4 + 4 + 1) + RM * (4 * 4 + 1) + w.R * NK * 4
+        out = {"route": N * E * 4 + NK * 8}
+        if T == 1:
+            out["layout"] = layout_bytes
+            out["permute"] = read[0] * row + RM * row + NK * 4 + RM
+            out["combine"] = kept[0] * row + N * row + NK * 8
+        else:
+            for r in range(T):
+                out[f"layout.{r}"] = layout_bytes
+                out[f"permute.{r}"] = read[r] * row + RM * row + NK * 4 + RM
+            out["restore"] = sum(kept) * row + N * row + NK * 4 * (T + 1)
+        out["combine_backward"] = N * row + kept[0] * row + RM * row + NK * 8 + NK * 4
+        out["permute_backward"] = kept[0] * row + N * row + NK * 4
+        return out
 
 
 def run_ours(args, ws, rank, local):
@@ -296,8 +333,7 @@ def run_ours(args, ws, rank, local):
     for i in range(args.warmup):
         step.run(i)
     torch.cuda.synchronize()
-    kept = [int(v) for v in step.layout["counters"].tolist()][1]
-    read_tokens = int((step.layout["dest_row"] >= 0).any(dim=1).sum().item())
+    abytes = step.algorithmic_bytes()
 
     nk = len(step.kernel_names)
     t0 = torch.cuda.Event(enable_timing=True)
@@ -329,7 +365,7 @@ def run_ours(args, ws, rank, local):
     for i in range(args.steps):
         for n, name in enumerate(step.kernel_names):
             per_kernel_ms[name].append(events[i][n][0].elapsed_time(events[i][n][1]))
-    status = step.layout.status()
+    status = step.status()
     if status != 0:
         raise RuntimeError(f"device status {status:#x} after the timed steps")
     elapsed_ms = max_over_ranks(elapsed_ms, device)
@@ -380,7 +416,6 @@ def run_ours(args, ws, rank, local):
         return None
 
     peak, peak_kind = measured_peaks()
-    abytes = algorithmic_bytes(w, step.problem, kept, read_tokens)
     kernels = {}
     for name in step.kernel_names:
         avg_ms = statistics.mean(per_kernel_ms[name])
@@ -441,10 +476,18 @@ def run_ours(args, ws, rank, local):
 def oracle_step(oracle, w, d):
     """The whole path on the CPU oracle for the batch in ``d``."""
     idx, probs = oracle.route_topk(d["logits"], w.k)
-    L = oracle.layout(idx, probs, E_log=w.E_log, R=w.R, C=w.capacity, num_replicas=w.num_replicas,
-                      align=w.row_align, local_topk=True)
-    send = oracle.permute(d["hidden"], L["dest_row"], L["rows_max"])
-    out = oracle.combine(send, L["dest_row"], probs)
+    T = max(w.tp_size, 1)
+    layouts, sends = [], []
+    for r in range(T):
+        L = oracle.layout(idx, probs, E_log=w.E_log, R=w.R, C=w.capacity, num_replicas=w.num_replicas,
+                          align=w.row_align, tp_size=w.tp_size, tp_rank=r, local_topk=True)
+        layouts.append(L)
+        sends.append(oracle.permute(d["hidden"], L["dest_row"], L["rows_max"]))
+    L, send = layouts[0], sends[0]
+    if T == 1:
+        out = oracle.combine(send, L["dest_row"], probs)
+    else:
+        out = oracle.restore_combined(sends, [x["dest_row"] for x in layouts], probs)
     if w.backward:
         gy, gp = oracle.combine_backward(d["grad_out"], send, L["dest_row"], L["row_token"], L["row_prob"])
         oracle.permute_backward(gy, L["dest_row"])

@@ -8,6 +8,7 @@ functions keep the C names:
     moe_dispatch_layout   reroute, histogram, ordinals, capacity, scan, splits, row maps
     moe_permute           send[dest_row[t, j]] = hidden[t]
     moe_combine           out[t] = bf16(sum_j p[t, j] * y[dest_row[t, j]]), fp32, ascending j
+    moe_restore_combined  the same over the buffers of TP peers (after TP folding)
     moe_permute_backward  grad_hidden[t] = bf16(sum_j grad_send[dest_row[t, j]])
     moe_combine_backward  grad_y[row] = bf16(p * grad_out[t]); grad_probs[t, j] = <grad_out[t], y[row]>
 
@@ -54,6 +55,7 @@ __all__ = [
     "moe_dispatch_layout_noalloc",
     "moe_permute",
     "moe_combine",
+    "moe_restore_combined",
     "moe_permute_backward",
     "moe_combine_backward",
     "load_library",
@@ -84,6 +86,8 @@ class Problem:
     num_replicas: int = 0
     flags: int = MOE_FLAG_NONE
     row_align: int = 0
+    tp_size: int = 0
+    tp_rank: int = 0
 
     @property
     def E(self) -> int:
@@ -104,6 +108,8 @@ class Problem:
             capacity=self.capacity,
             flags=self.flags,
             row_align=self.row_align,
+            tp_size=self.tp_size,
+            tp_rank=self.tp_rank,
         )
 
     @property
@@ -310,6 +316,28 @@ def moe_combine(problem: Problem, layout: Layout, expert_out: torch.Tensor, topk
     _native.check("moe_combine",
                   _native.lib().moe_combine(ctypes.byref(p), ctypes.byref(L), _ptr(expert_out), _ptr(topk_probs),
                                             _ptr(out), _stream(stream)))
+    return out
+
+
+def moe_restore_combined(problem: Problem, layouts, expert_outs, topk_probs: Optional[torch.Tensor],
+                         out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Slot-ordered combine over the TP peers' buffers (layouts[q], expert_outs[q] of peer q)."""
+    T = max(problem.tp_size, 1)
+    if len(layouts) != T or len(expert_outs) != T:
+        raise ValueError(f"need {T} peer layouts and expert outputs")
+    for q in range(T):
+        _need(expert_outs[q], f"expert_outs[{q}]", torch.bfloat16, (problem.rows_max, problem.H), layouts[0].device)
+    if topk_probs is not None:
+        _need(topk_probs, "topk_probs", torch.float32, (problem.N, problem.k), layouts[0].device)
+    if out is None:
+        out = torch.empty((problem.N, problem.H), dtype=torch.bfloat16, device=layouts[0].device)
+    _need(out, "out", torch.bfloat16, (problem.N, problem.H), layouts[0].device)
+    p = problem.c_struct()
+    Ls = (_native.MoeLayout * T)(*[L.c_struct() for L in layouts])
+    ys = (ctypes.c_void_p * T)(*[y.data_ptr() for y in expert_outs])
+    _native.check("moe_restore_combined",
+                  _native.lib().moe_restore_combined(ctypes.byref(p), Ls, ys, _ptr(topk_probs), _ptr(out),
+                                                     _stream(stream)))
     return out
 
 

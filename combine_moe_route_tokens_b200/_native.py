@@ -23,6 +23,7 @@ MOE_ERR_UNSUPPORTED = -2
 MOE_ERR_CUDA = -3
 MOE_ERR_SCRATCH_LIMIT = -4
 MOE_NOALLOC_MAX_E_LOG = 512
+MOE_MAX_TP = 8
 
 MOE_DEV_EXPERT_RANGE = 0x1
 MOE_DEV_TIMEOUT = 0x2
@@ -31,7 +32,7 @@ MOE_DEV_ROW_RANGE = 0x4
 MOE_FLAG_NONE = 0
 MOE_FLAG_TEST_BARRIER_TIMEOUT = 0x80000000
 
-ABI_VERSION = 2
+ABI_VERSION = 3
 
 
 class MoeProblem(ctypes.Structure):
@@ -45,6 +46,8 @@ class MoeProblem(ctypes.Structure):
         ("capacity", ctypes.c_int32),
         ("flags", ctypes.c_uint32),
         ("row_align", ctypes.c_int32),
+        ("tp_size", ctypes.c_int32),
+        ("tp_rank", ctypes.c_int32),
     ]
 
 
@@ -99,6 +102,7 @@ _SIGNATURES = {
     "moe_dispatch_layout_noalloc": (ctypes.c_int, [_PP, _VP, _VP, _PL, _VP]),
     "moe_permute": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP]),
     "moe_combine": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP]),
+    "moe_restore_combined": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP]),
     "moe_permute_backward": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP]),
     "moe_combine_backward": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP, _VP, _VP]),
 }

@@ -41,6 +41,10 @@ struct CombineArgs {
     int32_t k;
     int32_t V;       // 16-byte chunks per row (H / 8)
     int32_t nchunks; // CTAs per token
+    // restore after TP folding: T peer buffers and row maps (y / dest_row unused)
+    int32_t T;
+    const uint4 *ys[MOE_MAX_TP];
+    const int32_t *dests[MOE_MAX_TP];
 };
 
 __device__ __forceinline__ void fma8(float (&acc)[8], float p, const uint4 &y)
@@ -78,7 +82,42 @@ __device__ __forceinline__ void load_slot_meta(const int32_t *dest_row, const fl
     }
 }
 
-template <int K> // K > 0: top-k fixed at compile time; K == 0: runtime k <= 32
+// Restore after TP folding: slot j of token t lives in the one peer buffer whose
+// row map has a row for it. Lane j < k finds that peer and folds it into the
+// row index as peer * rows_max + row (peer_row() undoes it).
+__device__ __forceinline__ void load_slot_meta_peers(const CombineArgs &a, int64_t t, int k, int32_t &d, float &p)
+{
+    const int lane = threadIdx.x & 31;
+    d = -1;
+    p = 0.0f;
+    if (lane < k) {
+        p = a.probs != nullptr ? __ldg(a.probs + t * k + lane) : 1.0f;
+        for (int q = 0; q < a.T; ++q) {
+            const int32_t r = __ldg(a.dests[q] + t * k + lane);
+            if (r < -1 || r >= a.rows_max) {
+                atomicOr(a.status, MOE_DEV_ROW_RANGE);
+                continue;
+            }
+            if (r >= 0 && d < 0)
+                d = static_cast<int32_t>(q * a.rows_max + r);
+        }
+    }
+}
+
+__device__ __forceinline__ const uint4 *peer_row(const CombineArgs &a, int32_t folded)
+{
+    const int q = static_cast<int>(folded / a.rows_max);
+    const int64_t r = folded - static_cast<int64_t>(q) * a.rows_max;
+    const uint4 *base = a.ys[0];
+#pragma unroll
+    for (int i = 1; i < MOE_MAX_TP; ++i)
+        base = (q == i) ? a.ys[i] : base;
+    return base + r * a.V;
+}
+
+// K > 0: top-k fixed at compile time; K == 0: runtime k <= 32.
+// PEERS: gather from the TP peers' buffers (restore) instead of one buffer.
+template <int K, bool PEERS = false>
 __global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(CombineArgs a)
 {
     pdl_trigger();
@@ -90,7 +129,16 @@ __global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(CombineArgs a)
 
     int32_t d;
     float p;
-    load_slot_meta(a.dest_row, a.probs, t, k, a.rows_max, a.status, d, p);
+    if constexpr (PEERS)
+        load_slot_meta_peers(a, t, k, d, p);
+    else
+        load_slot_meta(a.dest_row, a.probs, t, k, a.rows_max, a.status, d, p);
+    auto row_ptr = [&](int32_t row) -> const uint4 * {
+        if constexpr (PEERS)
+            return peer_row(a, row);
+        else
+            return a.y + static_cast<int64_t>(row) * a.V;
+    };
 
     float acc[8];
 #pragma unroll
@@ -111,7 +159,7 @@ __global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(CombineArgs a)
 #pragma unroll
         for (int j = 0; j < K; ++j)
             if (dj[j] >= 0)
-                yj[j] = ld_stream_u4(a.y + static_cast<int64_t>(dj[j]) * a.V + v);
+                yj[j] = ld_stream_u4(row_ptr(dj[j]) + v);
 #pragma unroll
         for (int j = 0; j < K; ++j)
             if (dj[j] >= 0)
@@ -132,7 +180,7 @@ __global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(CombineArgs a)
 #pragma unroll
             for (int u = 0; u < 4; ++u)
                 if (dj[u] >= 0)
-                    yj[u] = ld_stream_u4(a.y + static_cast<int64_t>(dj[u]) * a.V + v);
+                    yj[u] = ld_stream_u4(row_ptr(dj[u]) + v);
 #pragma unroll
             for (int u = 0; u < 4; ++u)
                 if (dj[u] >= 0)

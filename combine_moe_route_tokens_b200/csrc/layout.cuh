@@ -47,7 +47,10 @@ struct LayoutArgs {
     int64_t NK;
     int64_t rows_max;
     int32_t k, E_log, E, R, E_loc, M, S, num_replicas, C;
-    int32_t A; // row alignment (1 = none)
+    int32_t A;       // row alignment (1 = none)
+    int32_t T;       // TP folding peers (1 = none)
+    int32_t tp_rank; // this peer
+    int32_t C_local; // capacity slots per expert in this peer's buffer: ceil(C / T)
     int32_t sub; // assignments per warp slice, a multiple of 32
     int32_t G;   // blocks
     int32_t *ws_counts;   // [G][E_log]: per-block logical totals
@@ -110,6 +113,14 @@ __device__ __forceinline__ bool layout_grid_barrier(uint32_t *bar, uint32_t targ
     }
     __syncthreads();
     return s_ok != 0;
+}
+
+// Rows this peer keeps of an expert with `raw` assignments: the capacity-kept
+// ones (min(raw, C)) whose ordinal is congruent to tp_rank modulo T.
+__device__ __forceinline__ int32_t layout_local_tokens(const LayoutArgs &a, int32_t raw)
+{
+    const int32_t t = a.C > 0 ? min(raw, a.C) : raw;
+    return t > a.tp_rank ? (t - a.tp_rank + a.T - 1) / a.T : 0;
 }
 
 __device__ __forceinline__ uint32_t lanemask_lt()
@@ -209,7 +220,7 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
     int32_t *s_off = s_raw + E;                                                // [E+1]
     __shared__ int32_t s_hot[LAYOUT_MAX_E_LOG];
     __shared__ int32_t s_part[2][LAYOUT_THREADS];
-    __shared__ int32_t s_wsum[3][LAYOUT_WARPS];
+    __shared__ int32_t s_wsum[4][LAYOUT_WARPS];
     __shared__ uint32_t s_err;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -373,20 +384,22 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
                 s_raw[s_repl[e]] = s_cnt[e] / 2;
         __syncthreads();
     }
-    int32_t total_valid, total_kept;
+    int32_t total_valid, total_kept, total_dropped;
     {
         constexpr int PER = 8; // E <= 4096 = LAYOUT_THREADS * PER
         const int q0 = tid * PER;
         int32_t rows[PER];
-        int32_t sum = 0, valid = 0, kept = 0;
+        int32_t sum = 0, valid = 0, kept = 0, dropped = 0;
 #pragma unroll
         for (int u = 0; u < PER; ++u) {
             const int q = q0 + u;
             const int32_t raw = q < E ? s_raw[q] : 0;
-            rows[u] = q < E ? (a.C > 0 ? a.C : ((raw + a.A - 1) / a.A) * a.A) : 0;
+            const int32_t local = layout_local_tokens(a, raw);
+            rows[u] = q < E ? (a.C > 0 ? a.C_local : ((local + a.A - 1) / a.A) * a.A) : 0;
             sum += rows[u];
             valid += raw;
-            kept += a.C > 0 ? min(raw, a.C) : raw;
+            kept += local;
+            dropped += a.C > 0 ? max(raw - a.C, 0) : 0;
         }
         int32_t inc = sum;
 #pragma unroll
@@ -399,22 +412,26 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
         for (int o = 16; o > 0; o >>= 1) {
             valid += __shfl_xor_sync(0xffffffffu, valid, o);
             kept += __shfl_xor_sync(0xffffffffu, kept, o);
+            dropped += __shfl_xor_sync(0xffffffffu, dropped, o);
         }
         if (lane == 31)
             s_wsum[0][warp] = inc;
         if (lane == 0) {
             s_wsum[1][warp] = valid;
             s_wsum[2][warp] = kept;
+            s_wsum[3][warp] = dropped;
         }
         __syncthreads();
         int32_t wpre = 0;
         total_valid = 0;
         total_kept = 0;
+        total_dropped = 0;
 #pragma unroll
         for (int w = 0; w < LAYOUT_WARPS; ++w) {
             wpre += w < warp ? s_wsum[0][w] : 0;
             total_valid += s_wsum[1][w];
             total_kept += s_wsum[2][w];
+            total_dropped += s_wsum[3][w];
         }
         int32_t run = wpre + inc - sum;
 #pragma unroll
@@ -437,7 +454,7 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
         }
         for (int q = tid; q < E; q += LAYOUT_THREADS) {
             o.counts_raw[q] = s_raw[q];
-            o.tokens_per_expert[q] = a.C > 0 ? min(s_raw[q], a.C) : s_raw[q];
+            o.tokens_per_expert[q] = layout_local_tokens(a, s_raw[q]);
         }
         for (int q = tid; q <= E; q += LAYOUT_THREADS)
             o.expert_offsets[q] = s_off[q];
@@ -452,7 +469,7 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
             *o.num_rows = s_off[E];
             o.counters[0] = total_valid;
             o.counters[1] = total_kept;
-            o.counters[2] = total_valid - total_kept;
+            o.counters[2] = total_dropped;
             o.counters[3] = static_cast<int32_t>(a.rows_max - total_kept);
             o.counters[4] = s_off[E];
             o.counters[5] = s_off[E];
@@ -480,8 +497,8 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
                 ord = lo;
             }
             drop = (a.C > 0 && ord >= a.C) ? 1 : 0;
-            if (!drop)
-                dest = s_off[q] + ord;
+            if (!drop && ord % a.T == a.tp_rank) // this peer's share under TP folding
+                dest = s_off[q] + ord / a.T;
             if (dest >= a.rows_max) { // cannot happen for consistent counts; never write out of bounds
                 atomicOr(o.status, MOE_DEV_ROW_RANGE);
                 dest = -1;
@@ -534,9 +551,9 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
         int32_t q;
         bool pad;
         if (a.C > 0) {
-            q = static_cast<int32_t>(row / a.C);
-            const int32_t slot = static_cast<int32_t>(row - static_cast<int64_t>(q) * a.C);
-            pad = slot >= min(s_raw[q], a.C);
+            q = static_cast<int32_t>(row / a.C_local);
+            const int32_t slot = static_cast<int32_t>(row - static_cast<int64_t>(q) * a.C_local);
+            pad = slot >= layout_local_tokens(a, s_raw[q]);
         } else if (row >= num_rows) {
             q = -1;
             pad = true;
@@ -550,7 +567,7 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
                     hi = mid;
             }
             q = lo;
-            pad = row - s_off[q] >= s_raw[q]; // alignment pad after the expert's tokens
+            pad = row - s_off[q] >= layout_local_tokens(a, s_raw[q]); // alignment pad after the expert's tokens
         }
         o.pad_mask[row] = pad ? 1 : 0;
         o.row_local_expert[row] = pad ? -1 : q - (q / a.E_loc) * a.E_loc;

@@ -137,6 +137,8 @@ struct Dims {
     int64_t rows_max = 0;
     int32_t E = 0, E_loc = 0, M = 0, S = 0;
     int32_t A = 1; // row alignment
+    int32_t T = 1; // TP folding peers
+    int32_t C_local = 0;
 };
 
 int check_problem(const moe_problem_t *p, Dims *d)
@@ -150,16 +152,20 @@ int check_problem(const moe_problem_t *p, Dims *d)
         return MOE_ERR_INVALID;
     if ((p->flags & ~MOE_FLAG_TEST_BARRIER_TIMEOUT) != 0)
         return MOE_ERR_INVALID;
-    if (p->row_align < 0)
+    if (p->row_align < 0 || p->tp_size < 0 || p->tp_rank < 0)
         return MOE_ERR_INVALID;
     const int64_t A = p->row_align > 1 ? p->row_align : 1;
-    if (p->capacity > 0 && p->capacity % A != 0)
+    const int64_t T = p->tp_size > 1 ? p->tp_size : 1;
+    if (T > MOE_MAX_TP || p->tp_rank >= T)
+        return MOE_ERR_INVALID;
+    const int64_t C_local = p->capacity > 0 ? (p->capacity + T - 1) / T : 0;
+    if (p->capacity > 0 && C_local % A != 0)
         return MOE_ERR_INVALID;
     const int64_t NK = p->N * static_cast<int64_t>(p->k);
     if (p->N > (int64_t(1) << 40) || NK > INT32_MAX)
         return MOE_ERR_INVALID;
     const int64_t E = static_cast<int64_t>(p->E_log) + p->num_replicas;
-    const int64_t rows_max = p->capacity > 0 ? E * p->capacity : NK + E * (A - 1);
+    const int64_t rows_max = p->capacity > 0 ? E * C_local : (NK + E * (T - 1)) / T + E * (A - 1);
     if (rows_max > INT32_MAX)
         return MOE_ERR_INVALID;
     if (p->k > COMBINE_MAX_K || p->E_log > LAYOUT_MAX_E_LOG)
@@ -175,6 +181,8 @@ int check_problem(const moe_problem_t *p, Dims *d)
     d->M = p->E_log / p->R;
     d->S = p->num_replicas / p->R;
     d->A = static_cast<int32_t>(A);
+    d->T = static_cast<int32_t>(T);
+    d->C_local = static_cast<int32_t>(C_local);
     return MOE_OK;
 }
 
@@ -356,6 +364,9 @@ int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, c
     a.num_replicas = problem->num_replicas;
     a.C = problem->capacity;
     a.A = d.A;
+    a.T = d.T;
+    a.tp_rank = problem->tp_rank;
+    a.C_local = d.C_local;
     a.sub = lg.sub;
     a.G = lg.G;
     a.ws_barrier = static_cast<uint32_t *>(workspace);
@@ -410,6 +421,35 @@ int moe_permute(const moe_problem_t *problem, const moe_layout_t *layout, const 
 
 namespace {
 
+// Grid and launch for the combine kernel; `a` carries everything but the grid
+// shape. PEERS selects the restore variant that gathers from TP peer buffers.
+extern "C++" template <bool PEERS>
+int launch_combine_args(CombineArgs a, int k, void *stream)
+{
+    // the widest CTA (up to 256 threads) that splits the row into equal parts
+    const int v32 = ((a.V + 31) / 32) * 32;
+    const int threads = v32 % 256 == 0 ? 256 : (v32 % 128 == 0 ? 128 : (v32 % 64 == 0 ? 64 : 32));
+    a.nchunks = (a.V + threads - 1) / threads;
+    const int64_t blocks = a.N * a.nchunks;
+    if (blocks > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    const dim3 grid(static_cast<unsigned>(blocks)), block(threads);
+    switch (k) {
+    case 1:
+        return launch(combine_kernel<1, PEERS>, grid, block, 0, stream, false, a);
+    case 2:
+        return launch(combine_kernel<2, PEERS>, grid, block, 0, stream, false, a);
+    case 4:
+        return launch(combine_kernel<4, PEERS>, grid, block, 0, stream, false, a);
+    case 6:
+        return launch(combine_kernel<6, PEERS>, grid, block, 0, stream, false, a);
+    case 8:
+        return launch(combine_kernel<8, PEERS>, grid, block, 0, stream, false, a);
+    default:
+        return launch(combine_kernel<0, PEERS>, grid, block, 0, stream, false, a);
+    }
+}
+
 int launch_combine(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *y, const float *probs,
                    uint16_t *out, void *stream)
 {
@@ -423,7 +463,7 @@ int launch_combine(const moe_problem_t *problem, const moe_layout_t *layout, con
         return MOE_OK;
     if (out == nullptr || !aligned16(out) || (d.rows_max > 0 && (y == nullptr || !aligned16(y))))
         return MOE_ERR_INVALID;
-    CombineArgs a;
+    CombineArgs a = {};
     a.y = reinterpret_cast<const uint4 *>(y);
     a.dest_row = layout->dest_row;
     a.probs = probs;
@@ -433,28 +473,8 @@ int launch_combine(const moe_problem_t *problem, const moe_layout_t *layout, con
     a.rows_max = d.rows_max;
     a.k = problem->k;
     a.V = problem->H / 8;
-    // the widest CTA (up to 256 threads) that splits the row into equal parts
-    const int v32 = ((a.V + 31) / 32) * 32;
-    const int threads = v32 % 256 == 0 ? 256 : (v32 % 128 == 0 ? 128 : (v32 % 64 == 0 ? 64 : 32));
-    a.nchunks = (a.V + threads - 1) / threads;
-    const int64_t blocks = problem->N * a.nchunks;
-    if (blocks > INT32_MAX)
-        return MOE_ERR_UNSUPPORTED;
-    const dim3 grid(static_cast<unsigned>(blocks)), block(threads);
-    switch (problem->k) {
-    case 1:
-        return launch(combine_kernel<1>, grid, block, 0, stream, false, a);
-    case 2:
-        return launch(combine_kernel<2>, grid, block, 0, stream, false, a);
-    case 4:
-        return launch(combine_kernel<4>, grid, block, 0, stream, false, a);
-    case 6:
-        return launch(combine_kernel<6>, grid, block, 0, stream, false, a);
-    case 8:
-        return launch(combine_kernel<8>, grid, block, 0, stream, false, a);
-    default:
-        return launch(combine_kernel<0>, grid, block, 0, stream, false, a);
-    }
+    a.T = 1;
+    return launch_combine_args<false>(a, problem->k, stream);
 }
 
 } // namespace
@@ -469,6 +489,43 @@ int moe_permute_backward(const moe_problem_t *problem, const moe_layout_t *layou
                          uint16_t *grad_hidden, void *stream)
 {
     return launch_combine(problem, layout, grad_send, nullptr, grad_hidden, stream);
+}
+
+int moe_restore_combined(const moe_problem_t *problem, const moe_layout_t *peer_layouts,
+                         const uint16_t *const *peer_expert_out, const float *topk_probs, uint16_t *out, void *stream)
+{
+    Dims d;
+    int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    if (peer_layouts == nullptr || peer_expert_out == nullptr)
+        return MOE_ERR_INVALID;
+    if (static_cast<int64_t>(d.T) * d.rows_max > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    for (int q = 0; q < d.T; ++q) {
+        if ((rc = check_layout(&peer_layouts[q], d, false)) != MOE_OK)
+            return rc;
+        if (d.rows_max > 0 && (peer_expert_out[q] == nullptr || !aligned16(peer_expert_out[q])))
+            return MOE_ERR_INVALID;
+    }
+    if (problem->N == 0)
+        return MOE_OK;
+    if (out == nullptr || !aligned16(out))
+        return MOE_ERR_INVALID;
+    CombineArgs a = {};
+    a.probs = topk_probs;
+    a.out = reinterpret_cast<uint4 *>(out);
+    a.status = peer_layouts[0].status;
+    a.N = problem->N;
+    a.rows_max = d.rows_max;
+    a.k = problem->k;
+    a.V = problem->H / 8;
+    a.T = d.T;
+    for (int q = 0; q < d.T; ++q) {
+        a.ys[q] = reinterpret_cast<const uint4 *>(peer_expert_out[q]);
+        a.dests[q] = peer_layouts[q].dest_row;
+    }
+    return launch_combine_args<true>(a, problem->k, stream);
 }
 
 int moe_combine_backward(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *grad_out,

@@ -22,8 +22,8 @@
  *   read of device data ([Megatron MORI]: sync-free counts and padded buffers).
  * Sizes.  Buffers have fixed upper-bound sizes ([Megatron MORI]: work on the
  *   full [max_tokens, ...] padded buffers and mask the tail). rows_max =
- *   E*capacity when capacity > 0, else N*k + E*(row_align - 1) (N*k without
- *   alignment). N*k and rows_max must be < 2^31.
+ *   E*ceil(capacity/T) when capacity > 0, else (N*k + E*(T-1))/T + E*(row_align - 1)
+ *   (N*k without alignment or TP folding, T = tp_size). N*k and rows_max must be < 2^31.
  * Returns.  MOE_OK or a negative host-detected error; on error nothing is
  *   enqueued. Device-detected problems are OR-ed into *layout->status as
  *   MOE_DEV_* bits; read them when convenient (no call waits for them).
@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-#define MOE_RT_ABI_VERSION 2
+#define MOE_RT_ABI_VERSION 3
 
 /* Every entry point is exported; everything else in the library is hidden. */
 #if defined(__GNUC__)
@@ -83,8 +83,15 @@ typedef struct {
     uint32_t flags;       /* MOE_FLAG_* */
     int32_t row_align;    /* 0 or 1 = none; A > 1: each expert's rows are padded up to a multiple of A
                              ([Megatron MORI]: router padding for FP8 grouped GEMMs). With a capacity,
-                             C must be a multiple of A. */
+                             ceil(C / tp_size) must be a multiple of A. */
+    int32_t tp_size;      /* TP folding ([DeepSpeed EP] partition_assignments): T peers share the
+                             assignments; 0 or 1 = none, at most MOE_MAX_TP */
+    int32_t tp_rank;      /* this peer, 0 <= tp_rank < T. The layout then keeps only the active
+                             assignments whose stable per-expert ordinal o satisfies o % T == tp_rank,
+                             at local ordinal o / T; capacity drops stay global. */
 } moe_problem_t;
+
+#define MOE_MAX_TP 8
 
 /*
  * Outputs of moe_dispatch_layout, all device buffers of the sizes shown
@@ -112,7 +119,8 @@ typedef struct {
     int32_t *output_splits; /* [R] equal to input_splits on one GPU */
     int32_t *rank_offsets;  /* [R+1] first row of each rank */
     /* scalars */
-    int32_t *counters; /* [8] assignments_total, kept, dropped, padded, split_sum_in, split_sum_out, num_rows, error */
+    int32_t *counters; /* [8] assignments_total (valid ids), kept (rows in this buffer; [DeepSpeed EP]
+                          assignments_local), dropped, padded, split_sum_in, split_sum_out, num_rows, error */
     int32_t *num_rows; /* [1] expert_offsets[E] */
     uint32_t *status;  /* [1] MOE_DEV_* bits; the caller zeroes it, calls only OR into it */
     /* per send-buffer row, [rows_max] */
@@ -133,7 +141,7 @@ MOE_API const char *moe_status_string(int code);
 
 /*
  * Number of send-buffer rows (the first dimension of send / expert_out /
- * row_* buffers): E*capacity if capacity > 0, else N*k + E*(row_align - 1). Host only.
+ * row_* buffers), see "Sizes" above. Host only.
  * Returns a negative MOE_ERR_* if the problem is invalid.
  */
 MOE_API int64_t moe_rows_max(const moe_problem_t *problem);
@@ -239,6 +247,24 @@ MOE_API int moe_permute(const moe_problem_t *problem, const moe_layout_t *layout
  */
 MOE_API int moe_combine(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *expert_out,
                 const float *topk_probs, uint16_t *out, void *stream);
+
+/*
+ * Restore after TP folding ([DeepSpeed EP] restore_combined: the peers' weighted
+ * rows are gathered and added back per token one top-k slot at a time in
+ * ascending slot order). On one GPU the gather is the set of peer buffers:
+ * peer q's layout (from moe_dispatch_layout with tp_rank = q) and its expert
+ * output. out[t,h] = bf16_rn( fp32 fmaf chain over ascending j of
+ * p[t,j] * y_q[dest_row_q[t,j], h], q the one peer with dest_row_q[t,j] >= 0 ),
+ * which equals moe_combine of the unfolded layout bit for bit.
+ *   problem          the per-peer problem; tp_size = T peers (tp_rank is ignored)
+ *   peer_layouts     host array of T layouts; reads dest_row and status of each
+ *   peer_expert_out  host array of T device pointers, peer q's [rows_max, H] bf16
+ *   topk_probs       [N, k] fp32 or NULL (unit weights); out [N, H] bf16
+ * Device status bits go to peer 0's status word.
+ */
+MOE_API int moe_restore_combined(const moe_problem_t *problem, const moe_layout_t *peer_layouts,
+                                 const uint16_t *const *peer_expert_out, const float *topk_probs, uint16_t *out,
+                                 void *stream);
 
 /*
  * Backward of permute ([Megatron MORI]: dispatch backward sums the row

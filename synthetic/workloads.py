@@ -14,6 +14,7 @@ Shapes follow the pages' problem statements:
                   skew; forward and backward.
 * ``ht_align16`` — the ``ht`` shape and inputs with every expert's rows padded up to
                   a multiple of 16 (grouped-GEMM / FP8 alignment).
+* ``ht_tp2``    — the ``ht`` shape and inputs folded over 2 TP peers.
 
 Recipe: logits are N(0,1) float32 plus, where a workload is skewed, a per-expert
 bias ``-s ln(rank+1)`` over a seeded ranking of the experts; hidden states and
@@ -51,6 +52,7 @@ class Workload:
     num_replicas: int = 0
     backward: bool = False
     row_align: int = 0
+    tp_size: int = 0
     seed: int = 0x5EED0000
     note: str = field(default="", compare=False)
 
@@ -81,6 +83,7 @@ class Workload:
             num_replicas=self.num_replicas,
             backward=self.backward,
             row_align=self.row_align,
+            tp_size=self.tp_size,
             seed=self.seed,
             note=self.note,
         )
@@ -104,6 +107,8 @@ class Workload:
             d["backward"] = True
         if self.row_align > 1:
             d["row_align"] = self.row_align
+        if self.tp_size > 1:
+            d["tp_size"] = self.tp_size
         return d
 
 
@@ -139,6 +144,9 @@ WORKLOADS = {
         # the 4096-token / e256 / top-8 shape with every expert's rows padded to a
         # multiple of 16 (grouped-GEMM / FP8 alignment); not one of the five configs
         Workload("ht_align16", N=4096, H=7168, E_log=256, k=8, R=4, row_align=16, seed=0x5EED0002),
+        # the same shape folded over 2 TP peers (each peer's layout and send buffer on
+        # this GPU, then one restore over both)
+        Workload("ht_tp2", N=4096, H=7168, E_log=256, k=8, R=4, tp_size=2, seed=0x5EED0002),
     ]
 }
 

@@ -48,6 +48,8 @@ def test_abi_version_and_status_strings(lib):
         (dict(N=0, H=8, k=2, E_log=4, R=2, capacity=3), 12),
         (dict(N=4096, H=7168, k=8, E_log=256, R=4, row_align=16), 32768 + 256 * 15),
         (dict(N=10, H=8, k=2, E_log=4, R=2, capacity=32, row_align=16), 128),
+        (dict(N=100, H=8, k=3, E_log=8, R=2, tp_size=3, tp_rank=1), (300 + 8 * 2) // 3),
+        (dict(N=100, H=8, k=3, E_log=8, R=2, capacity=10, tp_size=3), 8 * 4),
     ],
 )
 def test_rows_max(lib, kw, rows):
@@ -69,6 +71,9 @@ def test_rows_max(lib, kw, rows):
         dict(N=4, H=8, k=1, E_log=4, R=1, flags=0x1),  # unknown flag
         dict(N=4, H=8, k=1, E_log=4, R=1, row_align=-2),
         dict(N=4, H=8, k=1, E_log=4, R=1, capacity=10, row_align=4),  # capacity not a multiple of the alignment
+        dict(N=4, H=8, k=1, E_log=4, R=1, tp_size=2, tp_rank=2),  # rank outside the peers
+        dict(N=4, H=8, k=1, E_log=4, R=1, tp_size=9),  # more peers than MOE_MAX_TP
+        dict(N=4, H=8, k=1, E_log=4, R=1, capacity=10, row_align=8, tp_size=3),  # ceil(10/3) % 8 != 0
     ],
 )
 def test_invalid_problems_rejected(lib, kw):

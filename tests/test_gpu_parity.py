@@ -353,3 +353,45 @@ def test_route_edge_cases(E, k, kind):
     assert np.array_equal(host(gi), idx)
     tol = route_prob_tolerance(logits, idx) * probs.astype(np.float64)
     assert np.all(np.abs(host(gp).astype(np.float64) - probs.astype(np.float64)) <= tol)
+
+
+# ------------------------------------------------------------- TP folding
+
+
+TP_CASES = [
+    # N, H, k, E_log, R, C, reps, align, T
+    (1000, 64, 4, 32, 4, 0, 0, 0, 2),
+    (3000, 40, 2, 16, 2, 256, 0, 0, 4),  # capacity: drops are global, slots ceil(C/T)
+    (2049, 72, 8, 64, 8, 0, 8, 16, 3),  # reroute and alignment
+    (4096, 7168, 8, 256, 4, 0, 0, 0, 2),  # the 4096-token / e256 / top-8 shape
+]
+
+
+@pytest.mark.parametrize("case", TP_CASES, ids=[f"N{c[0]}_E{c[3]}_T{c[8]}" for c in TP_CASES])
+def test_tp_fold_layout_permute_restore(case):
+    N, H, k, E_log, R, C, reps, A, T = case
+    idx, probs, hidden = _small_case(N, H, k, E_log, R, C, reps, 0.05, seed=N + T, zipf=1.3)
+    full = oracle.layout(idx, probs, E_log=E_log, R=R, C=C, num_replicas=reps, align=A)
+    exp_send_full = oracle.permute(hidden, full["dest_row"], full["rows_max"])
+    expect = oracle.combine(exp_send_full, full["dest_row"], probs)
+    layouts, sends, oracle_sends, oracle_dests = [], [], [], []
+    for r in range(T):
+        L = oracle.layout(idx, probs, E_log=E_log, R=R, C=C, num_replicas=reps, align=A, tp_size=T, tp_rank=r)
+        p = moe.Problem(N=N, H=H, k=k, E_log=E_log, R=R, capacity=C, num_replicas=reps, row_align=A,
+                        tp_size=T, tp_rank=r)
+        G = moe.moe_dispatch_layout(p, dev(idx), dev(probs))
+        torch.cuda.synchronize()
+        assert_layout_equal(G, L)
+        send = moe.moe_permute(p, G, dev(hidden))
+        exp_send = oracle.permute(hidden, L["dest_row"], L["rows_max"])
+        assert np.array_equal(host(send), exp_send)
+        layouts.append(G)
+        sends.append(send)
+        oracle_sends.append(exp_send)
+        oracle_dests.append(L["dest_row"])
+    p0 = moe.Problem(N=N, H=H, k=k, E_log=E_log, R=R, capacity=C, num_replicas=reps, row_align=A, tp_size=T)
+    out = moe.moe_restore_combined(p0, layouts, sends, dev(probs))
+    got = host(out)
+    assert np.array_equal(got, oracle.restore_combined(oracle_sends, oracle_dests, probs))
+    assert np.array_equal(got, expect)  # restore over all peers = the unfolded combine
+    assert all(G.status() == 0 for G in layouts)
