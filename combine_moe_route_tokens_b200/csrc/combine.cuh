@@ -83,42 +83,45 @@ __device__ __forceinline__ void load_slot_meta(const int32_t *dest_row, const fl
 }
 
 // Restore after TP folding: slot j of token t lives in the one peer buffer whose
-// row map has a row for it. Lane j < k finds that peer and folds it into the
-// row index as peer * rows_max + row (peer_row() undoes it).
-__device__ __forceinline__ void load_slot_meta_peers(const CombineArgs &a, int64_t t, int k, int32_t &d, float &p)
+// row map has a row for it. Lane j < k finds that peer (src) and the row (d).
+__device__ __forceinline__ void load_slot_meta_peers(const CombineArgs &a, int64_t t, int k, int32_t &d, float &p,
+                                                     int32_t &src)
 {
     const int lane = threadIdx.x & 31;
     d = -1;
     p = 0.0f;
+    src = 0;
     if (lane < k) {
         p = a.probs != nullptr ? __ldg(a.probs + t * k + lane) : 1.0f;
-        for (int q = 0; q < a.T; ++q) {
-            const int32_t r = __ldg(a.dests[q] + t * k + lane);
-            if (r < -1 || r >= a.rows_max) {
+        int32_t r[MOE_MAX_TP];
+#pragma unroll
+        for (int q = 0; q < MOE_MAX_TP; ++q)
+            r[q] = q < a.T ? __ldg(a.dests[q] + t * k + lane) : -1;
+#pragma unroll
+        for (int q = 0; q < MOE_MAX_TP; ++q) {
+            if (r[q] < -1 || r[q] >= a.rows_max) {
                 atomicOr(a.status, MOE_DEV_ROW_RANGE);
-                continue;
+            } else if (r[q] >= 0 && d < 0) {
+                d = r[q];
+                src = q;
             }
-            if (r >= 0 && d < 0)
-                d = static_cast<int32_t>(q * a.rows_max + r);
         }
     }
 }
 
-__device__ __forceinline__ const uint4 *peer_row(const CombineArgs &a, int32_t folded)
+__device__ __forceinline__ const uint4 *peer_base(const CombineArgs &a, int32_t src)
 {
-    const int q = static_cast<int>(folded / a.rows_max);
-    const int64_t r = folded - static_cast<int64_t>(q) * a.rows_max;
     const uint4 *base = a.ys[0];
 #pragma unroll
     for (int i = 1; i < MOE_MAX_TP; ++i)
-        base = (q == i) ? a.ys[i] : base;
-    return base + r * a.V;
+        base = (src == i) ? a.ys[i] : base;
+    return base;
 }
 
 // K > 0: top-k fixed at compile time; K == 0: runtime k <= 32.
 // PEERS: gather from the TP peers' buffers (restore) instead of one buffer.
 template <int K, bool PEERS = false>
-__global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(CombineArgs a)
+__global__ void __launch_bounds__(COMBINE_THREADS, 4) combine_kernel(CombineArgs a)
 {
     pdl_trigger();
     pdl_wait();
@@ -127,15 +130,15 @@ __global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(CombineArgs a)
     const int v = c * blockDim.x + threadIdx.x;
     const int k = K > 0 ? K : a.k;
 
-    int32_t d;
+    int32_t d, src = 0;
     float p;
     if constexpr (PEERS)
-        load_slot_meta_peers(a, t, k, d, p);
+        load_slot_meta_peers(a, t, k, d, p, src);
     else
         load_slot_meta(a.dest_row, a.probs, t, k, a.rows_max, a.status, d, p);
-    auto row_ptr = [&](int32_t row) -> const uint4 * {
+    auto row_ptr = [&](int32_t row, int32_t peer) -> const uint4 * {
         if constexpr (PEERS)
-            return peer_row(a, row);
+            return peer_base(a, peer) + static_cast<int64_t>(row) * a.V;
         else
             return a.y + static_cast<int64_t>(row) * a.V;
     };
@@ -146,20 +149,21 @@ __global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(CombineArgs a)
         acc[e] = 0.0f;
 
     if constexpr (K > 0) {
-        int32_t dj[K];
+        int32_t dj[K], sj[K];
         float pj[K];
         uint4 yj[K];
 #pragma unroll
         for (int j = 0; j < K; ++j) {
             dj[j] = __shfl_sync(0xffffffffu, d, j);
             pj[j] = __shfl_sync(0xffffffffu, p, j);
+            sj[j] = PEERS ? __shfl_sync(0xffffffffu, src, j) : 0;
         }
         if (v >= a.V)
             return;
 #pragma unroll
         for (int j = 0; j < K; ++j)
             if (dj[j] >= 0)
-                yj[j] = ld_stream_u4(row_ptr(dj[j]) + v);
+                yj[j] = ld_stream_u4(row_ptr(dj[j], sj[j]) + v);
 #pragma unroll
         for (int j = 0; j < K; ++j)
             if (dj[j] >= 0)
@@ -167,20 +171,21 @@ __global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(CombineArgs a)
     } else {
         const bool active = v < a.V;
         for (int j0 = 0; j0 < k; j0 += 4) {
-            int32_t dj[4];
+            int32_t dj[4], sj[4];
             float pj[4];
             uint4 yj[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 dj[u] = __shfl_sync(0xffffffffu, d, (j0 + u) & 31);
                 pj[u] = __shfl_sync(0xffffffffu, p, (j0 + u) & 31);
+                sj[u] = PEERS ? __shfl_sync(0xffffffffu, src, (j0 + u) & 31) : 0;
                 if (j0 + u >= k || !active)
                     dj[u] = -1;
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u)
                 if (dj[u] >= 0)
-                    yj[u] = ld_stream_u4(row_ptr(dj[u]) + v);
+                    yj[u] = ld_stream_u4(row_ptr(dj[u], sj[u]) + v);
 #pragma unroll
             for (int u = 0; u < 4; ++u)
                 if (dj[u] >= 0)

@@ -500,8 +500,6 @@ int moe_restore_combined(const moe_problem_t *problem, const moe_layout_t *peer_
         return rc;
     if (peer_layouts == nullptr || peer_expert_out == nullptr)
         return MOE_ERR_INVALID;
-    if (static_cast<int64_t>(d.T) * d.rows_max > INT32_MAX)
-        return MOE_ERR_UNSUPPORTED;
     for (int q = 0; q < d.T; ++q) {
         if ((rc = check_layout(&peer_layouts[q], d, false)) != MOE_OK)
             return rc;
