@@ -15,6 +15,8 @@ from .oracle import (
     permute,
     combine,
     restore_combined,
+    dedup_layout,
+    dedup_combine_local,
     permute_backward,
     combine_backward,
     bf16_from_f32,
@@ -31,6 +33,8 @@ __all__ = [
     "permute",
     "combine",
     "restore_combined",
+    "dedup_layout",
+    "dedup_combine_local",
     "permute_backward",
     "combine_backward",
     "bf16_from_f32",

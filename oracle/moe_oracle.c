@@ -375,6 +375,124 @@ int oracle_layout(const oracle_problem *p, const int32_t *topk_idx, const float 
     return 0;
 }
 
+/* --------------------------------------------------------------- dedup ---- */
+
+/*
+ * DeepEP-style dispatch layout ([Megatron MORI]: the DeepEP contract the MORI
+ * dispatcher follows; the receiver gets each token once, its local top-k ids
+ * with -1 sentinels and receiver-side weights, and _indices_to_multihot turns
+ * those into a [tokens, local experts] routing map with probs).
+ * Rank r receives token t iff some kept slot j of t (dest_row >= 0) has a
+ * physical expert on r. Rows are rank-major and token-ascending within a rank:
+ *   token_rank_row[t,r] = recv_rank_offsets[r] + #{t' < t received by r}.
+ * At most min(k, R) rows per token: recv_max = N * min(k, R).
+ */
+int64_t oracle_dedup_rows_max(const oracle_problem *p)
+{
+    int64_t m = p->k < p->R ? p->k : p->R;
+    return p->N * m;
+}
+
+int oracle_dedup_layout(const oracle_problem *p, const int32_t *phys_idx, const int32_t *dest_row,
+                        const float *topk_probs, const oracle_dedup_out *o)
+{
+    if (!oracle_problem_valid(p))
+        return -1;
+    const int64_t N = p->N;
+    const int32_t k = p->k, R = p->R;
+    const int32_t E_loc = oracle_num_experts(p) / R;
+    const int64_t recv_max = oracle_dedup_rows_max(p);
+    /* is_token_in_rank and the per-rank token counts */
+    for (int32_t r = 0; r < R; ++r)
+        o->num_tokens_per_rank[r] = 0;
+    for (int64_t t = 0; t < N; ++t)
+        for (int32_t r = 0; r < R; ++r) {
+            uint8_t in = 0;
+            for (int32_t j = 0; j < k; ++j)
+                if (dest_row[t * k + j] >= 0 && phys_idx[t * k + j] / E_loc == r)
+                    in = 1;
+            o->is_token_in_rank[t * R + r] = in;
+            o->num_tokens_per_rank[r] += in;
+        }
+    o->recv_rank_offsets[0] = 0;
+    for (int32_t r = 0; r < R; ++r)
+        o->recv_rank_offsets[r + 1] = o->recv_rank_offsets[r] + o->num_tokens_per_rank[r];
+    *o->num_recv = o->recv_rank_offsets[R];
+    /* every receive row starts as a tail row: token -1, ids -1, weights / map / probs 0 */
+    for (int64_t row = 0; row < recv_max; ++row) {
+        o->recv_src_token[row] = -1;
+        o->recv_pad_mask[row] = 1;
+        for (int32_t j = 0; j < k; ++j) {
+            o->recv_topk_idx[row * k + j] = -1;
+            o->recv_topk_weights[row * k + j] = 0.0f;
+        }
+        for (int32_t e = 0; e < E_loc; ++e) {
+            o->recv_routing_map[row * E_loc + e] = 0;
+            o->recv_probs[row * E_loc + e] = 0.0f;
+        }
+    }
+    /* rank-major rows, tokens in ascending order within a rank */
+    for (int32_t r = 0; r < R; ++r) {
+        int32_t next = o->recv_rank_offsets[r];
+        for (int64_t t = 0; t < N; ++t) {
+            if (!o->is_token_in_rank[t * R + r]) {
+                o->token_rank_row[t * R + r] = -1;
+                continue;
+            }
+            int32_t row = next++;
+            o->token_rank_row[t * R + r] = row;
+            o->recv_src_token[row] = (int32_t)t;
+            o->recv_pad_mask[row] = 0;
+            for (int32_t j = 0; j < k; ++j) {
+                int32_t q = phys_idx[t * k + j];
+                if (dest_row[t * k + j] < 0 || q / E_loc != r)
+                    continue;
+                int32_t local = q - r * E_loc;
+                float w = topk_probs ? topk_probs[t * k + j] : 0.0f;
+                o->recv_topk_idx[(int64_t)row * k + j] = local;
+                o->recv_topk_weights[(int64_t)row * k + j] = w;
+                /* _indices_to_multihot: a set bit per local expert, its prob beside it */
+                o->recv_routing_map[(int64_t)row * E_loc + local] = 1;
+                o->recv_probs[(int64_t)row * E_loc + local] = w;
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Receiver side of the DeepEP-style combine: each rank reduces, per received
+ * token, the weighted outputs of the token's kept slots whose row lies in that
+ * rank's part of the send buffer, in ascending slot order, fp32 fused
+ * multiply-add from +0, rounded once to bf16. Tail rows are 0. The sender then
+ * sums the partials over ranks (the unit-weight combine over token_rank_row).
+ */
+void oracle_dedup_combine_local(const oracle_problem *p, int32_t H, int64_t recv_max, const int32_t *dest_row,
+                                const int32_t *rank_offsets, const int32_t *recv_src_token,
+                                const int32_t *recv_rank_offsets, const uint16_t *expert_out,
+                                const float *topk_probs, uint16_t *partial)
+{
+    for (int64_t row = 0; row < recv_max; ++row) {
+        int32_t t = recv_src_token[row];
+        int32_t r = -1;
+        for (int32_t q = 0; q < p->R; ++q)
+            if (row >= recv_rank_offsets[q] && row < recv_rank_offsets[q + 1])
+                r = q;
+        for (int32_t h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            if (t >= 0 && r >= 0)
+                for (int32_t j = 0; j < p->k; ++j) {
+                    int32_t d = dest_row[(int64_t)t * p->k + j];
+                    if (d < rank_offsets[r] || d >= rank_offsets[r + 1])
+                        continue;
+                    float w = topk_probs ? topk_probs[(int64_t)t * p->k + j] : 1.0f;
+                    acc = fmaf(w, oracle_f32_from_bf16(expert_out[(int64_t)d * H + h]), acc);
+                }
+            partial[row * H + h] = oracle_bf16_from_f32(acc);
+        }
+    }
+}
+
 /* ------------------------------------------------------------- permute ---- */
 
 /*

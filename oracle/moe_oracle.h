@@ -97,6 +97,29 @@ void oracle_combine_backward(const oracle_problem *p, int32_t H, int64_t rows_ma
                              const int32_t *row_token, const float *row_prob, const uint16_t *grad_out,
                              const uint16_t *expert_out, uint16_t *grad_expert_out, float *grad_probs);
 
+/* DeepEP-style token-dedup view (one row per (token, rank) with any kept slot on the rank). */
+typedef struct {
+    int32_t *num_tokens_per_rank; /* [R] */
+    int32_t *recv_rank_offsets;   /* [R+1] */
+    int32_t *num_recv;            /* [1] */
+    uint8_t *is_token_in_rank;    /* [N*R] */
+    int32_t *token_rank_row;      /* [N*R] */
+    int32_t *recv_src_token;      /* [recv_max] */
+    int32_t *recv_topk_idx;       /* [recv_max*k] */
+    float *recv_topk_weights;     /* [recv_max*k] */
+    uint8_t *recv_routing_map;    /* [recv_max*E_loc] */
+    float *recv_probs;            /* [recv_max*E_loc] */
+    uint8_t *recv_pad_mask;       /* [recv_max] */
+} oracle_dedup_out;
+
+int64_t oracle_dedup_rows_max(const oracle_problem *p);
+int oracle_dedup_layout(const oracle_problem *p, const int32_t *phys_idx, const int32_t *dest_row,
+                        const float *topk_probs, const oracle_dedup_out *o);
+void oracle_dedup_combine_local(const oracle_problem *p, int32_t H, int64_t recv_max, const int32_t *dest_row,
+                                const int32_t *rank_offsets, const int32_t *recv_src_token,
+                                const int32_t *recv_rank_offsets, const uint16_t *expert_out,
+                                const float *topk_probs, uint16_t *partial);
+
 uint16_t oracle_bf16_from_f32(float x);
 float oracle_f32_from_bf16(uint16_t b);
 

@@ -104,6 +104,22 @@ class _LayoutOut(ctypes.Structure):
     ]
 
 
+class _DedupOut(ctypes.Structure):
+    _fields_ = [
+        ("num_tokens_per_rank", _P),
+        ("recv_rank_offsets", _P),
+        ("num_recv", _P),
+        ("is_token_in_rank", _P),
+        ("token_rank_row", _P),
+        ("recv_src_token", _P),
+        ("recv_topk_idx", _P),
+        ("recv_topk_weights", _P),
+        ("recv_routing_map", _P),
+        ("recv_probs", _P),
+        ("recv_pad_mask", _P),
+    ]
+
+
 _lib_handle: Optional[ctypes.CDLL] = None
 
 
@@ -144,6 +160,13 @@ def _lib() -> ctypes.CDLL:
             _P,
             _P,
         ]
+        lib.oracle_dedup_rows_max.restype = ctypes.c_int64
+        lib.oracle_dedup_rows_max.argtypes = [ctypes.POINTER(_Problem)]
+        lib.oracle_dedup_layout.restype = ctypes.c_int
+        lib.oracle_dedup_layout.argtypes = [ctypes.POINTER(_Problem), _P, _P, _P, ctypes.POINTER(_DedupOut)]
+        lib.oracle_dedup_combine_local.restype = None
+        lib.oracle_dedup_combine_local.argtypes = [ctypes.POINTER(_Problem), ctypes.c_int32, ctypes.c_int64, _P, _P,
+                                                   _P, _P, _P, _P, _P]
         lib.oracle_bf16_from_f32.restype = ctypes.c_uint16
         lib.oracle_bf16_from_f32.argtypes = [ctypes.c_float]
         _lib_handle = lib
@@ -241,6 +264,59 @@ def layout(topk_idx: np.ndarray, topk_probs: Optional[np.ndarray], *, E_log: int
     out["rows_max"] = RM
     out["E"] = E
     return out
+
+
+def dedup_layout(L: dict, topk_probs: Optional[np.ndarray], *, E_log: int, R: int, num_replicas: int = 0) -> dict:
+    """DeepEP-style one-row-per-(token, rank) view of a layout (see moe_oracle.c)."""
+    phys = _c(L["phys_idx"], np.int32)
+    dest = _c(L["dest_row"], np.int32)
+    N, k = phys.shape
+    p = _Problem(N=N, k=k, E_log=E_log, num_replicas=num_replicas, R=R, C=0)
+    lib = _lib()
+    RM = int(lib.oracle_dedup_rows_max(ctypes.byref(p)))
+    E_loc = (E_log + num_replicas) // R
+    probs = None if topk_probs is None else _c(topk_probs, np.float32)
+    out = {
+        "num_tokens_per_rank": np.empty(R, np.int32),
+        "recv_rank_offsets": np.empty(R + 1, np.int32),
+        "num_recv": np.empty(1, np.int32),
+        "is_token_in_rank": np.empty(N * R, np.uint8),
+        "token_rank_row": np.empty(N * R, np.int32),
+        "recv_src_token": np.empty(RM, np.int32),
+        "recv_topk_idx": np.empty(RM * k, np.int32),
+        "recv_topk_weights": np.empty(RM * k, np.float32),
+        "recv_routing_map": np.empty(RM * E_loc, np.uint8),
+        "recv_probs": np.empty(RM * E_loc, np.float32),
+        "recv_pad_mask": np.empty(RM, np.uint8),
+    }
+    o = _DedupOut(**{name: _ptr(arr) for name, arr in out.items()})
+    if lib.oracle_dedup_layout(ctypes.byref(p), _ptr(phys), _ptr(dest), _ptr(probs), ctypes.byref(o)) != 0:
+        raise ValueError("oracle_dedup_layout rejected the problem")
+    out["is_token_in_rank"] = out["is_token_in_rank"].reshape(N, R)
+    out["token_rank_row"] = out["token_rank_row"].reshape(N, R)
+    out["recv_topk_idx"] = out["recv_topk_idx"].reshape(RM, k)
+    out["recv_topk_weights"] = out["recv_topk_weights"].reshape(RM, k)
+    out["recv_routing_map"] = out["recv_routing_map"].reshape(RM, E_loc)
+    out["recv_probs"] = out["recv_probs"].reshape(RM, E_loc)
+    out["recv_max"] = RM
+    return out
+
+
+def dedup_combine_local(expert_out: np.ndarray, L: dict, D: dict, topk_probs: Optional[np.ndarray], R: int) -> np.ndarray:
+    """Receiver-side partial per (token, rank) row (see moe_oracle.c)."""
+    expert_out = _c(expert_out, np.uint16)
+    dest = _c(L["dest_row"], np.int32)
+    N, k = dest.shape
+    H = expert_out.shape[1]
+    RM = D["recv_max"]
+    probs = None if topk_probs is None else _c(topk_probs, np.float32)
+    p = _Problem(N=N, k=k, E_log=R, num_replicas=0, R=R, C=0)
+    partial = np.empty((RM, H), np.uint16)
+    _lib().oracle_dedup_combine_local(ctypes.byref(p), H, RM, _ptr(dest), _ptr(_c(L["rank_offsets"], np.int32)),
+                                      _ptr(_c(D["recv_src_token"], np.int32)),
+                                      _ptr(_c(D["recv_rank_offsets"], np.int32)), _ptr(expert_out), _ptr(probs),
+                                      _ptr(partial))
+    return partial
 
 
 def permute(hidden: np.ndarray, dest_row: np.ndarray, rows_max: int) -> np.ndarray:
