@@ -208,6 +208,11 @@ class Step:
             self.gy = torch.empty((RM, H), dtype=torch.bfloat16, device=device)
             self.gp = torch.empty((N, k), dtype=torch.float32, device=device)
             self.gh = torch.empty((N, H), dtype=torch.bfloat16, device=device)
+        if w.dedup:
+            self.dedup = moe.DedupView.allocate(p, device)
+            self._D = self.dedup.c_struct()
+            self.recv_x = torch.empty((self.dedup.recv_max, H), dtype=torch.bfloat16, device=device)
+            self.partial = torch.empty((self.dedup.recv_max, H), dtype=torch.bfloat16, device=device)
         self._ps = [q.c_struct() for q in self.problems]
         self._Ls = [L.c_struct() for L in self.layouts]
         self._L_arr = (native.MoeLayout * T)(*self._Ls)
@@ -220,7 +225,21 @@ class Step:
         for s in sets:
             c = [("route", self.lib.moe_route_topk,
                   (vp(s["logits"]), None, N, w.E_log, k, vp(self.idx), vp(self.probs), self._s))]
-            if T == 1:
+            if T == 1 and w.dedup:
+                ws = self.layout.workspace
+                D = ctypes.byref(self._D)
+                c += [
+                    ("layout", self.lib.moe_dispatch_layout,
+                     (P, vp(self.idx), vp(self.probs), L, vp(ws), ws.numel(), self._s)),
+                    ("dedup_layout", self.lib.moe_dedup_layout,
+                     (P, L, vp(self.probs), D, vp(self.dedup.workspace), self.dedup.workspace.numel(), self._s)),
+                    ("dedup_dispatch", self.lib.moe_dedup_dispatch, (P, D, vp(s["hidden"]), vp(self.recv_x), self._s)),
+                    ("permute", self.lib.moe_permute, (P, L, vp(s["hidden"]), vp(self.send), self._s)),
+                    ("dedup_combine_local", self.lib.moe_dedup_combine_local,
+                     (P, L, D, vp(self.send), vp(self.probs), vp(self.partial), self._s)),
+                    ("dedup_combine", self.lib.moe_dedup_combine, (P, D, vp(self.partial), vp(self.out), self._s)),
+                ]
+            elif T == 1:
                 ws = self.layout.workspace
                 c += [
                     ("layout", self.lib.moe_dispatch_layout,
@@ -262,6 +281,8 @@ class Step:
         st = 0
         for L in self.layouts:
             st |= L.status()
+        if self.w.dedup:
+            st |= self.dedup.status()
         return st
 
     def algorithmic_bytes(self) -> dict:
@@ -285,6 +306,13 @@ class Step:
                 out[f"layout.{r}"] = layout_bytes
                 out[f"permute.{r}"] = read[r] * row + RM * row + NK * 4 + RM
             out["restore"] = sum(kept) * row + N * row + NK * 4 * (T + 1)
+        if w.dedup:
+            RR = self.dedup.recv_max
+            nrecv = int(self.dedup["num_recv"].item())
+            out["dedup_layout"] = NK * 8 + NK * 4 + N * w.R * 5 + RR * (4 + 1 + k * 8 + (w.R and (E // w.R)) * 5)
+            out["dedup_dispatch"] = read[0] * row + RR * row + N * w.R * 4 + RR
+            out["dedup_combine_local"] = kept[0] * row + RR * row + NK * 8 + RR * 4
+            out["dedup_combine"] = nrecv * row + N * row + N * w.R * 4
         out["combine_backward"] = N * row + kept[0] * row + RM * row + NK * 8 + NK * 4
         out["permute_backward"] = kept[0] * row + N * row + NK * 4
         return out
@@ -484,7 +512,12 @@ def oracle_step(oracle, w, d):
         layouts.append(L)
         sends.append(oracle.permute(d["hidden"], L["dest_row"], L["rows_max"]))
     L, send = layouts[0], sends[0]
-    if T == 1:
+    if T == 1 and w.dedup:
+        D = oracle.dedup_layout(L, probs, E_log=w.E_log, R=w.R, num_replicas=w.num_replicas)
+        oracle.permute(d["hidden"], D["token_rank_row"], D["recv_max"])
+        partial = oracle.dedup_combine_local(send, L, D, probs, w.R)
+        out = oracle.combine(partial, D["token_rank_row"], None)
+    elif T == 1:
         out = oracle.combine(send, L["dest_row"], probs)
     else:
         out = oracle.restore_combined(sends, [x["dest_row"] for x in layouts], probs)

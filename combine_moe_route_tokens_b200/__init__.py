@@ -9,6 +9,7 @@ functions keep the C names:
     moe_permute           send[dest_row[t, j]] = hidden[t]
     moe_combine           out[t] = bf16(sum_j p[t, j] * y[dest_row[t, j]]), fp32, ascending j
     moe_restore_combined  the same over the buffers of TP peers (after TP folding)
+    moe_dedup_*           DeepEP-style view: one receive row per (token, rank), two-level combine
     moe_permute_backward  grad_hidden[t] = bf16(sum_j grad_send[dest_row[t, j]])
     moe_combine_backward  grad_y[row] = bf16(p * grad_out[t]); grad_probs[t, j] = <grad_out[t], y[row]>
 
@@ -56,6 +57,11 @@ __all__ = [
     "moe_permute",
     "moe_combine",
     "moe_restore_combined",
+    "DedupView",
+    "moe_dedup_layout",
+    "moe_dedup_dispatch",
+    "moe_dedup_combine_local",
+    "moe_dedup_combine",
     "moe_permute_backward",
     "moe_combine_backward",
     "load_library",
@@ -222,6 +228,127 @@ class Layout:
     def counters(self) -> Dict[str, int]:
         """dispatch_counters as a dict. Synchronises."""
         return dict(zip(COUNTER_NAMES, (int(v) for v in self.tensors["counters"].tolist())))
+
+
+@dataclass
+class DedupView:
+    """Device buffers of the DeepEP-style token-dedup view plus its workspace."""
+
+    problem: Problem
+    tensors: Dict[str, torch.Tensor] = field(default_factory=dict)
+    workspace: Optional[torch.Tensor] = None
+
+    @property
+    def recv_max(self) -> int:
+        p = self.problem.c_struct()
+        v = _native.lib().moe_dedup_rows_max(ctypes.byref(p))
+        if v < 0:
+            _native.check("moe_dedup_rows_max", int(v))
+        return int(v)
+
+    @classmethod
+    def allocate(cls, problem: Problem, device=None) -> "DedupView":
+        device = torch.device("cuda") if device is None else torch.device(device)
+        view = cls(problem=problem)
+        N, k, R = problem.N, problem.k, problem.R
+        E_loc = problem.E_loc
+        RM = view.recv_max
+        i32, f32, u8 = torch.int32, torch.float32, torch.uint8
+        view.tensors = {
+            "num_tokens_per_rank": torch.empty(R, dtype=i32, device=device),
+            "recv_rank_offsets": torch.empty(R + 1, dtype=i32, device=device),
+            "num_recv": torch.empty(1, dtype=i32, device=device),
+            "is_token_in_rank": torch.empty((N, R), dtype=u8, device=device),
+            "token_rank_row": torch.empty((N, R), dtype=i32, device=device),
+            "recv_src_token": torch.empty(RM, dtype=i32, device=device),
+            "recv_topk_idx": torch.empty((RM, k), dtype=i32, device=device),
+            "recv_topk_weights": torch.empty((RM, k), dtype=f32, device=device),
+            "recv_routing_map": torch.empty((RM, E_loc), dtype=u8, device=device),
+            "recv_probs": torch.empty((RM, E_loc), dtype=f32, device=device),
+            "recv_pad_mask": torch.empty(RM, dtype=u8, device=device),
+            "status": torch.zeros(1, dtype=i32, device=device),
+        }
+        n = ctypes.c_size_t(0)
+        pc = problem.c_struct()
+        _native.check("moe_dedup_workspace_bytes",
+                      _native.lib().moe_dedup_workspace_bytes(ctypes.byref(pc), ctypes.byref(n)))
+        view.workspace = torch.zeros(int(n.value), dtype=u8, device=device)
+        return view
+
+    def __getitem__(self, name: str) -> torch.Tensor:
+        return self.tensors[name]
+
+    def c_struct(self) -> _native.MoeDedup:
+        return _native.MoeDedup(**{name: self.tensors[name].data_ptr() for name in _native.DEDUP_FIELDS})
+
+    def status(self) -> int:
+        return int(self.tensors["status"].item()) & 0xFFFFFFFF
+
+
+def moe_dedup_layout(problem: Problem, layout: Layout, topk_probs: Optional[torch.Tensor],
+                     dedup: Optional[DedupView] = None, stream=None) -> DedupView:
+    """DeepEP-style view (one receive row per (token, rank)) of a dispatch layout."""
+    if dedup is None:
+        dedup = DedupView.allocate(problem, layout.device)
+    if topk_probs is not None:
+        _need(topk_probs, "topk_probs", torch.float32, (problem.N, problem.k), layout.device)
+    p = problem.c_struct()
+    L = layout.c_struct()
+    D = dedup.c_struct()
+    _native.check("moe_dedup_layout",
+                  _native.lib().moe_dedup_layout(ctypes.byref(p), ctypes.byref(L), _ptr(topk_probs), ctypes.byref(D),
+                                                 _ptr(dedup.workspace), dedup.workspace.numel(), _stream(stream)))
+    return dedup
+
+
+def moe_dedup_dispatch(problem: Problem, dedup: DedupView, hidden: torch.Tensor,
+                       recv_x: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """recv_x[token_rank_row[t, r]] = hidden[t]; tail rows zero."""
+    _need(hidden, "hidden", torch.bfloat16, (problem.N, problem.H))
+    if recv_x is None:
+        recv_x = torch.empty((dedup.recv_max, problem.H), dtype=torch.bfloat16, device=hidden.device)
+    _need(recv_x, "recv_x", torch.bfloat16, (dedup.recv_max, problem.H), hidden.device)
+    p = problem.c_struct()
+    D = dedup.c_struct()
+    _native.check("moe_dedup_dispatch",
+                  _native.lib().moe_dedup_dispatch(ctypes.byref(p), ctypes.byref(D), _ptr(hidden), _ptr(recv_x),
+                                                   _stream(stream)))
+    return recv_x
+
+
+def moe_dedup_combine_local(problem: Problem, layout: Layout, dedup: DedupView, expert_out: torch.Tensor,
+                            topk_probs: Optional[torch.Tensor], partial: Optional[torch.Tensor] = None,
+                            stream=None) -> torch.Tensor:
+    """Receiver-side partial per receive row (fp32 chain over the row's local slots, one bf16 rounding)."""
+    _need(expert_out, "expert_out", torch.bfloat16, (problem.rows_max, problem.H), layout.device)
+    if topk_probs is not None:
+        _need(topk_probs, "topk_probs", torch.float32, (problem.N, problem.k), layout.device)
+    if partial is None:
+        partial = torch.empty((dedup.recv_max, problem.H), dtype=torch.bfloat16, device=layout.device)
+    _need(partial, "partial", torch.bfloat16, (dedup.recv_max, problem.H), layout.device)
+    p = problem.c_struct()
+    L = layout.c_struct()
+    D = dedup.c_struct()
+    _native.check("moe_dedup_combine_local",
+                  _native.lib().moe_dedup_combine_local(ctypes.byref(p), ctypes.byref(L), ctypes.byref(D),
+                                                        _ptr(expert_out), _ptr(topk_probs), _ptr(partial),
+                                                        _stream(stream)))
+    return partial
+
+
+def moe_dedup_combine(problem: Problem, dedup: DedupView, partial: torch.Tensor, out: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """out[t] = bf16(fp32 sum over ascending r of partial[token_rank_row[t, r]])."""
+    _need(partial, "partial", torch.bfloat16, (dedup.recv_max, problem.H))
+    if out is None:
+        out = torch.empty((problem.N, problem.H), dtype=torch.bfloat16, device=partial.device)
+    _need(out, "out", torch.bfloat16, (problem.N, problem.H), partial.device)
+    p = problem.c_struct()
+    D = dedup.c_struct()
+    _native.check("moe_dedup_combine",
+                  _native.lib().moe_dedup_combine(ctypes.byref(p), ctypes.byref(D), _ptr(partial), _ptr(out),
+                                                  _stream(stream)))
+    return out
 
 
 def moe_route_topk(logits: torch.Tensor, k: int, token_mask: Optional[torch.Tensor] = None,

@@ -24,6 +24,7 @@ MOE_ERR_CUDA = -3
 MOE_ERR_SCRATCH_LIMIT = -4
 MOE_NOALLOC_MAX_E_LOG = 512
 MOE_MAX_TP = 8
+MOE_MAX_DEDUP_RANKS = 32
 
 MOE_DEV_EXPERT_RANGE = 0x1
 MOE_DEV_TIMEOUT = 0x2
@@ -32,7 +33,7 @@ MOE_DEV_ROW_RANGE = 0x4
 MOE_FLAG_NONE = 0
 MOE_FLAG_TEST_BARRIER_TIMEOUT = 0x80000000
 
-ABI_VERSION = 3
+ABI_VERSION = 4
 
 
 class MoeProblem(ctypes.Structure):
@@ -80,6 +81,26 @@ class MoeLayout(ctypes.Structure):
     _fields_ = [(name, ctypes.c_void_p) for name in LAYOUT_FIELDS]
 
 
+DEDUP_FIELDS = (
+    "num_tokens_per_rank",
+    "recv_rank_offsets",
+    "num_recv",
+    "is_token_in_rank",
+    "token_rank_row",
+    "recv_src_token",
+    "recv_topk_idx",
+    "recv_topk_weights",
+    "recv_routing_map",
+    "recv_probs",
+    "recv_pad_mask",
+    "status",
+)
+
+
+class MoeDedup(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in DEDUP_FIELDS]
+
+
 class MoeError(RuntimeError):
     def __init__(self, fn: str, code: int, text: str):
         super().__init__(f"{fn} failed: {code} ({text})")
@@ -91,6 +112,7 @@ _lib: Optional[ctypes.CDLL] = None
 _VP = ctypes.c_void_p
 _PP = ctypes.POINTER(MoeProblem)
 _PL = ctypes.POINTER(MoeLayout)
+_PD = ctypes.POINTER(MoeDedup)
 
 _SIGNATURES = {
     "moe_abi_version": (ctypes.c_int, []),
@@ -105,6 +127,12 @@ _SIGNATURES = {
     "moe_restore_combined": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP]),
     "moe_permute_backward": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP]),
     "moe_combine_backward": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "moe_dedup_rows_max": (ctypes.c_int64, [_PP]),
+    "moe_dedup_workspace_bytes": (ctypes.c_int, [_PP, ctypes.POINTER(ctypes.c_size_t)]),
+    "moe_dedup_layout": (ctypes.c_int, [_PP, _PL, _VP, _PD, _VP, ctypes.c_size_t, _VP]),
+    "moe_dedup_dispatch": (ctypes.c_int, [_PP, _PD, _VP, _VP, _VP]),
+    "moe_dedup_combine_local": (ctypes.c_int, [_PP, _PL, _PD, _VP, _VP, _VP, _VP]),
+    "moe_dedup_combine": (ctypes.c_int, [_PP, _PD, _VP, _VP, _VP]),
 }
 
 

@@ -120,6 +120,8 @@ __device__ __forceinline__ bool layout_grid_barrier(uint32_t *bar, uint32_t targ
 __device__ __forceinline__ int32_t layout_local_tokens(const LayoutArgs &a, int32_t raw)
 {
     const int32_t t = a.C > 0 ? min(raw, a.C) : raw;
+    if (a.T == 1) // no folding: skip the division
+        return t;
     return t > a.tp_rank ? (t - a.tp_rank + a.T - 1) / a.T : 0;
 }
 
@@ -497,8 +499,8 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
                 ord = lo;
             }
             drop = (a.C > 0 && ord >= a.C) ? 1 : 0;
-            if (!drop && ord % a.T == a.tp_rank) // this peer's share under TP folding
-                dest = s_off[q] + ord / a.T;
+            if (!drop && (a.T == 1 || ord % a.T == a.tp_rank)) // this peer's share under TP folding
+                dest = s_off[q] + (a.T == 1 ? ord : ord / a.T);
             if (dest >= a.rows_max) { // cannot happen for consistent counts; never write out of bounds
                 atomicOr(o.status, MOE_DEV_ROW_RANGE);
                 dest = -1;

@@ -20,6 +20,7 @@
 #include "layout.cuh"
 #include "permute.cuh"
 #include "combine.cuh"
+#include "dedup.cuh"
 
 namespace {
 
@@ -524,6 +525,262 @@ int moe_restore_combined(const moe_problem_t *problem, const moe_layout_t *peer_
         a.dests[q] = peer_layouts[q].dest_row;
     }
     return launch_combine_args<true>(a, problem->k, stream);
+}
+
+int64_t moe_dedup_rows_max(const moe_problem_t *problem)
+{
+    Dims d;
+    const int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    return problem->N * static_cast<int64_t>(problem->k < problem->R ? problem->k : problem->R);
+}
+
+int moe_dedup_workspace_bytes(const moe_problem_t *problem, size_t *bytes)
+{
+    Dims d;
+    const int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    if (bytes == nullptr)
+        return MOE_ERR_INVALID;
+    *bytes = WS_BARRIER_BYTES + static_cast<size_t>(DEDUP_MAX_BLOCKS) * problem->R * 4;
+    return MOE_OK;
+}
+
+int moe_dedup_layout(const moe_problem_t *problem, const moe_layout_t *layout, const float *topk_probs,
+                     const moe_dedup_t *dedup, void *workspace, size_t workspace_bytes, void *stream)
+{
+    Dims d;
+    int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    if (problem->R > MOE_MAX_DEDUP_RANKS)
+        return MOE_ERR_UNSUPPORTED;
+    const int64_t recv_max = moe_dedup_rows_max(problem);
+    const moe_dedup_t *o = dedup;
+    if (layout == nullptr || o == nullptr || o->status == nullptr || o->num_tokens_per_rank == nullptr ||
+        o->recv_rank_offsets == nullptr || o->num_recv == nullptr)
+        return MOE_ERR_INVALID;
+    if (d.NK > 0 && (layout->phys_idx == nullptr || layout->dest_row == nullptr || o->is_token_in_rank == nullptr ||
+                     o->token_rank_row == nullptr))
+        return MOE_ERR_INVALID;
+    if (recv_max > 0 && (o->recv_src_token == nullptr || o->recv_topk_idx == nullptr ||
+                         o->recv_topk_weights == nullptr || o->recv_routing_map == nullptr ||
+                         o->recv_probs == nullptr || o->recv_pad_mask == nullptr))
+        return MOE_ERR_INVALID;
+    if (recv_max > 0 && (d.E_loc & 15) == 0 && (!aligned16(o->recv_routing_map) || !aligned16(o->recv_probs)))
+        return MOE_ERR_INVALID;
+    if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+        workspace_bytes < WS_BARRIER_BYTES + static_cast<size_t>(DEDUP_MAX_BLOCKS) * problem->R * 4)
+        return MOE_ERR_INVALID;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev)) != MOE_OK)
+        return rc;
+    int tpl = 1;
+    while (tpl <= DEDUP_MAX_TPL &&
+           (problem->N + static_cast<int64_t>(DEDUP_THREADS) * tpl - 1) / (static_cast<int64_t>(DEDUP_THREADS) * tpl) >
+               DEDUP_MAX_BLOCKS)
+        tpl <<= 1;
+    if (tpl > DEDUP_MAX_TPL)
+        return MOE_ERR_UNSUPPORTED;
+    int64_t G = (problem->N + static_cast<int64_t>(DEDUP_THREADS) * tpl - 1) / (static_cast<int64_t>(DEDUP_THREADS) * tpl);
+    if (G < 1)
+        G = 1;
+    if (G > dev.sms)
+        return MOE_ERR_UNSUPPORTED;
+    DedupArgs a;
+    a.phys_idx = layout->phys_idx;
+    a.dest_row = layout->dest_row;
+    a.probs = topk_probs;
+    a.N = problem->N;
+    a.recv_max = recv_max;
+    a.k = problem->k;
+    a.R = problem->R;
+    a.E_loc = d.E_loc;
+    a.G = static_cast<int32_t>(G);
+    a.ws_barrier = static_cast<uint32_t *>(workspace);
+    a.ws_counts = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + WS_BARRIER_BYTES);
+    a.barrier_limit_ns = WAIT_LIMIT_NS;
+    a.out = *o;
+    const dim3 grid(static_cast<unsigned>(G)), block(DEDUP_THREADS);
+    switch (tpl) {
+    case 1:
+        rc = launch(dedup_layout_kernel<1>, grid, block, 0, stream, true, a);
+        break;
+    case 2:
+        rc = launch(dedup_layout_kernel<2>, grid, block, 0, stream, true, a);
+        break;
+    case 4:
+        rc = launch(dedup_layout_kernel<4>, grid, block, 0, stream, true, a);
+        break;
+    default:
+        rc = launch(dedup_layout_kernel<8>, grid, block, 0, stream, true, a);
+        break;
+    }
+    if (rc != MOE_OK || recv_max == 0)
+        return rc;
+    DedupFillArgs f;
+    f.phys_idx = layout->phys_idx;
+    f.dest_row = layout->dest_row;
+    f.probs = topk_probs;
+    f.recv_max = recv_max;
+    f.k = problem->k;
+    f.R = problem->R;
+    f.E_loc = d.E_loc;
+    f.out = *o;
+    const int64_t fill_blocks = (recv_max + 255) / 256;
+    if (fill_blocks > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    return launch(dedup_fill_kernel, dim3(static_cast<unsigned>(fill_blocks)), dim3(256), 0, stream, false, f);
+}
+
+int moe_dedup_dispatch(const moe_problem_t *problem, const moe_dedup_t *dedup, const uint16_t *hidden,
+                       uint16_t *recv_x, void *stream)
+{
+    Dims d;
+    int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    if (problem->R > MOE_MAX_DEDUP_RANKS)
+        return MOE_ERR_UNSUPPORTED;
+    const int64_t recv_max = moe_dedup_rows_max(problem);
+    if (dedup == nullptr || dedup->status == nullptr || (d.NK > 0 && dedup->token_rank_row == nullptr) ||
+        (recv_max > 0 && dedup->recv_pad_mask == nullptr))
+        return MOE_ERR_INVALID;
+    if ((problem->N > 0 && (hidden == nullptr || !aligned16(hidden))) ||
+        (recv_max > 0 && (recv_x == nullptr || !aligned16(recv_x))))
+        return MOE_ERR_INVALID;
+    if (recv_max == 0)
+        return MOE_OK;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev)) != MOE_OK)
+        return rc;
+    PermuteArgs a;
+    a.hidden = reinterpret_cast<const uint4 *>(hidden);
+    a.send = reinterpret_cast<uint4 *>(recv_x);
+    a.dest_row = dedup->token_rank_row;
+    a.pad_mask = dedup->recv_pad_mask;
+    a.status = dedup->status;
+    a.N = problem->N;
+    a.rows_max = recv_max;
+    a.k = problem->R;
+    a.V = problem->H / 8;
+    a.group = a.V <= 32 * PERMUTE_CHUNKS ? 32 : (a.V <= 64 * PERMUTE_CHUNKS ? 64 : PERMUTE_THREADS);
+    a.pieces = (a.V + a.group * PERMUTE_CHUNKS - 1) / (a.group * PERMUTE_CHUNKS);
+    const int64_t zb = (recv_max + PERMUTE_THREADS - 1) / PERMUTE_THREADS;
+    a.zero_blocks = static_cast<int32_t>(zb < 4 * dev.sms ? zb : 4 * dev.sms);
+    const int64_t groups = PERMUTE_THREADS / a.group;
+    const int64_t blocks = a.zero_blocks + (problem->N * a.pieces + groups - 1) / groups;
+    if (blocks > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    return launch(permute_kernel, dim3(static_cast<unsigned>(blocks)), dim3(PERMUTE_THREADS), 0, stream, false, a);
+}
+
+int moe_dedup_combine_local(const moe_problem_t *problem, const moe_layout_t *layout, const moe_dedup_t *dedup,
+                            const uint16_t *expert_out, const float *topk_probs, uint16_t *partial, void *stream)
+{
+    Dims d;
+    int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    if (problem->R > MOE_MAX_DEDUP_RANKS)
+        return MOE_ERR_UNSUPPORTED;
+    const int64_t recv_max = moe_dedup_rows_max(problem);
+    if ((rc = check_layout(layout, d, false)) != MOE_OK)
+        return rc;
+    if (layout->rank_offsets == nullptr || dedup == nullptr || dedup->status == nullptr ||
+        dedup->num_recv == nullptr || (d.NK > 0 && dedup->token_rank_row == nullptr))
+        return MOE_ERR_INVALID;
+    if ((d.rows_max > 0 && (expert_out == nullptr || !aligned16(expert_out))) ||
+        (recv_max > 0 && (partial == nullptr || !aligned16(partial))))
+        return MOE_ERR_INVALID;
+    if (recv_max == 0)
+        return MOE_OK;
+    DedupCombineArgs a;
+    a.y = reinterpret_cast<const uint4 *>(expert_out);
+    a.dest_row = layout->dest_row;
+    a.probs = topk_probs;
+    a.rank_offsets = layout->rank_offsets;
+    a.token_rank_row = dedup->token_rank_row;
+    a.partial = reinterpret_cast<uint4 *>(partial);
+    a.status = dedup->status;
+    a.N = problem->N;
+    a.recv_max = recv_max;
+    a.rows_max = d.rows_max;
+    a.k = problem->k;
+    a.R = problem->R;
+    a.V = problem->H / 8;
+    // token-major, as the combine: the widest CTA (up to 256 threads) that splits the row into equal parts
+    const int v32 = ((a.V + 31) / 32) * 32;
+    const int threads = v32 % 256 == 0 ? 256 : (v32 % 128 == 0 ? 128 : (v32 % 64 == 0 ? 64 : 32));
+    a.nchunks = (a.V + threads - 1) / threads;
+    const int64_t blocks = problem->N * a.nchunks;
+    if (blocks > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    if (blocks > 0) {
+        const dim3 grid(static_cast<unsigned>(blocks)), block(threads);
+        switch (problem->k) {
+        case 1:
+            rc = launch(dedup_combine_local_kernel<1>, grid, block, 0, stream, false, a);
+            break;
+        case 2:
+            rc = launch(dedup_combine_local_kernel<2>, grid, block, 0, stream, false, a);
+            break;
+        case 4:
+            rc = launch(dedup_combine_local_kernel<4>, grid, block, 0, stream, false, a);
+            break;
+        case 6:
+            rc = launch(dedup_combine_local_kernel<6>, grid, block, 0, stream, false, a);
+            break;
+        case 8:
+            rc = launch(dedup_combine_local_kernel<8>, grid, block, 0, stream, false, a);
+            break;
+        default:
+            rc = launch(dedup_combine_local_kernel<0>, grid, block, 0, stream, false, a);
+            break;
+        }
+        if (rc != MOE_OK)
+            return rc;
+    }
+    // receive rows past num_recv: zero partials (their count is known on the device only)
+    DeviceInfo dev;
+    if ((rc = device_info(&dev)) != MOE_OK)
+        return rc;
+    const int64_t tail_work = (recv_max * a.V + 127) / 128;
+    const int64_t tail_blocks = tail_work < 2 * dev.sms ? tail_work : 2 * dev.sms;
+    return launch(dedup_zero_tail_kernel, dim3(static_cast<unsigned>(tail_blocks)), dim3(128), 0, stream, false,
+                  a.partial, static_cast<const int32_t *>(dedup->num_recv), recv_max, a.V);
+}
+
+int moe_dedup_combine(const moe_problem_t *problem, const moe_dedup_t *dedup, const uint16_t *partial,
+                      uint16_t *out, void *stream)
+{
+    Dims d;
+    int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    if (problem->R > MOE_MAX_DEDUP_RANKS)
+        return MOE_ERR_UNSUPPORTED;
+    const int64_t recv_max = moe_dedup_rows_max(problem);
+    if (dedup == nullptr || dedup->status == nullptr || (d.NK > 0 && dedup->token_rank_row == nullptr))
+        return MOE_ERR_INVALID;
+    if (problem->N == 0)
+        return MOE_OK;
+    if (out == nullptr || !aligned16(out) || (recv_max > 0 && (partial == nullptr || !aligned16(partial))))
+        return MOE_ERR_INVALID;
+    CombineArgs a = {};
+    a.y = reinterpret_cast<const uint4 *>(partial);
+    a.dest_row = dedup->token_rank_row;
+    a.probs = nullptr; // unit weights: the partials are already weighted
+    a.out = reinterpret_cast<uint4 *>(out);
+    a.status = dedup->status;
+    a.N = problem->N;
+    a.rows_max = recv_max;
+    a.k = problem->R;
+    a.V = problem->H / 8;
+    a.T = 1;
+    return launch_combine_args<false>(a, problem->R, stream);
 }
 
 int moe_combine_backward(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *grad_out,

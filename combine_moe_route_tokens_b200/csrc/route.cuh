@@ -10,11 +10,11 @@
 // selection compares logits, so the ids never depend on expf rounding.
 //
 // Lane l holds experts l, l+32, ... as 32-bit order-preserving keys (0 marks
-// an empty slot) and sorts them once, descending (equal keys: lower id first),
-// with a static bitonic network. Each of the k rounds then compares only the
-// lanes' heads: the warp maximum with one redux.sync, and among the lanes
-// holding it the lowest expert id with a second; the winning lane shifts its
-// list. The key maps back to the logit exactly, so no shuffle is needed.
+// an empty or already chosen slot). Each of the k rounds scans the lane's keys
+// for its best (first occurrence = lowest id), takes the warp maximum with one
+// redux.sync and, among the lanes holding it, the lowest expert id with a
+// second; the owner clears that key. The key maps back to the logit exactly, so
+// no shuffle is needed; lane j turns the j-th winner into its prob at the end.
 #pragma once
 
 #include <cstdint>
@@ -77,57 +77,34 @@ __global__ void __launch_bounds__(ROUTE_WARPS_PER_BLOCK * 32)
 
     float s = 0.0f;
     uint32_t key[VPL];
-    int slot[VPL]; // i of expert i * 32 + lane
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
         const bool in = i * 32 + lane < E;
         s += in ? expf(v[i] - m) : 0.0f;
         key[i] = in ? route_key(v[i]) : 0u;
-        slot[i] = i;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
         s += __shfl_xor_sync(0xffffffffu, s, o);
 
-    // bitonic sort of the lane's keys, descending; equal keys keep the lower slot first
-#pragma unroll
-    for (int size = 2; size <= VPL; size <<= 1) {
-#pragma unroll
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-#pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                const int j = i ^ stride;
-                if (j > i) {
-                    const bool first_greater = key[i] > key[j] || (key[i] == key[j] && slot[i] < slot[j]);
-                    const bool want_greater_first = (i & size) == 0;
-                    if (first_greater != want_greater_first) {
-                        const uint32_t tk = key[i];
-                        key[i] = key[j];
-                        key[j] = tk;
-                        const int ts = slot[i];
-                        slot[i] = slot[j];
-                        slot[j] = ts;
-                    }
-                }
-            }
-        }
-    }
-
     int my_id = -1;
     uint32_t my_key = 0;
     for (int j = 0; j < k; ++j) {
-        const uint32_t head = key[0];
-        const uint32_t wmax = __reduce_max_sync(0xffffffffu, head);
-        const uint32_t cand = (head == wmax && head != 0u) ? ~static_cast<uint32_t>(slot[0] * 32 + lane) : 0u;
-        const int e = static_cast<int>(~__reduce_max_sync(0xffffffffu, cand));
-        if ((e & 31) == lane) {
+        uint32_t best = 0;
+        int bi = 0;
 #pragma unroll
-            for (int i = 0; i + 1 < VPL; ++i) {
-                key[i] = key[i + 1];
-                slot[i] = slot[i + 1];
-            }
-            key[VPL - 1] = 0u;
+        for (int i = 0; i < VPL; ++i) {
+            const bool better = key[i] > best;
+            best = better ? key[i] : best;
+            bi = better ? i : bi;
         }
+        const uint32_t wmax = __reduce_max_sync(0xffffffffu, best);
+        const uint32_t cand = (best == wmax && best != 0u) ? ~static_cast<uint32_t>(bi * 32 + lane) : 0u;
+        const int e = static_cast<int>(~__reduce_max_sync(0xffffffffu, cand));
+        const bool mine = (e & 31) == lane;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i)
+            key[i] = (mine && i == (e >> 5)) ? 0u : key[i];
         if (lane == j) {
             my_id = e;
             my_key = wmax;

@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-#define MOE_RT_ABI_VERSION 3
+#define MOE_RT_ABI_VERSION 4
 
 /* Every entry point is exported; everything else in the library is hidden. */
 #if defined(__GNUC__)
@@ -265,6 +265,73 @@ MOE_API int moe_combine(const moe_problem_t *problem, const moe_layout_t *layout
 MOE_API int moe_restore_combined(const moe_problem_t *problem, const moe_layout_t *peer_layouts,
                                  const uint16_t *const *peer_expert_out, const float *topk_probs, uint16_t *out,
                                  void *stream);
+
+/*
+ * DeepEP-style token-dedup view ([Megatron MORI]: the MORI dispatcher follows
+ * the DeepEP contract: each token goes once to each rank that owns one of its
+ * kept slots; the receiver gets local top-k ids with -1 sentinels and
+ * receiver-side weights, and _indices_to_multihot turns them into a
+ * [tokens, local experts] routing map with probs). One receive row per
+ * (token, rank) pair, rank-major and token-ascending within a rank;
+ * recv_max = N * min(k, R) rows, the rows past num_recv are tail rows
+ * (token -1, ids -1, weights / map / probs 0, pad 1). R <= MOE_MAX_DEDUP_RANKS.
+ */
+#define MOE_MAX_DEDUP_RANKS 32
+
+typedef struct {
+    int32_t *num_tokens_per_rank; /* [R] tokens each rank receives */
+    int32_t *recv_rank_offsets;   /* [R+1] first receive row of each rank */
+    int32_t *num_recv;            /* [1] recv_rank_offsets[R] */
+    uint8_t *is_token_in_rank;    /* [N, R] */
+    int32_t *token_rank_row;      /* [N, R] receive row of (t, r), -1 if t is not sent to r */
+    int32_t *recv_src_token;      /* [recv_max] source token, -1 in the tail */
+    int32_t *recv_topk_idx;       /* [recv_max, k] rank-local expert id of slot j, -1 if not on this rank */
+    float *recv_topk_weights;     /* [recv_max, k] receiver-side prob, 0 where the id is -1 */
+    uint8_t *recv_routing_map;    /* [recv_max, E_loc] multihot over the rank's experts */
+    float *recv_probs;            /* [recv_max, E_loc] the prob at each set bit, else 0 */
+    uint8_t *recv_pad_mask;       /* [recv_max] 1 in the tail */
+    uint32_t *status;             /* [1] MOE_DEV_* bits, OR-ed */
+} moe_dedup_t;
+
+/* recv_max = N * min(k, R), or a negative MOE_ERR_* for an invalid problem. Host only. */
+MOE_API int64_t moe_dedup_rows_max(const moe_problem_t *problem);
+
+/* Scratch bytes of moe_dedup_layout (zero-filled before first use, as for the layout). Host only. */
+MOE_API int moe_dedup_workspace_bytes(const moe_problem_t *problem, size_t *bytes);
+
+/*
+ * Build the dedup view from a dispatch layout (reads layout->phys_idx and
+ * layout->dest_row: a slot counts where dest_row >= 0): one cooperative
+ * launch with a bounded grid barrier places the (token, rank) pairs, a second
+ * launch fills the per-row receive data. topk_probs [N, k] fp32 or NULL
+ * (weights 0). Limits: R <= MOE_MAX_DEDUP_RANKS, N <= 262144.
+ */
+MOE_API int moe_dedup_layout(const moe_problem_t *problem, const moe_layout_t *layout, const float *topk_probs,
+                             const moe_dedup_t *dedup, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Dispatch each token once per receiving rank: recv_x[token_rank_row[t,r]] = hidden[t]; tail rows zero.
+ *   hidden [N, H] bf16; recv_x [recv_max, H] bf16 */
+MOE_API int moe_dedup_dispatch(const moe_problem_t *problem, const moe_dedup_t *dedup, const uint16_t *hidden,
+                               uint16_t *recv_x, void *stream);
+
+/*
+ * Receiver side of the DeepEP-style combine: for receive row w of token t on
+ * rank r, partial[w] = bf16_rn( fp32 fmaf chain over ascending j of
+ * p[t,j] * y[dest_row[t,j]] for the kept slots whose row lies in rank r's range
+ * [rank_offsets[r], rank_offsets[r+1]) of the layout ); tail rows 0.
+ * Reads dedup->token_rank_row and dedup->num_recv (of moe_dedup_layout on the
+ * same layout); every kept slot row is read once per token.
+ *   expert_out [rows_max, H] bf16 (the layout's send-buffer order);
+ *   topk_probs [N, k] fp32 or NULL (unit weights); partial [recv_max, H] bf16
+ */
+MOE_API int moe_dedup_combine_local(const moe_problem_t *problem, const moe_layout_t *layout,
+                                    const moe_dedup_t *dedup, const uint16_t *expert_out, const float *topk_probs,
+                                    uint16_t *partial, void *stream);
+
+/* Sender side: out[t] = bf16_rn( fp32 sum over ascending r of partial[token_rank_row[t,r]] ).
+ *   partial [recv_max, H] bf16; out [N, H] bf16 */
+MOE_API int moe_dedup_combine(const moe_problem_t *problem, const moe_dedup_t *dedup, const uint16_t *partial,
+                              uint16_t *out, void *stream);
 
 /*
  * Backward of permute ([Megatron MORI]: dispatch backward sums the row

@@ -15,6 +15,7 @@ Shapes follow the pages' problem statements:
 * ``ht_align16`` — the ``ht`` shape and inputs with every expert's rows padded up to
                   a multiple of 16 (grouped-GEMM / FP8 alignment).
 * ``ht_tp2``    — the ``ht`` shape and inputs folded over 2 TP peers.
+* ``ht_dedup``  — the ``ht`` shape and inputs through the DeepEP-style token-dedup path.
 
 Recipe: logits are N(0,1) float32 plus, where a workload is skewed, a per-expert
 bias ``-s ln(rank+1)`` over a seeded ranking of the experts; hidden states and
@@ -53,6 +54,7 @@ class Workload:
     backward: bool = False
     row_align: int = 0
     tp_size: int = 0
+    dedup: bool = False
     seed: int = 0x5EED0000
     note: str = field(default="", compare=False)
 
@@ -84,6 +86,7 @@ class Workload:
             backward=self.backward,
             row_align=self.row_align,
             tp_size=self.tp_size,
+            dedup=self.dedup,
             seed=self.seed,
             note=self.note,
         )
@@ -109,6 +112,8 @@ class Workload:
             d["row_align"] = self.row_align
         if self.tp_size > 1:
             d["tp_size"] = self.tp_size
+        if self.dedup:
+            d["dedup"] = True
         return d
 
 
@@ -147,6 +152,9 @@ WORKLOADS = {
         # the same shape folded over 2 TP peers (each peer's layout and send buffer on
         # this GPU, then one restore over both)
         Workload("ht_tp2", N=4096, H=7168, E_log=256, k=8, R=4, tp_size=2, seed=0x5EED0002),
+        # the same shape through the DeepEP-style path: each token sent once per rank,
+        # receiver-side partials, sender-side sum over ranks
+        Workload("ht_dedup", N=4096, H=7168, E_log=256, k=8, R=4, dedup=True, seed=0x5EED0002),
     ]
 }
 

@@ -395,3 +395,45 @@ def test_tp_fold_layout_permute_restore(case):
     assert np.array_equal(got, oracle.restore_combined(oracle_sends, oracle_dests, probs))
     assert np.array_equal(got, expect)  # restore over all peers = the unfolded combine
     assert all(G.status() == 0 for G in layouts)
+
+
+# ------------------------------------------------------- DeepEP-style dedup
+
+
+DEDUP_CASES = [
+    # N, H, k, E_log, R, C, reps, align, T
+    (4096, 7168, 8, 256, 4, 0, 0, 0, 0),  # the 4096-token / e256 / top-8 shape
+    (1000, 72, 4, 32, 8, 0, 0, 0, 0),
+    (3000, 40, 2, 16, 2, 256, 0, 16, 0),  # capacity + alignment
+    (2049, 24, 8, 64, 8, 0, 8, 0, 2),  # reroute + TP folding (peer 0)
+    (300, 16, 12, 48, 16, 0, 0, 0, 0),  # k > 8, E_loc not a multiple of 16
+    (70000, 8, 1, 4, 2, 0, 0, 0, 0),  # many tokens, several per lane
+]
+
+
+@pytest.mark.parametrize("case", DEDUP_CASES, ids=[f"N{c[0]}_k{c[2]}_E{c[3]}_R{c[4]}" for c in DEDUP_CASES])
+def test_dedup_path(case):
+    N, H, k, E_log, R, C, reps, A, T = case
+    idx, probs, hidden = _small_case(N, H, k, E_log, R, C, reps, 0.05, seed=N + R, zipf=1.3)
+    L = oracle.layout(idx, probs, E_log=E_log, R=R, C=C, num_replicas=reps, align=A, tp_size=T)
+    D = oracle.dedup_layout(L, probs, E_log=E_log, R=R, num_replicas=reps)
+    p = moe.Problem(N=N, H=H, k=k, E_log=E_log, R=R, capacity=C, num_replicas=reps, row_align=A, tp_size=T)
+    G = moe.moe_dispatch_layout(p, dev(idx), dev(probs))
+    V = moe.moe_dedup_layout(p, G, dev(probs))
+    torch.cuda.synchronize()
+    for key in ("num_tokens_per_rank", "recv_rank_offsets", "num_recv", "is_token_in_rank", "token_rank_row",
+                "recv_src_token", "recv_topk_idx", "recv_topk_weights", "recv_routing_map", "recv_probs",
+                "recv_pad_mask"):
+        got = host(V[key]).reshape(-1)
+        exp = np.asarray(D[key]).reshape(-1)
+        assert np.array_equal(got.view(np.uint8), exp.astype(got.dtype).view(np.uint8)), key
+    recv_x = moe.moe_dedup_dispatch(p, V, dev(hidden))
+    assert np.array_equal(host(recv_x), oracle.permute(hidden, D["token_rank_row"], D["recv_max"]))
+    send = moe.moe_permute(p, G, dev(hidden))
+    exp_send = oracle.permute(hidden, L["dest_row"], L["rows_max"])
+    partial = moe.moe_dedup_combine_local(p, G, V, send, dev(probs))
+    exp_partial = oracle.dedup_combine_local(exp_send, L, D, probs, R)
+    assert np.array_equal(host(partial), exp_partial)
+    out = moe.moe_dedup_combine(p, V, partial)
+    assert np.array_equal(host(out), oracle.combine(exp_partial, D["token_rank_row"], None))
+    assert G.status() == 0 and V.status() == 0
