@@ -335,6 +335,8 @@ def run_ours(args, ws, rank, local):
     moe.load_library()
 
     w = get_workload(args.workload)
+    if args.tokens:  # a smaller batch of the same workload (profiling captures), named as such
+        w = w.scaled(args.tokens)
     host = rank_inputs(w, rank)
     set_bytes = sum(v.nbytes for v in host.values())
     nsets = max(2, min(8, math.ceil(2 * L2_BYTES / set_bytes)))
@@ -398,44 +400,82 @@ def run_ours(args, ws, rank, local):
         raise RuntimeError(f"device status {status:#x} after the timed steps")
     elapsed_ms = max_over_ranks(elapsed_ms, device)
 
-    # end to end through the public API: pinned host inputs in, result out, every step
+    # end to end through the public API: every step copies its inputs in from pinned host
+    # memory and its combined output back out. Two pipelines of device buffers alternate, so
+    # step i's copy-out (one copy engine) overlaps step i+1's copy-in (the other) and its
+    # kernels; each step waits for the copy-in of its own inputs, and a buffer is written
+    # again only after its previous copy-out finished.
     e2e = None
     if not args.no_e2e:
         pin = {key: torch.from_numpy(v if v.dtype != np.uint16 else v.view(np.int16)).pin_memory()
                for key, v in host.items()}
-        out_host = torch.empty((w.N, w.H), dtype=torch.int16).pin_memory()
-        dst = step.sets[0]
-        views = {key: (dst[key].view(torch.int16) if dst[key].dtype == torch.bfloat16 else dst[key])
-                 for key in pin}
+        outs_host = [torch.empty((w.N, w.H), dtype=torch.int16).pin_memory() for _ in range(2)]
+        h2d_s = torch.cuda.Stream(device)
+        d2h_s = torch.cuda.Stream(device)
+        comp_s = torch.cuda.Stream(device)
+        pipes = []
+        with torch.cuda.stream(comp_s):
+            for b in range(2):
+                dset = {key: torch.empty_like(step.sets[0][key]) for key in pin}
+                pipes.append(Step(w, moe, _native, torch, [dset], device))
+        views = [{key: (q.sets[0][key].view(torch.int16) if q.sets[0][key].dtype == torch.bfloat16
+                        else q.sets[0][key]) for key in pin} for q in pipes]
         h2d = sum(t.numel() * t.element_size() for t in pin.values())
-        d2h = out_host.numel() * out_host.element_size()
+        d2h = outs_host[0].numel() * outs_host[0].element_size()
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        started = [False, False]
 
         def e2e_step(i):
-            for key in pin:
-                views[key].copy_(pin[key], non_blocking=True)
-            step.run(0)
-            out_host.copy_(step.out.view(torch.int16), non_blocking=True)
+            b = i % 2
+            if started[b]:
+                h2d_s.wait_event(comp_done[b])  # the kernels of step i-2 finished reading these inputs
+            with torch.cuda.stream(h2d_s):
+                for key in pin:
+                    views[b][key].copy_(pin[key], non_blocking=True)
+            in_done[b].record(h2d_s)
+            comp_s.wait_event(in_done[b])
+            if started[b]:
+                comp_s.wait_event(out_done[b])  # step i-2's output has left the device
+            pipes[b].run(0)
+            comp_done[b].record(comp_s)
+            d2h_s.wait_event(comp_done[b])
+            with torch.cuda.stream(d2h_s):
+                outs_host[b].copy_(pipes[b].out.view(torch.int16), non_blocking=True)
+            out_done[b].record(d2h_s)
+            started[b] = True
 
-        for i in range(max(1, min(args.warmup, 3))):
+        for i in range(max(2, min(args.warmup, 4))):
             e2e_step(i)
+        torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         barrier()
         torch.cuda.synchronize()
-        e0.record(step.stream)
+        e0.record(h2d_s)
+        comp_s.wait_event(e0)
         for i in range(args.steps):
             e2e_step(i)
-        e1.record(step.stream)
+        for b in range(2):  # the timed region ends when the last output is on the host
+            d2h_s.wait_event(out_done[b])
+        e1.record(d2h_s)
         torch.cuda.synchronize()
         barrier()
         e_ms = max_over_ranks(e0.elapsed_time(e1), device)
+        st = 0
+        for q in pipes:
+            st |= q.status()
+        if st != 0:
+            raise RuntimeError(f"device status {st:#x} after the end-to-end steps")
         e2e = {
-            "value": w.N * args.steps * ws / (e_ms / 1e3),
+            "value": round(w.N * args.steps * ws / (e_ms / 1e3), 1),
             "unit": "tokens/s",
             "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
-            "ms_per_step": e_ms / args.steps,
+            "ms_per_step": round(e_ms / args.steps, 4),
+            "pipelining": "2 device buffer sets; copy-in, kernels and copy-out on three streams",
         }
+        del pipes
 
     if ws > 1:
         tdist.barrier()
@@ -447,8 +487,12 @@ def run_ours(args, ws, rank, local):
     kernels = {}
     for name in step.kernel_names:
         avg_ms = statistics.mean(per_kernel_ms[name])
+        qs = statistics.quantiles(per_kernel_ms[name], n=10) if len(per_kernel_ms[name]) > 1 else [avg_ms] * 9
         kernels[name] = {
             "us": round(avg_ms * 1e3, 2),
+            "median_us": round(statistics.median(per_kernel_ms[name]) * 1e3, 2),
+            "p10_us": round(qs[0] * 1e3, 2),
+            "p90_us": round(qs[8] * 1e3, 2),
             "algorithmic_bytes": abytes[name],
             "gbs": round(abytes[name] / (avg_ms * 1e-3) / 1e9, 1),
         }
@@ -610,6 +654,7 @@ def main():
     ap.add_argument("--workload", default="ht", help="tiny | ht | qwen3 | capacity | ultraep")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0, help="run the workload with this many tokens (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()

@@ -19,6 +19,7 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 
 #include "moe_rt.h"
 #include "permute.cuh"
@@ -83,20 +84,31 @@ __device__ __forceinline__ void load_slot_meta(const int32_t *dest_row, const fl
 }
 
 // Restore after TP folding: slot j of token t lives in the one peer buffer whose
-// row map has a row for it. Lane j < k finds that peer (src) and the row (d).
-__device__ __forceinline__ void load_slot_meta_peers(const CombineArgs &a, int64_t t, int k, int32_t &d, float &p,
-                                                     int32_t &src)
+// row map has a row for it. Lane j < k finds that peer and the row and returns
+// the row's address (null if no peer holds the slot), so the per-thread gather
+// needs no per-slot peer selection.
+__device__ __forceinline__ const uint4 *peer_base(const CombineArgs &a, int32_t src)
+{
+    const uint4 *base = a.ys[0];
+#pragma unroll
+    for (int i = 1; i < MOE_MAX_TP; ++i)
+        base = (src == i) ? a.ys[i] : base;
+    return base;
+}
+
+__device__ __forceinline__ void load_slot_meta_peers(const CombineArgs &a, int64_t t, int k, const uint4 *&row,
+                                                     float &p)
 {
     const int lane = threadIdx.x & 31;
-    d = -1;
+    row = nullptr;
     p = 0.0f;
-    src = 0;
     if (lane < k) {
         p = a.probs != nullptr ? __ldg(a.probs + t * k + lane) : 1.0f;
         int32_t r[MOE_MAX_TP];
 #pragma unroll
         for (int q = 0; q < MOE_MAX_TP; ++q)
             r[q] = q < a.T ? __ldg(a.dests[q] + t * k + lane) : -1;
+        int32_t d = -1, src = 0;
 #pragma unroll
         for (int q = 0; q < MOE_MAX_TP; ++q) {
             if (r[q] < -1 || r[q] >= a.rows_max) {
@@ -106,16 +118,9 @@ __device__ __forceinline__ void load_slot_meta_peers(const CombineArgs &a, int64
                 src = q;
             }
         }
+        if (d >= 0)
+            row = peer_base(a, src) + static_cast<int64_t>(d) * a.V;
     }
-}
-
-__device__ __forceinline__ const uint4 *peer_base(const CombineArgs &a, int32_t src)
-{
-    const uint4 *base = a.ys[0];
-#pragma unroll
-    for (int i = 1; i < MOE_MAX_TP; ++i)
-        base = (src == i) ? a.ys[i] : base;
-    return base;
 }
 
 // K > 0: top-k fixed at compile time; K == 0: runtime k <= 32.
@@ -130,17 +135,40 @@ __global__ void __launch_bounds__(COMBINE_THREADS, 4) combine_kernel(CombineArgs
     const int v = c * blockDim.x + threadIdx.x;
     const int k = K > 0 ? K : a.k;
 
-    int32_t d, src = 0;
+    // lane j < k: slot j's source row and weight. One buffer: the row index;
+    // TP peers: the row's address in the peer buffer that holds it.
+    using Src = typename std::conditional<PEERS, const uint4 *, int32_t>::type;
+    Src src;
     float p;
-    if constexpr (PEERS)
-        load_slot_meta_peers(a, t, k, d, p, src);
-    else
-        load_slot_meta(a.dest_row, a.probs, t, k, a.rows_max, a.status, d, p);
-    auto row_ptr = [&](int32_t row, int32_t peer) -> const uint4 * {
+    if constexpr (PEERS) {
+        load_slot_meta_peers(a, t, k, src, p);
+    } else {
+        load_slot_meta(a.dest_row, a.probs, t, k, a.rows_max, a.status, src, p);
+    }
+    auto shfl_src = [&](int j) -> Src {
         if constexpr (PEERS)
-            return peer_base(a, peer) + static_cast<int64_t>(row) * a.V;
+            return reinterpret_cast<const uint4 *>(
+                __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(src), j));
         else
-            return a.y + static_cast<int64_t>(row) * a.V;
+            return __shfl_sync(0xffffffffu, src, j);
+    };
+    auto valid = [](Src s) -> bool {
+        if constexpr (PEERS)
+            return s != nullptr;
+        else
+            return s >= 0;
+    };
+    auto row_ptr = [&](Src s) -> const uint4 * {
+        if constexpr (PEERS)
+            return s;
+        else
+            return a.y + static_cast<int64_t>(s) * a.V;
+    };
+    auto none = []() -> Src {
+        if constexpr (PEERS)
+            return nullptr;
+        else
+            return -1;
     };
 
     float acc[8];
@@ -149,46 +177,44 @@ __global__ void __launch_bounds__(COMBINE_THREADS, 4) combine_kernel(CombineArgs
         acc[e] = 0.0f;
 
     if constexpr (K > 0) {
-        int32_t dj[K], sj[K];
+        Src sj[K];
         float pj[K];
         uint4 yj[K];
 #pragma unroll
         for (int j = 0; j < K; ++j) {
-            dj[j] = __shfl_sync(0xffffffffu, d, j);
+            sj[j] = shfl_src(j);
             pj[j] = __shfl_sync(0xffffffffu, p, j);
-            sj[j] = PEERS ? __shfl_sync(0xffffffffu, src, j) : 0;
         }
         if (v >= a.V)
             return;
 #pragma unroll
         for (int j = 0; j < K; ++j)
-            if (dj[j] >= 0)
-                yj[j] = ld_stream_u4(row_ptr(dj[j], sj[j]) + v);
+            if (valid(sj[j]))
+                yj[j] = ld_stream_u4(row_ptr(sj[j]) + v);
 #pragma unroll
         for (int j = 0; j < K; ++j)
-            if (dj[j] >= 0)
+            if (valid(sj[j]))
                 fma8(acc, pj[j], yj[j]);
     } else {
         const bool active = v < a.V;
         for (int j0 = 0; j0 < k; j0 += 4) {
-            int32_t dj[4], sj[4];
+            Src sj[4];
             float pj[4];
             uint4 yj[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                dj[u] = __shfl_sync(0xffffffffu, d, (j0 + u) & 31);
+                sj[u] = shfl_src((j0 + u) & 31);
                 pj[u] = __shfl_sync(0xffffffffu, p, (j0 + u) & 31);
-                sj[u] = PEERS ? __shfl_sync(0xffffffffu, src, (j0 + u) & 31) : 0;
                 if (j0 + u >= k || !active)
-                    dj[u] = -1;
+                    sj[u] = none();
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-                if (dj[u] >= 0)
-                    yj[u] = ld_stream_u4(row_ptr(dj[u], sj[u]) + v);
+                if (valid(sj[u]))
+                    yj[u] = ld_stream_u4(row_ptr(sj[u]) + v);
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-                if (dj[u] >= 0)
+                if (valid(sj[u]))
                     fma8(acc, pj[u], yj[u]);
         }
         if (!active)

@@ -23,6 +23,7 @@
 
 #include "moe_rt.h"
 #include "combine.cuh"
+#include "grid_barrier.cuh"
 #include "ptx.cuh"
 
 namespace moert {
@@ -41,7 +42,7 @@ struct DedupArgs {
     int32_t k, R, E_loc;
     int32_t G;
     int32_t *ws_counts;   // [G][R]
-    uint32_t *ws_barrier; // [3] as in the layout
+    uint32_t *ws_barrier; // [3] as in the layout: ticket word, unused, error bits
     uint64_t barrier_limit_ns;
     moe_dedup_t out;
 };
@@ -51,41 +52,6 @@ __device__ __forceinline__ uint32_t dedup_lanemask_lt()
     uint32_t m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
     return m;
-}
-
-__device__ __forceinline__ uint32_t dedup_ld_acquire(const uint32_t *p)
-{
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// The same bounded, generation-counted grid barrier as the layout's.
-__device__ __forceinline__ bool dedup_grid_barrier(uint32_t *bar, uint32_t target, uint64_t limit_ns)
-{
-    __shared__ int s_ok;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const uint32_t gen = dedup_ld_acquire(bar + 1);
-        uint32_t arrived;
-        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(arrived) : "l"(bar) : "memory");
-        int ok = 1;
-        if (arrived == target - 1) {
-            atomicExch(bar, 0u);
-            asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar + 1) : "memory");
-        } else {
-            const uint64_t t0 = global_timer_ns();
-            while (dedup_ld_acquire(bar + 1) == gen) {
-                if (global_timer_ns() - t0 > limit_ns) {
-                    ok = 0;
-                    break;
-                }
-            }
-        }
-        s_ok = ok;
-    }
-    __syncthreads();
-    return s_ok != 0;
 }
 
 template <int TPL> // tokens per lane; a warp owns 32 * TPL consecutive tokens
@@ -143,7 +109,7 @@ __global__ void __launch_bounds__(DEDUP_THREADS) dedup_layout_kernel(DedupArgs a
         a.ws_counts[static_cast<int64_t>(b) * R + tid] = static_cast<int32_t>(run);
     }
 
-    if (!dedup_grid_barrier(a.ws_barrier, static_cast<uint32_t>(a.G), a.barrier_limit_ns)) {
+    if (!grid_barrier_ticket(a.ws_barrier, static_cast<uint32_t>(a.G), 0u, a.barrier_limit_ns)) {
         if (tid == 0)
             atomicOr(a.out.status, MOE_DEV_TIMEOUT);
         return;

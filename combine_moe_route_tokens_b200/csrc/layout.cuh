@@ -29,6 +29,7 @@
 #include <cstdint>
 
 #include "moe_rt.h"
+#include "grid_barrier.cuh"
 #include "ptx.cuh"
 
 namespace moert {
@@ -42,8 +43,8 @@ constexpr int LAYOUT_MAX_IPL = 8; // assignments per lane held in registers
 constexpr int LAYOUT_ITEMS_PER_BLOCK = 512; // target slice per block before the block cap
 
 struct LayoutArgs {
-    const int32_t *topk_idx;
-    const float *topk_probs;
+    const int32_t *topk_idx; // [N, k]
+    const float *topk_probs; // [N, k] or null
     int64_t NK;
     int64_t rows_max;
     int32_t k, E_log, E, R, E_loc, M, S, num_replicas, C;
@@ -54,7 +55,7 @@ struct LayoutArgs {
     int32_t sub; // assignments per warp slice, a multiple of 32
     int32_t G;   // blocks
     int32_t *ws_counts;   // [G][E_log]: per-block logical totals
-    uint32_t *ws_barrier; // [3]: arrival count, generation, error bits of this call
+    uint32_t *ws_barrier; // [3]: arrival ticket word, (unused), error bits of this call
     uint64_t barrier_limit_ns;
     uint32_t barrier_extra; // test hook: extra arrivals the barrier waits for
     moe_layout_t out;
@@ -66,53 +67,6 @@ __host__ __device__ inline size_t layout_smem_words(int E_log, int E)
     return static_cast<size_t>(LAYOUT_WARPS) * E_log // per-warp counters, then prefixes
            + 3 * static_cast<size_t>(E_log)          // block prefix, totals, placement
            + 2 * static_cast<size_t>(E) + 1;         // physical counts, offsets
-}
-
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p)
-{
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ uint32_t atom_add_acq_rel_u32(uint32_t *p, uint32_t v)
-{
-    uint32_t old;
-    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
-}
-
-__device__ __forceinline__ void red_release_add_u32(uint32_t *p, uint32_t v)
-{
-    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Bounded grid barrier with a generation word. The arrival count goes back to
-// 0 for the next launch unless the wait ran out.
-__device__ __forceinline__ bool layout_grid_barrier(uint32_t *bar, uint32_t target, uint64_t limit_ns)
-{
-    __shared__ int s_ok;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const uint32_t gen = ld_acquire_u32(bar + 1);
-        const uint32_t arrived = atom_add_acq_rel_u32(bar, 1u);
-        int ok = 1;
-        if (arrived == target - 1) {
-            atomicExch(bar, 0u);
-            red_release_add_u32(bar + 1, 1u);
-        } else {
-            const uint64_t t0 = global_timer_ns();
-            while (ld_acquire_u32(bar + 1) == gen) {
-                if (global_timer_ns() - t0 > limit_ns) {
-                    ok = 0;
-                    break;
-                }
-            }
-        }
-        s_ok = ok;
-    }
-    __syncthreads();
-    return s_ok != 0;
 }
 
 // Rows this peer keeps of an expert with `raw` assignments: the capacity-kept
@@ -221,7 +175,7 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
     int32_t *s_raw = s_repl + E_log;                                           // [E]
     int32_t *s_off = s_raw + E;                                                // [E+1]
     __shared__ int32_t s_hot[LAYOUT_MAX_E_LOG];
-    __shared__ int32_t s_part[2][LAYOUT_THREADS];
+    __shared__ __align__(16) int32_t s_part[2][4 * LAYOUT_THREADS]; // phase 2a partial sums
     __shared__ int32_t s_wsum[4][LAYOUT_WARPS];
     __shared__ uint32_t s_err;
 
@@ -304,15 +258,66 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
     if (tid == 0 && s_err != 0)
         atomicOr(a.ws_barrier + 2, s_err);
 
-    if (!layout_grid_barrier(a.ws_barrier, static_cast<uint32_t>(a.G) + a.barrier_extra, a.barrier_limit_ns)) {
+    if (!grid_barrier_ticket(a.ws_barrier, static_cast<uint32_t>(a.G), a.barrier_extra, a.barrier_limit_ns)) {
         if (tid == 0)
             atomicOr(a.out.status, MOE_DEV_TIMEOUT);
         return;
     }
 
-    // ---- phase 2a: block prefix and totals per logical expert. P threads
-    // share an expert; each sums every P-th block with all its loads in flight.
-    {
+    // ---- phase 2a: block prefix and totals per logical expert. With E_log a
+    // multiple of 4, thread (group g, column c) sums experts 4c..4c+3 over the
+    // blocks g, g+P, ... with 16-byte loads (up to 8 in flight), then the P
+    // groups are merged through shared memory. Otherwise P threads share an
+    // expert and read it 4 bytes at a time.
+    if ((E_log & 3) == 0) {
+        const int E4 = E_log >> 2;
+        const int P = min(32, LAYOUT_THREADS / E4); // E4 <= 512 = LAYOUT_THREADS
+        if (tid < P * E4) {
+            const int c = tid % E4, g = tid / E4;
+            const int4 *col = reinterpret_cast<const int4 *>(a.ws_counts) + c;
+            int4 pre = make_int4(0, 0, 0, 0), tot = make_int4(0, 0, 0, 0);
+            for (int bb0 = g; bb0 < a.G; bb0 += 8 * P) {
+                int4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int bb = bb0 + u * P;
+                    v[u] = bb < a.G ? __ldcg(col + static_cast<int64_t>(bb) * E4) : make_int4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const bool before = bb0 + u * P < b;
+                    tot.x += v[u].x;
+                    tot.y += v[u].y;
+                    tot.z += v[u].z;
+                    tot.w += v[u].w;
+                    pre.x += before ? v[u].x : 0;
+                    pre.y += before ? v[u].y : 0;
+                    pre.z += before ? v[u].z : 0;
+                    pre.w += before ? v[u].w : 0;
+                }
+            }
+            // g * E_log + 4c + i < P * E_log <= 4 * LAYOUT_THREADS: in bounds
+            reinterpret_cast<int4 *>(&s_part[0][0])[tid] = pre;
+            reinterpret_cast<int4 *>(&s_part[1][0])[tid] = tot;
+        }
+        if (b == 0 && tid == LAYOUT_THREADS - 1) {
+            // every block OR-ed its error bits in before the barrier; block 0 reports and clears them
+            s_err = __ldcg(a.ws_barrier + 2);
+            a.ws_barrier[2] = 0;
+        }
+        __syncthreads();
+        for (int e = tid; e < E_log; e += LAYOUT_THREADS) {
+            int32_t pre = 0, tot = 0;
+            for (int g = 0; g < P; ++g) {
+                pre += s_part[0][g * E_log + e];
+                tot += s_part[1][g * E_log + e];
+            }
+            s_pre[e] = pre;
+            s_cnt[e] = tot;
+            s_repl[e] = -1;
+        }
+        __syncthreads();
+    } else {
         const int P = E_log >= LAYOUT_THREADS ? 1 : min(32, LAYOUT_THREADS / E_log);
         for (int item = tid; item < E_log * P; item += LAYOUT_THREADS) {
             const int e = item % E_log, part = item / E_log;
@@ -340,7 +345,6 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
             }
         }
         if (b == 0 && tid == LAYOUT_THREADS - 1) {
-            // every block OR-ed its error bits in before the barrier; block 0 reports and clears them
             s_err = __ldcg(a.ws_barrier + 2);
             a.ws_barrier[2] = 0;
         }
@@ -397,7 +401,7 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
             const int q = q0 + u;
             const int32_t raw = q < E ? s_raw[q] : 0;
             const int32_t local = layout_local_tokens(a, raw);
-            rows[u] = q < E ? (a.C > 0 ? a.C_local : ((local + a.A - 1) / a.A) * a.A) : 0;
+            rows[u] = q < E ? (a.C > 0 ? a.C_local : (a.A == 1 ? local : ((local + a.A - 1) / a.A) * a.A)) : 0;
             sum += rows[u];
             valid += raw;
             kept += local;

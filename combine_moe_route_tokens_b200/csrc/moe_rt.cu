@@ -48,6 +48,8 @@ LayoutKernel layout_kernel_for(int ipl)
     }
 }
 
+constexpr int LAYOUT_IPLS[] = {0, 1, 2, 4, 8};
+
 // Programmatic dependent launch is used unless the driver refuses it for a
 // kind of launch; then that kind falls back to ordinary stream order.
 std::atomic<bool> g_pdl_plain{true};
@@ -99,6 +101,7 @@ int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, void *s
 struct DeviceInfo {
     int sms = 0;
     int smem_optin = 0;
+    int layout_dyn_max = 0; // dynamic shared memory the layout kernels may take (opt-in limit less their static part)
     bool ready = false;
 };
 
@@ -118,11 +121,20 @@ int device_info(DeviceInfo *out)
             cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
             return MOE_ERR_CUDA;
         cudaError_t e = cudaSuccess;
-        for (int ipl : {0, 1, 2, 4, 8})
+        int static_max = 0;
+        for (int ipl : LAYOUT_IPLS) {
+            cudaFuncAttributes fa;
+            if (e == cudaSuccess)
+                e = cudaFuncGetAttributes(&fa, layout_kernel_for(ipl));
+            if (e == cudaSuccess && static_cast<int>(fa.sharedSizeBytes) > static_max)
+                static_max = static_cast<int>(fa.sharedSizeBytes);
+        }
+        d.layout_dyn_max = d.smem_optin - static_max;
+        for (int ipl : LAYOUT_IPLS)
             if (e == cudaSuccess)
                 e = cudaFuncSetAttribute(layout_kernel_for(ipl), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         d.smem_optin - 16 * 1024);
-        if (e != cudaSuccess)
+                                         d.layout_dyn_max);
+        if (e != cudaSuccess || d.layout_dyn_max <= 0)
             return MOE_ERR_CUDA;
         d.ready = true;
     }
@@ -347,7 +359,7 @@ int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, c
     if (lg.G > dev.sms)
         return MOE_ERR_UNSUPPORTED;
     const size_t smem = layout_smem_words(problem->E_log, d.E) * 4;
-    if (smem > static_cast<size_t>(dev.smem_optin - 16 * 1024))
+    if (smem > static_cast<size_t>(dev.layout_dyn_max))
         return MOE_ERR_UNSUPPORTED;
 
     LayoutArgs a;

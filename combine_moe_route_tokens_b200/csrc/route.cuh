@@ -38,35 +38,23 @@ __device__ __forceinline__ float route_unkey(uint32_t k)
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-template <int VPL> // logits held per lane: E <= 32 * VPL
-__global__ void __launch_bounds__(ROUTE_WARPS_PER_BLOCK * 32)
-    route_topk_kernel(const float *__restrict__ logits, const uint8_t *__restrict__ mask, int64_t N, int E, int k,
-                      int32_t *__restrict__ topk_idx, float *__restrict__ topk_probs)
+// Lane l loads experts l, l+32, ... of one token's logits (-inf past E).
+template <int VPL>
+__device__ __forceinline__ void route_load(const float *__restrict__ row, int E, int lane, float (&v)[VPL])
 {
-    pdl_trigger();
-    pdl_wait();
-    const int lane = threadIdx.x & 31;
-    const int64_t t = static_cast<int64_t>(blockIdx.x) * ROUTE_WARPS_PER_BLOCK + (threadIdx.x >> 5);
-    if (t >= N)
-        return;
-    int32_t *idx_out = topk_idx + t * k;
-    float *prob_out = topk_probs + t * k;
-    if (mask != nullptr && mask[t] != 0) {
-        if (lane < k) {
-            idx_out[lane] = -1;
-            prob_out[lane] = 0.0f;
-        }
-        return;
-    }
-
-    const float *row = logits + t * E;
-    float v[VPL];
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
         const int e = i * 32 + lane;
         v[i] = e < E ? __ldg(row + e) : -INFINITY;
     }
+}
 
+// Softmax + top-k of one token held by the warp (route_load layout). Lane j < k
+// ends with the j-th chosen expert id and its prob; other lanes get -1 / 0.
+// Every lane of the warp must call it.
+template <int VPL>
+__device__ __forceinline__ void route_select(const float (&v)[VPL], int E, int k, int lane, int32_t &id, float &prob)
+{
     float m = v[0];
 #pragma unroll
     for (int i = 1; i < VPL; ++i)
@@ -110,9 +98,38 @@ __global__ void __launch_bounds__(ROUTE_WARPS_PER_BLOCK * 32)
             my_key = wmax;
         }
     }
-    if (lane < k) { // lane j turns the j-th winning logit into its prob
-        idx_out[lane] = my_id;
-        prob_out[lane] = expf(route_unkey(my_key) - m) / s;
+    id = lane < k ? my_id : -1;
+    prob = lane < k ? expf(route_unkey(my_key) - m) / s : 0.0f; // lane j turns the j-th winning logit into its prob
+}
+
+template <int VPL> // logits held per lane: E <= 32 * VPL
+__global__ void __launch_bounds__(ROUTE_WARPS_PER_BLOCK * 32)
+    route_topk_kernel(const float *__restrict__ logits, const uint8_t *__restrict__ mask, int64_t N, int E, int k,
+                      int32_t *__restrict__ topk_idx, float *__restrict__ topk_probs)
+{
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * ROUTE_WARPS_PER_BLOCK + (threadIdx.x >> 5);
+    if (t >= N)
+        return;
+    int32_t *idx_out = topk_idx + t * k;
+    float *prob_out = topk_probs + t * k;
+    if (mask != nullptr && mask[t] != 0) {
+        if (lane < k) {
+            idx_out[lane] = -1;
+            prob_out[lane] = 0.0f;
+        }
+        return;
+    }
+    float v[VPL];
+    route_load(logits + t * E, E, lane, v);
+    int32_t id;
+    float prob;
+    route_select(v, E, k, lane, id, prob);
+    if (lane < k) {
+        idx_out[lane] = id;
+        prob_out[lane] = prob;
     }
 }
 

@@ -437,3 +437,4 @@ def test_dedup_path(case):
     out = moe.moe_dedup_combine(p, V, partial)
     assert np.array_equal(host(out), oracle.combine(exp_partial, D["token_rank_row"], None))
     assert G.status() == 0 and V.status() == 0
+
