@@ -237,6 +237,28 @@ __global__ void __launch_bounds__(256) dedup_fill_kernel(DedupFillArgs a)
     o.recv_pad_mask[w] = t < 0 ? 1 : 0;
     uint8_t *map_row = o.recv_routing_map + w * E_loc;
     float *prob_row = o.recv_probs + w * E_loc;
+    // the token's slots, eight at a time, all loads of a batch in flight together
+    // (the first batch before the row is zeroed, so that nothing waits in between)
+    constexpr int B = 8;
+    int32_t dj[B], qj[B];
+    float wj[B];
+    auto load_batch = [&](int j0) {
+#pragma unroll
+        for (int u = 0; u < B; ++u) {
+            const int j = j0 + u;
+            dj[u] = -1;
+            qj[u] = -1;
+            wj[u] = 0.0f;
+            if (t >= 0 && j < k) {
+                const int64_t s = static_cast<int64_t>(t) * k + j;
+                dj[u] = __ldg(a.dest_row + s);
+                qj[u] = __ldg(a.phys_idx + s);
+                if (a.probs != nullptr)
+                    wj[u] = __ldg(a.probs + s);
+            }
+        }
+    };
+    load_batch(0);
     if ((E_loc & 15) == 0) {
         for (int c = 0; c < E_loc; c += 16)
             *reinterpret_cast<uint4 *>(map_row + c) = make_uint4(0, 0, 0, 0);
@@ -248,56 +270,95 @@ __global__ void __launch_bounds__(256) dedup_fill_kernel(DedupFillArgs a)
             prob_row[c] = 0.0f;
         }
     }
-    for (int j = 0; j < k; ++j) {
-        int32_t local = -1;
-        float wt = 0.0f;
-        if (t >= 0) {
-            const int32_t d = __ldg(a.dest_row + static_cast<int64_t>(t) * k + j);
-            const int32_t q = __ldg(a.phys_idx + static_cast<int64_t>(t) * k + j);
-            if (d >= 0 && q >= 0 && q / E_loc == r) {
-                local = q - r * E_loc;
-                wt = a.probs != nullptr ? __ldg(a.probs + static_cast<int64_t>(t) * k + j) : 0.0f;
+    for (int j0 = 0; j0 < k; j0 += B) {
+        if (j0 > 0)
+            load_batch(j0);
+#pragma unroll
+        for (int u = 0; u < B; ++u) {
+            const int j = j0 + u;
+            if (j >= k)
+                break;
+            int32_t local = -1;
+            float wt = 0.0f;
+            if (dj[u] >= 0 && qj[u] >= 0 && qj[u] / E_loc == r) {
+                local = qj[u] - r * E_loc;
+                wt = wj[u];
                 map_row[local] = 1;
                 prob_row[local] = wt;
             }
+            o.recv_topk_idx[w * k + j] = local;
+            o.recv_topk_weights[w * k + j] = wt;
         }
-        o.recv_topk_idx[w * k + j] = local;
-        o.recv_topk_weights[w * k + j] = wt;
     }
 }
 
 // Receiver-side partials, token-major: one thread per 16-byte column chunk of
-// one token. Lane j holds slot j's row and prob and the rank owning that row
-// (from the layout's rank offsets); lane r holds the token's receive row on
-// rank r. All kept slot chunks are loaded up front; then, for each rank, the
-// ballot of its slots is folded in ascending slot order into one partial,
-// stored once. Every kept row is read once and every partial written once.
+// one token. Lane j holds slot j's row, prob and owning rank (from the layout's
+// rank offsets). The kept slots are put in (rank, slot) order with a few warp
+// ballots; the chunks are loaded in that order, all in flight at once, and
+// folded with one accumulator that is stored as rank r's partial and reset
+// whenever the rank changes, so each rank's slots accumulate in ascending slot
+// order from +0 and every multiply-add is issued once. Every kept row is read
+// once and every partial written once. The trailing `zero_blocks` CTAs zero
+// the receive rows past num_recv.
 struct DedupCombineArgs {
-    const uint4 *y;              // [rows_max, V] expert outputs in send-buffer order
-    const int32_t *dest_row;     // [N, k]
-    const float *probs;          // [N, k] or null (unit weights)
-    const int32_t *rank_offsets; // [R+1] of the layout
+    const uint4 *y;                // [rows_max, V] expert outputs in send-buffer order
+    const int32_t *dest_row;       // [N, k]
+    const float *probs;            // [N, k] or null (unit weights)
+    const int32_t *rank_offsets;   // [R+1] of the layout
     const int32_t *token_rank_row; // [N, R]
-    uint4 *partial;              // [recv_max, V]
+    const int32_t *num_recv;       // [1]
+    uint4 *partial;                // [recv_max, V]
     uint32_t *status;
     int64_t N;
     int64_t recv_max;
     int64_t rows_max;
     int32_t k, R, V, nchunks;
+    int64_t token_blocks; // N * nchunks; the blocks after them zero the tail
 };
 
+__device__ __forceinline__ void dedup_zero_tail(const DedupCombineArgs &a, int64_t worker, int64_t nworkers)
+{
+    const int64_t first = __ldg(a.num_recv);
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    const int64_t total = (a.recv_max - first) * a.V;
+    for (int64_t i = worker; i < total; i += nworkers)
+        st_u4(a.partial + first * a.V + i, z);
+}
+
+// Lane j < k: position of kept slot j in (rank, slot) order, from one ballot per
+// rank; dropped slots (rank R) come last. Returns the number of kept slots.
+__device__ __forceinline__ int dedup_slot_order(int32_t rank, int k, int R, int lane, int32_t &pos)
+{
+    const uint32_t lt = (1u << lane) - 1u;
+    int before = 0; // kept slots of lower ranks
+    pos = 0;
+    for (int r = 0; r < R; ++r) {
+        const uint32_t m = __ballot_sync(0xffffffffu, lane < k && rank == r);
+        if (rank == r)
+            pos = before + __popc(m & lt);
+        before += __popc(m);
+    }
+    return before;
+}
+
 template <int K> // top-k at compile time (1..8); 0 = runtime k <= 32, slots taken eight at a time
-__global__ void __launch_bounds__(256, (K == 0 || K >= 8) ? 3 : 4) dedup_combine_local_kernel(DedupCombineArgs a)
+__global__ void __launch_bounds__(256, 4) dedup_combine_local_kernel(DedupCombineArgs a)
 {
     pdl_trigger();
     pdl_wait();
+    if (blockIdx.x >= a.token_blocks) {
+        dedup_zero_tail(a, (blockIdx.x - a.token_blocks) * blockDim.x + threadIdx.x,
+                        (gridDim.x - a.token_blocks) * blockDim.x);
+        return;
+    }
     const int64_t t = blockIdx.x / a.nchunks;
     const int c = static_cast<int>(blockIdx.x - t * a.nchunks);
     const int v = c * blockDim.x + threadIdx.x;
     const int lane = threadIdx.x & 31;
     const int k = K > 0 ? K : a.k;
     const int R = a.R;
-    // slot metadata
+    // slot metadata: row, prob and owning rank (R for a dropped slot)
     int32_t d = -1;
     float p = 0.0f;
     if (lane < k) {
@@ -310,90 +371,63 @@ __global__ void __launch_bounds__(256, (K == 0 || K >= 8) ? 3 : 4) dedup_combine
     }
     const int32_t rank_end = lane < R ? __ldg(a.rank_offsets + lane + 1) : INT32_MAX;
     const int32_t my_row = lane < R ? __ldg(a.token_rank_row + t * R + lane) : -1;
-    int32_t slot_rank = 0; // ranks whose rows end at or before this slot's row
+    int32_t rank = 0; // ranks whose rows end at or before this slot's row
     for (int r = 0; r < R; ++r)
-        slot_rank += (d >= __shfl_sync(0xffffffffu, rank_end, r)) ? 1 : 0;
+        rank += (d >= __shfl_sync(0xffffffffu, rank_end, r)) ? 1 : 0;
+    if (d < 0)
+        rank = R;
+    int32_t pos;
+    const int kept = dedup_slot_order(rank, k, R, lane, pos);
+    // lane i < kept takes the row, prob and rank of the slot at position i
+    int32_t at = 0;
+    for (int j = 0; j < k; ++j) {
+        const int32_t pj = __shfl_sync(0xffffffffu, pos, j);
+        const bool keptj = __shfl_sync(0xffffffffu, rank, j) < R;
+        at = (keptj && pj == lane) ? j : at;
+    }
+    const int32_t d_at = __shfl_sync(0xffffffffu, d, at);
+    const float p_at = __shfl_sync(0xffffffffu, p, at);
+    const int32_t r_at = __shfl_sync(0xffffffffu, rank, at);
+    // bit i: position i ends a rank's run (the last kept slot, or the next one has another rank)
+    const int32_t r_next = __shfl_down_sync(0xffffffffu, r_at, 1);
+    const uint32_t ends = __ballot_sync(0xffffffffu, lane < kept && (lane == kept - 1 || r_next != r_at));
     const bool active = v < a.V;
     float acc[8];
-    if constexpr (K > 0) {
-        float pj[K];
-        uint4 yj[K];
 #pragma unroll
-        for (int j = 0; j < K; ++j) {
-            const int32_t dj = __shfl_sync(0xffffffffu, d, j);
-            pj[j] = __shfl_sync(0xffffffffu, p, j);
-            yj[j] = make_uint4(0, 0, 0, 0);
-            if (dj >= 0 && active)
-                yj[j] = ld_stream_u4(a.y + static_cast<int64_t>(dj) * a.V + v);
+    for (int e = 0; e < 8; ++e)
+        acc[e] = 0.0f;
+    constexpr int STEP = K > 0 ? K : 8;
+    for (int i0 = 0; i0 < kept; i0 += STEP) {
+        uint4 yi[STEP];
+#pragma unroll
+        for (int u = 0; u < STEP; ++u) {
+            const int32_t di = __shfl_sync(0xffffffffu, d_at, (i0 + u) & 31);
+            if (i0 + u < kept && active)
+                yi[u] = ld_stream_u4(a.y + static_cast<int64_t>(di) * a.V + v);
         }
-        for (int r = 0; r < R; ++r) {
-            const uint32_t m = __ballot_sync(0xffffffffu, lane < k && d >= 0 && slot_rank == r);
-            const int32_t row = __shfl_sync(0xffffffffu, my_row, r);
-            if (m == 0 || !active)
-                continue;
-            if (row < 0 || row >= a.recv_max) { // a view of another layout
-                atomicOr(a.status, MOE_DEV_ROW_RANGE);
-                continue;
-            }
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-                acc[e] = 0.0f;
-#pragma unroll
-            for (int j = 0; j < K; ++j)
-                if ((m >> j) & 1u)
-                    fma8(acc, pj[j], yj[j]);
-            st_u4(a.partial + static_cast<int64_t>(row) * a.V + v, pack8(acc));
-        }
-    } else {
-        for (int r = 0; r < R; ++r) {
-            const uint32_t m = __ballot_sync(0xffffffffu, lane < k && d >= 0 && slot_rank == r);
-            const int32_t row = __shfl_sync(0xffffffffu, my_row, r);
-            if (m == 0)
-                continue;
-            if (row < 0 || row >= a.recv_max) { // a view of another layout
-                if (threadIdx.x == 0)
-                    atomicOr(a.status, MOE_DEV_ROW_RANGE);
-                continue;
-            }
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                acc[e] = 0.0f;
-            for (int j0 = 0; j0 < k; j0 += 8) {
-                int32_t dj[8];
-                float pj[8];
-                uint4 yj[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    dj[u] = __shfl_sync(0xffffffffu, d, (j0 + u) & 31);
-                    pj[u] = __shfl_sync(0xffffffffu, p, (j0 + u) & 31);
-                    if (!((m >> ((j0 + u) & 31)) & 1u) || j0 + u >= k || !active)
-                        dj[u] = -1;
-                    if (dj[u] >= 0)
-                        yj[u] = ld_stream_u4(a.y + static_cast<int64_t>(dj[u]) * a.V + v);
+        for (int u = 0; u < STEP; ++u) {
+            const int i = i0 + u;
+            if (i >= kept)
+                break; // uniform over the warp
+            const float pi = __shfl_sync(0xffffffffu, p_at, i);
+            if (active)
+                fma8(acc, pi, yi[u]);
+            if ((ends >> i) & 1u) { // store rank r's partial and start the next rank from +0
+                const int32_t r = __shfl_sync(0xffffffffu, r_at, i);
+                const int32_t row = __shfl_sync(0xffffffffu, my_row, r);
+                if (active) {
+                    if (row < 0 || row >= a.recv_max) // a view of another layout
+                        atomicOr(a.status, MOE_DEV_ROW_RANGE);
+                    else
+                        st_u4(a.partial + static_cast<int64_t>(row) * a.V + v, pack8(acc));
                 }
 #pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    if (dj[u] >= 0)
-                        fma8(acc, pj[u], yj[u]);
+                for (int e = 0; e < 8; ++e)
+                    acc[e] = 0.0f;
             }
-            if (active)
-                st_u4(a.partial + static_cast<int64_t>(row) * a.V + v, pack8(acc));
         }
     }
-}
-
-// Receive rows no token reaches (past num_recv) get zero partials.
-__global__ void __launch_bounds__(128) dedup_zero_tail_kernel(uint4 *partial, const int32_t *num_recv,
-                                                               int64_t recv_max, int32_t V)
-{
-    pdl_trigger();
-    pdl_wait();
-    const int64_t first = __ldg(num_recv);
-    const uint4 z = make_uint4(0, 0, 0, 0);
-    const int64_t total = (recv_max - first) * V;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-        st_u4(partial + first * V + i, z);
 }
 
 } // namespace moert

@@ -27,6 +27,7 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 
 #include "moe_rt.h"
 #include "grid_barrier.cuh"
@@ -164,7 +165,7 @@ __device__ void layout_placement(const LayoutArgs &a, const int32_t *s_cnt, int3
 }
 
 template <int IPL> // IPL > 0: each lane keeps IPL assignments in registers (sub = 32 * IPL); 0: any sub
-__global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
+__global__ void __launch_bounds__(LAYOUT_THREADS, 1) layout_kernel(LayoutArgs a)
 {
     extern __shared__ __align__(16) uint32_t layout_smem[];
     const int E_log = a.E_log, E = a.E;
@@ -390,9 +391,12 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
                 s_raw[s_repl[e]] = s_cnt[e] / 2;
         __syncthreads();
     }
-    int32_t total_valid, total_kept, total_dropped;
-    {
-        constexpr int PER = 8; // E <= 4096 = LAYOUT_THREADS * PER
+    // exclusive scan of the rows each physical expert owns; the valid / kept /
+    // dropped totals only in block 0, which publishes them. PER experts per
+    // thread: 1 when E <= LAYOUT_THREADS, else 8 (E <= 4096).
+    int32_t total_valid = 0, total_kept = 0, total_dropped = 0;
+    auto scan_rows = [&](auto per_tag) {
+        constexpr int PER = decltype(per_tag)::value;
         const int q0 = tid * PER;
         int32_t rows[PER];
         int32_t sum = 0, valid = 0, kept = 0, dropped = 0;
@@ -401,7 +405,7 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
             const int q = q0 + u;
             const int32_t raw = q < E ? s_raw[q] : 0;
             const int32_t local = layout_local_tokens(a, raw);
-            rows[u] = q < E ? (a.C > 0 ? a.C_local : (a.A == 1 ? local : ((local + a.A - 1) / a.A) * a.A)) : 0;
+            rows[u] = q >= E ? 0 : a.C > 0 ? a.C_local : a.A == 1 ? local : ((local + a.A - 1) / a.A) * a.A;
             sum += rows[u];
             valid += raw;
             kept += local;
@@ -414,30 +418,33 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
             if (lane >= o)
                 inc += n;
         }
+        if (b == 0) { // block-uniform
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            valid += __shfl_xor_sync(0xffffffffu, valid, o);
-            kept += __shfl_xor_sync(0xffffffffu, kept, o);
-            dropped += __shfl_xor_sync(0xffffffffu, dropped, o);
+            for (int o = 16; o > 0; o >>= 1) {
+                valid += __shfl_xor_sync(0xffffffffu, valid, o);
+                kept += __shfl_xor_sync(0xffffffffu, kept, o);
+                dropped += __shfl_xor_sync(0xffffffffu, dropped, o);
+            }
+            if (lane == 0) {
+                s_wsum[1][warp] = valid;
+                s_wsum[2][warp] = kept;
+                s_wsum[3][warp] = dropped;
+            }
         }
         if (lane == 31)
             s_wsum[0][warp] = inc;
-        if (lane == 0) {
-            s_wsum[1][warp] = valid;
-            s_wsum[2][warp] = kept;
-            s_wsum[3][warp] = dropped;
-        }
         __syncthreads();
         int32_t wpre = 0;
-        total_valid = 0;
-        total_kept = 0;
-        total_dropped = 0;
 #pragma unroll
-        for (int w = 0; w < LAYOUT_WARPS; ++w) {
+        for (int w = 0; w < LAYOUT_WARPS; ++w)
             wpre += w < warp ? s_wsum[0][w] : 0;
-            total_valid += s_wsum[1][w];
-            total_kept += s_wsum[2][w];
-            total_dropped += s_wsum[3][w];
+        if (b == 0) {
+#pragma unroll
+            for (int w = 0; w < LAYOUT_WARPS; ++w) {
+                total_valid += s_wsum[1][w];
+                total_kept += s_wsum[2][w];
+                total_dropped += s_wsum[3][w];
+            }
         }
         int32_t run = wpre + inc - sum;
 #pragma unroll
@@ -449,7 +456,11 @@ __global__ void __launch_bounds__(LAYOUT_THREADS) layout_kernel(LayoutArgs a)
         }
         if (tid == LAYOUT_THREADS - 1)
             s_off[E] = run;
-    }
+    };
+    if (E <= LAYOUT_THREADS)
+        scan_rows(std::integral_constant<int, 1>{});
+    else
+        scan_rows(std::integral_constant<int, 8>{});
     __syncthreads();
 
     const moe_layout_t &o = a.out;

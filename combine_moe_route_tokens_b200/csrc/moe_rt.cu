@@ -727,42 +727,32 @@ int moe_dedup_combine_local(const moe_problem_t *problem, const moe_layout_t *la
     const int v32 = ((a.V + 31) / 32) * 32;
     const int threads = v32 % 256 == 0 ? 256 : (v32 % 128 == 0 ? 128 : (v32 % 64 == 0 ? 64 : 32));
     a.nchunks = (a.V + threads - 1) / threads;
-    const int64_t blocks = problem->N * a.nchunks;
-    if (blocks > INT32_MAX)
-        return MOE_ERR_UNSUPPORTED;
-    if (blocks > 0) {
-        const dim3 grid(static_cast<unsigned>(blocks)), block(threads);
-        switch (problem->k) {
-        case 1:
-            rc = launch(dedup_combine_local_kernel<1>, grid, block, 0, stream, false, a);
-            break;
-        case 2:
-            rc = launch(dedup_combine_local_kernel<2>, grid, block, 0, stream, false, a);
-            break;
-        case 4:
-            rc = launch(dedup_combine_local_kernel<4>, grid, block, 0, stream, false, a);
-            break;
-        case 6:
-            rc = launch(dedup_combine_local_kernel<6>, grid, block, 0, stream, false, a);
-            break;
-        case 8:
-            rc = launch(dedup_combine_local_kernel<8>, grid, block, 0, stream, false, a);
-            break;
-        default:
-            rc = launch(dedup_combine_local_kernel<0>, grid, block, 0, stream, false, a);
-            break;
-        }
-        if (rc != MOE_OK)
-            return rc;
-    }
-    // receive rows past num_recv: zero partials (their count is known on the device only)
+    a.num_recv = dedup->num_recv;
+    a.token_blocks = problem->N * a.nchunks;
+    // trailing CTAs zero the receive rows past num_recv (a count known on the device only)
     DeviceInfo dev;
     if ((rc = device_info(&dev)) != MOE_OK)
         return rc;
-    const int64_t tail_work = (recv_max * a.V + 127) / 128;
-    const int64_t tail_blocks = tail_work < 2 * dev.sms ? tail_work : 2 * dev.sms;
-    return launch(dedup_zero_tail_kernel, dim3(static_cast<unsigned>(tail_blocks)), dim3(128), 0, stream, false,
-                  a.partial, static_cast<const int32_t *>(dedup->num_recv), recv_max, a.V);
+    const int64_t tail_work = (recv_max * a.V + threads - 1) / threads;
+    const int64_t zero_blocks = tail_work < 2 * dev.sms ? tail_work : 2 * dev.sms;
+    const int64_t blocks = a.token_blocks + zero_blocks;
+    if (blocks > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    const dim3 grid(static_cast<unsigned>(blocks)), block(threads);
+    switch (problem->k) {
+    case 1:
+        return launch(dedup_combine_local_kernel<1>, grid, block, 0, stream, false, a);
+    case 2:
+        return launch(dedup_combine_local_kernel<2>, grid, block, 0, stream, false, a);
+    case 4:
+        return launch(dedup_combine_local_kernel<4>, grid, block, 0, stream, false, a);
+    case 6:
+        return launch(dedup_combine_local_kernel<6>, grid, block, 0, stream, false, a);
+    case 8:
+        return launch(dedup_combine_local_kernel<8>, grid, block, 0, stream, false, a);
+    default:
+        return launch(dedup_combine_local_kernel<0>, grid, block, 0, stream, false, a);
+    }
 }
 
 int moe_dedup_combine(const moe_problem_t *problem, const moe_dedup_t *dedup, const uint16_t *partial,
