@@ -10,6 +10,7 @@ functions keep the C names:
     moe_combine           out[t] = bf16(sum_j p[t, j] * y[dest_row[t, j]]), fp32, ascending j
     moe_restore_combined  the same over the buffers of TP peers (after TP folding)
     moe_dedup_*           DeepEP-style view: one receive row per (token, rank), two-level combine
+    moe_ep_*              expert-parallel exchange: dispatch into / combine from the ranks' receive buffers
     moe_permute_backward  grad_hidden[t] = bf16(sum_j grad_send[dest_row[t, j]])
     moe_combine_backward  grad_y[row] = bf16(p * grad_out[t]); grad_probs[t, j] = <grad_out[t], y[row]>
 
@@ -58,6 +59,12 @@ __all__ = [
     "moe_combine",
     "moe_restore_combined",
     "DedupView",
+    "EpPlan",
+    "peer_table",
+    "moe_ep_recv_rows_max",
+    "moe_ep_plan",
+    "moe_ep_dispatch",
+    "moe_ep_combine",
     "moe_dedup_layout",
     "moe_dedup_dispatch",
     "moe_dedup_combine_local",
@@ -465,6 +472,101 @@ def moe_restore_combined(problem: Problem, layouts, expert_outs, topk_probs: Opt
     _native.check("moe_restore_combined",
                   _native.lib().moe_restore_combined(ctypes.byref(p), Ls, ys, _ptr(topk_probs), _ptr(out),
                                                      _stream(stream)))
+    return out
+
+
+# ------------------------------------------------- expert-parallel exchange
+
+
+def moe_ep_recv_rows_max(problem: Problem) -> int:
+    """Rows of one rank's receive buffer for the exchange (an upper bound, fixed per problem)."""
+    p = problem.c_struct()
+    v = int(_native.lib().moe_ep_recv_rows_max(ctypes.byref(p)))
+    if v < 0:
+        _native.check("moe_ep_recv_rows_max", v)
+    return v
+
+
+@dataclass
+class EpPlan:
+    """moe_ep_plan outputs for one source rank (device tensors)."""
+
+    base: torch.Tensor                 # [E] int32
+    recv_expert_offsets: torch.Tensor  # [E_loc + 1] int32
+    num_recv: torch.Tensor             # [1] int32
+    status: torch.Tensor               # [1] int32 (MOE_DEV_* bits)
+
+    @classmethod
+    def allocate(cls, problem: Problem, device=None) -> "EpPlan":
+        device = torch.device("cuda") if device is None else torch.device(device)
+        i32 = torch.int32
+        return cls(base=torch.empty(problem.E, dtype=i32, device=device),
+                   recv_expert_offsets=torch.empty(problem.E_loc + 1, dtype=i32, device=device),
+                   num_recv=torch.empty(1, dtype=i32, device=device),
+                   status=torch.zeros(1, dtype=i32, device=device))
+
+
+def peer_table(buffers, device=None) -> torch.Tensor:
+    """A device array of the buffers' device addresses (rank order), for the exchange calls."""
+    device = buffers[0].device if device is None else torch.device(device)
+    return torch.tensor([b.data_ptr() for b in buffers], dtype=torch.int64, device=device)
+
+
+def moe_ep_plan(problem: Problem, offsets_all: torch.Tensor, src_rank: int, plan: Optional[EpPlan] = None,
+                stream=None) -> EpPlan:
+    """Where this rank's rows go on the owners, and this rank's receive layout.
+
+    ``offsets_all``: [R, E+1] int32, every rank's layout ``expert_offsets`` (gathered by the caller).
+    """
+    _need(offsets_all, "offsets_all", torch.int32, (problem.R, problem.E + 1))
+    if plan is None:
+        plan = EpPlan.allocate(problem, offsets_all.device)
+    p = problem.c_struct()
+    _native.check("moe_ep_plan", _native.lib().moe_ep_plan(
+        ctypes.byref(p), _ptr(offsets_all), int(src_rank), _ptr(plan.base), _ptr(plan.recv_expert_offsets),
+        _ptr(plan.num_recv), _ptr(plan.status), _stream(stream)))
+    return plan
+
+
+def _table(peers, device) -> torch.Tensor:
+    if isinstance(peers, torch.Tensor) and peers.dtype == torch.int64:
+        return peers
+    return peer_table(list(peers), device)
+
+
+def moe_ep_dispatch(problem: Problem, layout: Layout, plan: EpPlan, hidden: torch.Tensor, peer_recv,
+                    stream=None) -> None:
+    """Write this rank's kept rows into the owners' receive buffers (and its padding rows as zeros).
+
+    ``peer_recv``: the R receive buffers ([moe_ep_recv_rows_max, H] bf16 each), or
+    their ``peer_table``.
+    """
+    _need(hidden, "hidden", torch.bfloat16, (problem.N, problem.H), layout.device)
+    table = _table(peer_recv, layout.device)
+    if table.numel() != problem.R:
+        raise ValueError("peer_recv needs one buffer per rank")
+    p = problem.c_struct()
+    L = layout.c_struct()
+    _native.check("moe_ep_dispatch", _native.lib().moe_ep_dispatch(
+        ctypes.byref(p), ctypes.byref(L), _ptr(plan.base), _ptr(hidden), _ptr(table), _stream(stream)))
+
+
+def moe_ep_combine(problem: Problem, layout: Layout, plan: EpPlan, peer_expert_out, topk_probs: Optional[torch.Tensor],
+                   out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out[t] = bf16(fp32 sum over ascending kept j of p[t,j] * (row of slot j on its expert's owner))."""
+    table = _table(peer_expert_out, layout.device)
+    if table.numel() != problem.R:
+        raise ValueError("peer_expert_out needs one buffer per rank")
+    if topk_probs is not None:
+        _need(topk_probs, "topk_probs", torch.float32, (problem.N, problem.k), layout.device)
+    if out is None:
+        out = torch.empty((problem.N, problem.H), dtype=torch.bfloat16, device=layout.device)
+    _need(out, "out", torch.bfloat16, (problem.N, problem.H), layout.device)
+    p = problem.c_struct()
+    L = layout.c_struct()
+    _native.check("moe_ep_combine", _native.lib().moe_ep_combine(
+        ctypes.byref(p), ctypes.byref(L), _ptr(plan.base), _ptr(table), _ptr(topk_probs), _ptr(out),
+        _stream(stream)))
     return out
 
 

@@ -33,7 +33,7 @@ MOE_DEV_ROW_RANGE = 0x4
 MOE_FLAG_NONE = 0
 MOE_FLAG_TEST_BARRIER_TIMEOUT = 0x80000000
 
-ABI_VERSION = 4
+ABI_VERSION = 5
 
 
 class MoeProblem(ctypes.Structure):
@@ -127,6 +127,10 @@ _SIGNATURES = {
     "moe_restore_combined": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP]),
     "moe_permute_backward": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP]),
     "moe_combine_backward": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "moe_ep_recv_rows_max": (ctypes.c_int64, [_PP]),
+    "moe_ep_plan": (ctypes.c_int, [_PP, _VP, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP]),
+    "moe_ep_dispatch": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP]),
+    "moe_ep_combine": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP, _VP]),
     "moe_dedup_rows_max": (ctypes.c_int64, [_PP]),
     "moe_dedup_workspace_bytes": (ctypes.c_int, [_PP, ctypes.POINTER(ctypes.c_size_t)]),
     "moe_dedup_layout": (ctypes.c_int, [_PP, _PL, _VP, _PD, _VP, ctypes.c_size_t, _VP]),

@@ -46,7 +46,18 @@ struct CombineArgs {
     int32_t T;
     const uint4 *ys[MOE_MAX_TP];
     const int32_t *dests[MOE_MAX_TP];
+    // expert-parallel exchange: slot j's row d of expert q sits in the receive
+    // buffer of q's owner at row ep_base[q] + d - ep_offsets[q]
+    const uint4 *const *ep_peers; // [R] device pointers
+    const int32_t *phys_idx;      // [N, k]
+    const int32_t *ep_base;       // [E]
+    const int32_t *ep_offsets;    // [E + 1]
+    int64_t recv_max;
+    int32_t E, E_loc;
 };
+
+// Where the combine reads slot rows from.
+enum CombineSrc : int { SRC_LOCAL = 0, SRC_TP_PEERS = 1, SRC_EP = 2 };
 
 __device__ __forceinline__ void fma8(float (&acc)[8], float p, const uint4 &y)
 {
@@ -123,9 +134,35 @@ __device__ __forceinline__ void load_slot_meta_peers(const CombineArgs &a, int64
     }
 }
 
+// Expert-parallel exchange: lane j < k finds slot j's row in the receive buffer
+// of the rank owning its expert and returns its address (null if the slot has no
+// row or the row lies outside the receive buffer, the latter flagged).
+__device__ __forceinline__ void load_slot_meta_ep(const CombineArgs &a, int64_t t, int k, const uint4 *&row, float &p)
+{
+    const int lane = threadIdx.x & 31;
+    row = nullptr;
+    p = 0.0f;
+    if (lane < k) {
+        p = a.probs != nullptr ? __ldg(a.probs + t * k + lane) : 1.0f;
+        const int32_t d = __ldg(a.dest_row + t * k + lane);
+        const int32_t q = d >= 0 ? __ldg(a.phys_idx + t * k + lane) : -1;
+        if (d >= 0 && (q < 0 || q >= a.E || d >= a.rows_max)) {
+            atomicOr(a.status, MOE_DEV_ROW_RANGE);
+        } else if (d >= 0) {
+            const int64_t r = static_cast<int64_t>(__ldg(a.ep_base + q)) + d - __ldg(a.ep_offsets + q);
+            if (r < 0 || r >= a.recv_max)
+                atomicOr(a.status, MOE_DEV_ROW_RANGE);
+            else
+                row = a.ep_peers[q / a.E_loc] + r * a.V;
+        } else if (d < -1) {
+            atomicOr(a.status, MOE_DEV_ROW_RANGE);
+        }
+    }
+}
+
 // K > 0: top-k fixed at compile time; K == 0: runtime k <= 32.
-// PEERS: gather from the TP peers' buffers (restore) instead of one buffer.
-template <int K, bool PEERS = false>
+// SRC: one buffer, the TP peers' buffers (restore), or the EP receive buffers.
+template <int K, int SRC = SRC_LOCAL>
 __global__ void __launch_bounds__(COMBINE_THREADS, 4) combine_kernel(CombineArgs a)
 {
     pdl_trigger();
@@ -137,35 +174,38 @@ __global__ void __launch_bounds__(COMBINE_THREADS, 4) combine_kernel(CombineArgs
 
     // lane j < k: slot j's source row and weight. One buffer: the row index;
     // TP peers: the row's address in the peer buffer that holds it.
-    using Src = typename std::conditional<PEERS, const uint4 *, int32_t>::type;
+    constexpr bool PTR = SRC != SRC_LOCAL; // slots resolved to addresses
+    using Src = typename std::conditional<PTR, const uint4 *, int32_t>::type;
     Src src;
     float p;
-    if constexpr (PEERS) {
+    if constexpr (SRC == SRC_TP_PEERS) {
         load_slot_meta_peers(a, t, k, src, p);
+    } else if constexpr (SRC == SRC_EP) {
+        load_slot_meta_ep(a, t, k, src, p);
     } else {
         load_slot_meta(a.dest_row, a.probs, t, k, a.rows_max, a.status, src, p);
     }
     auto shfl_src = [&](int j) -> Src {
-        if constexpr (PEERS)
+        if constexpr (PTR)
             return reinterpret_cast<const uint4 *>(
                 __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(src), j));
         else
             return __shfl_sync(0xffffffffu, src, j);
     };
     auto valid = [](Src s) -> bool {
-        if constexpr (PEERS)
+        if constexpr (PTR)
             return s != nullptr;
         else
             return s >= 0;
     };
     auto row_ptr = [&](Src s) -> const uint4 * {
-        if constexpr (PEERS)
+        if constexpr (PTR)
             return s;
         else
             return a.y + static_cast<int64_t>(s) * a.V;
     };
     auto none = []() -> Src {
-        if constexpr (PEERS)
+        if constexpr (PTR)
             return nullptr;
         else
             return -1;

@@ -21,6 +21,7 @@
 #include "permute.cuh"
 #include "combine.cuh"
 #include "dedup.cuh"
+#include "ep.cuh"
 
 namespace {
 
@@ -429,14 +430,15 @@ int moe_permute(const moe_problem_t *problem, const moe_layout_t *layout, const 
     const int64_t blocks = a.zero_blocks + (problem->N * a.pieces + groups - 1) / groups;
     if (blocks > INT32_MAX)
         return MOE_ERR_UNSUPPORTED;
-    return launch(permute_kernel, dim3(static_cast<unsigned>(blocks)), dim3(PERMUTE_THREADS), 0, stream, false, a);
+    return launch(permute_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(PERMUTE_THREADS), 0, stream, false, a);
 }
 
 namespace {
 
 // Grid and launch for the combine kernel; `a` carries everything but the grid
-// shape. PEERS selects the restore variant that gathers from TP peer buffers.
-extern "C++" template <bool PEERS>
+// shape. SRC selects where slot rows are read: one buffer, TP peer buffers
+// (restore) or EP receive buffers.
+extern "C++" template <int SRC>
 int launch_combine_args(CombineArgs a, int k, void *stream)
 {
     // the widest CTA (up to 256 threads) that splits the row into equal parts
@@ -449,17 +451,17 @@ int launch_combine_args(CombineArgs a, int k, void *stream)
     const dim3 grid(static_cast<unsigned>(blocks)), block(threads);
     switch (k) {
     case 1:
-        return launch(combine_kernel<1, PEERS>, grid, block, 0, stream, false, a);
+        return launch(combine_kernel<1, SRC>, grid, block, 0, stream, false, a);
     case 2:
-        return launch(combine_kernel<2, PEERS>, grid, block, 0, stream, false, a);
+        return launch(combine_kernel<2, SRC>, grid, block, 0, stream, false, a);
     case 4:
-        return launch(combine_kernel<4, PEERS>, grid, block, 0, stream, false, a);
+        return launch(combine_kernel<4, SRC>, grid, block, 0, stream, false, a);
     case 6:
-        return launch(combine_kernel<6, PEERS>, grid, block, 0, stream, false, a);
+        return launch(combine_kernel<6, SRC>, grid, block, 0, stream, false, a);
     case 8:
-        return launch(combine_kernel<8, PEERS>, grid, block, 0, stream, false, a);
+        return launch(combine_kernel<8, SRC>, grid, block, 0, stream, false, a);
     default:
-        return launch(combine_kernel<0, PEERS>, grid, block, 0, stream, false, a);
+        return launch(combine_kernel<0, SRC>, grid, block, 0, stream, false, a);
     }
 }
 
@@ -487,7 +489,7 @@ int launch_combine(const moe_problem_t *problem, const moe_layout_t *layout, con
     a.k = problem->k;
     a.V = problem->H / 8;
     a.T = 1;
-    return launch_combine_args<false>(a, problem->k, stream);
+    return launch_combine_args<SRC_LOCAL>(a, problem->k, stream);
 }
 
 } // namespace
@@ -536,7 +538,7 @@ int moe_restore_combined(const moe_problem_t *problem, const moe_layout_t *peer_
         a.ys[q] = reinterpret_cast<const uint4 *>(peer_expert_out[q]);
         a.dests[q] = peer_layouts[q].dest_row;
     }
-    return launch_combine_args<true>(a, problem->k, stream);
+    return launch_combine_args<SRC_TP_PEERS>(a, problem->k, stream);
 }
 
 int64_t moe_dedup_rows_max(const moe_problem_t *problem)
@@ -686,7 +688,7 @@ int moe_dedup_dispatch(const moe_problem_t *problem, const moe_dedup_t *dedup, c
     const int64_t blocks = a.zero_blocks + (problem->N * a.pieces + groups - 1) / groups;
     if (blocks > INT32_MAX)
         return MOE_ERR_UNSUPPORTED;
-    return launch(permute_kernel, dim3(static_cast<unsigned>(blocks)), dim3(PERMUTE_THREADS), 0, stream, false, a);
+    return launch(permute_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(PERMUTE_THREADS), 0, stream, false, a);
 }
 
 int moe_dedup_combine_local(const moe_problem_t *problem, const moe_layout_t *layout, const moe_dedup_t *dedup,
@@ -782,7 +784,145 @@ int moe_dedup_combine(const moe_problem_t *problem, const moe_dedup_t *dedup, co
     a.k = problem->R;
     a.V = problem->H / 8;
     a.T = 1;
-    return launch_combine_args<false>(a, problem->R, stream);
+    return launch_combine_args<SRC_LOCAL>(a, problem->R, stream);
+}
+
+int64_t moe_ep_recv_rows_max(const moe_problem_t *problem)
+{
+    Dims d;
+    const int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    if (d.T != 1 || problem->R > MOE_MAX_EP_RANKS)
+        return MOE_ERR_UNSUPPORTED;
+    // rows one source can send to one rank, times the sources
+    int64_t per = problem->capacity > 0 ? static_cast<int64_t>(d.E_loc) * d.C_local
+                                        : d.NK + static_cast<int64_t>(d.E_loc) * (d.A - 1);
+    if (per > d.rows_max)
+        per = d.rows_max;
+    return per * problem->R;
+}
+
+int moe_ep_plan(const moe_problem_t *problem, const int32_t *offsets_all, int32_t src_rank, int32_t *base,
+                int32_t *recv_expert_offsets, int32_t *num_recv, uint32_t *status, void *stream)
+{
+    Dims d;
+    int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    const int64_t recv_max = moe_ep_recv_rows_max(problem);
+    if (recv_max < 0)
+        return static_cast<int>(recv_max);
+    if (d.E > EP_PLAN_THREADS * EP_PLAN_PER)
+        return MOE_ERR_UNSUPPORTED;
+    if (src_rank < 0 || src_rank >= problem->R || offsets_all == nullptr || base == nullptr ||
+        recv_expert_offsets == nullptr || num_recv == nullptr || status == nullptr)
+        return MOE_ERR_INVALID;
+    if (recv_max > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    EpPlanArgs a;
+    a.offsets_all = offsets_all;
+    a.R = problem->R;
+    a.E = d.E;
+    a.E_loc = d.E_loc;
+    a.src = src_rank;
+    a.recv_max = recv_max;
+    a.base = base;
+    a.recv_expert_offsets = recv_expert_offsets;
+    a.num_recv = num_recv;
+    a.status = status;
+    const size_t smem = (2 * static_cast<size_t>(d.E) + 1) * sizeof(int32_t);
+    return launch(ep_plan_kernel, dim3(1), dim3(EP_PLAN_THREADS), smem, stream, false, a);
+}
+
+int moe_ep_dispatch(const moe_problem_t *problem, const moe_layout_t *layout, const int32_t *base,
+                    const uint16_t *hidden, uint16_t *const *peer_recv, void *stream)
+{
+    Dims d;
+    int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    const int64_t recv_max = moe_ep_recv_rows_max(problem);
+    if (recv_max < 0)
+        return static_cast<int>(recv_max);
+    if ((rc = check_layout(layout, d, false)) != MOE_OK)
+        return rc;
+    if (layout->expert_offsets == nullptr || layout->tokens_per_expert == nullptr || base == nullptr ||
+        peer_recv == nullptr || (d.NK > 0 && layout->phys_idx == nullptr))
+        return MOE_ERR_INVALID;
+    if (problem->N > 0 && (hidden == nullptr || !aligned16(hidden)))
+        return MOE_ERR_INVALID;
+    if (problem->N == 0)
+        return MOE_OK;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev)) != MOE_OK)
+        return rc;
+    PermuteArgs a = {};
+    a.hidden = reinterpret_cast<const uint4 *>(hidden);
+    a.dest_row = layout->dest_row;
+    a.status = layout->status;
+    a.N = problem->N;
+    a.rows_max = d.rows_max;
+    a.k = problem->k;
+    a.V = problem->H / 8;
+    a.group = a.V <= 32 * PERMUTE_CHUNKS ? 32 : (a.V <= 64 * PERMUTE_CHUNKS ? 64 : PERMUTE_THREADS);
+    a.pieces = (a.V + a.group * PERMUTE_CHUNKS - 1) / (a.group * PERMUTE_CHUNKS);
+    a.ep_peers = reinterpret_cast<uint4 *const *>(peer_recv);
+    a.phys_idx = layout->phys_idx;
+    a.ep_base = base;
+    a.ep_offsets = layout->expert_offsets;
+    a.ep_tokens = layout->tokens_per_expert;
+    a.recv_max = recv_max;
+    a.E = d.E;
+    a.E_loc = d.E_loc;
+    // padding rows exist only with a capacity or a row alignment: one warp per expert
+    const bool pads = problem->capacity > 0 || d.A > 1;
+    const int64_t zb = pads ? (d.E + PERMUTE_THREADS / 32 - 1) / (PERMUTE_THREADS / 32) : 0;
+    a.zero_blocks = static_cast<int32_t>(zb < 4 * dev.sms ? zb : 4 * dev.sms);
+    const int64_t groups = PERMUTE_THREADS / a.group;
+    const int64_t blocks = a.zero_blocks + (problem->N * a.pieces + groups - 1) / groups;
+    if (blocks > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    return launch(permute_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(PERMUTE_THREADS), 0, stream, false, a);
+}
+
+int moe_ep_combine(const moe_problem_t *problem, const moe_layout_t *layout, const int32_t *base,
+                   const uint16_t *const *peer_expert_out, const float *topk_probs, uint16_t *out, void *stream)
+{
+    Dims d;
+    int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    const int64_t recv_max = moe_ep_recv_rows_max(problem);
+    if (recv_max < 0)
+        return static_cast<int>(recv_max);
+    if ((rc = check_layout(layout, d, false)) != MOE_OK)
+        return rc;
+    if (layout->expert_offsets == nullptr || base == nullptr || peer_expert_out == nullptr ||
+        (d.NK > 0 && layout->phys_idx == nullptr))
+        return MOE_ERR_INVALID;
+    if (problem->N == 0)
+        return MOE_OK;
+    if (out == nullptr || !aligned16(out))
+        return MOE_ERR_INVALID;
+    CombineArgs a = {};
+    a.dest_row = layout->dest_row;
+    a.probs = topk_probs;
+    a.out = reinterpret_cast<uint4 *>(out);
+    a.status = layout->status;
+    a.N = problem->N;
+    a.rows_max = d.rows_max;
+    a.k = problem->k;
+    a.V = problem->H / 8;
+    a.T = 1;
+    a.ep_peers = reinterpret_cast<const uint4 *const *>(peer_expert_out);
+    a.phys_idx = layout->phys_idx;
+    a.ep_base = base;
+    a.ep_offsets = layout->expert_offsets;
+    a.recv_max = recv_max;
+    a.E = d.E;
+    a.E_loc = d.E_loc;
+    return launch_combine_args<SRC_EP>(a, problem->k, stream);
 }
 
 int moe_combine_backward(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *grad_out,

@@ -22,6 +22,7 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 
 #include "moe_rt.h"
 #include "ptx.cuh"
@@ -44,7 +45,39 @@ struct PermuteArgs {
     int32_t group;       // threads per token piece: 32, 64 or 128
     int32_t pieces;      // pieces per token
     int32_t zero_blocks; // leading CTAs that zero pad rows
+    // expert-parallel exchange: slot j's row d of expert q goes to the receive
+    // buffer of q's owner, row ep_base[q] + d - ep_offsets[q]; the leading CTAs
+    // zero this source's padding rows there (rows tokens[q] .. of each expert)
+    uint4 *const *ep_peers;     // [R] device pointers
+    const int32_t *phys_idx;    // [N, k]
+    const int32_t *ep_base;     // [E]
+    const int32_t *ep_offsets;  // [E + 1]
+    const int32_t *ep_tokens;   // [E] tokens_per_expert
+    int64_t recv_max;
+    int32_t E, E_loc;
 };
+
+// Expert-parallel exchange: zero this source's padding rows of every expert in
+// the owners' receive buffers; one warp per expert at a time.
+__device__ __forceinline__ void ep_zero_pad_rows_warp(const PermuteArgs &a, int64_t worker, int64_t nworkers)
+{
+    const int lane = threadIdx.x & 31;
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (int64_t q = worker; q < a.E; q += nworkers) {
+        const int32_t rows = __ldg(a.ep_offsets + q + 1) - __ldg(a.ep_offsets + q);
+        const int32_t first = __ldg(a.ep_tokens + q);
+        const int64_t b = __ldg(a.ep_base + q);
+        if (b < 0 || b + rows > a.recv_max) {
+            if (lane == 0 && rows > first)
+                atomicOr(a.status, MOE_DEV_ROW_RANGE);
+            continue;
+        }
+        uint4 *dst = a.ep_peers[q / a.E_loc];
+        for (int32_t i = first; i < rows; ++i)
+            for (int32_t c = lane; c < a.V; c += 32)
+                st_u4(dst + (b + i) * a.V + c, z);
+    }
+}
 
 // Zero-fill every row r of `base` (V 16-byte chunks each) with pad_mask[r] != 0,
 // for r = worker, worker + nworkers, ... ; one warp per worker.
@@ -67,16 +100,21 @@ __device__ __forceinline__ void zero_pad_rows_warp(uint4 *base, const uint8_t *p
     }
 }
 
+// EP: the destinations are rows of the experts' owners' receive buffers.
+template <bool EP = false>
 __global__ void __launch_bounds__(PERMUTE_THREADS) permute_kernel(PermuteArgs a)
 {
-    __shared__ int32_t s_dest[PERMUTE_THREADS / 32][32];
+    using Dst = typename std::conditional<EP, uint4 *, int32_t>::type;
+    __shared__ Dst s_dest[PERMUTE_THREADS / 32][32];
     pdl_trigger();
     pdl_wait();
     if (blockIdx.x < static_cast<uint32_t>(a.zero_blocks)) {
         const int64_t per = PERMUTE_THREADS / 32;
-        zero_pad_rows_warp(a.send, a.pad_mask, a.rows_max, a.V,
-                           static_cast<int64_t>(blockIdx.x) * per + (threadIdx.x >> 5),
-                           static_cast<int64_t>(a.zero_blocks) * per);
+        const int64_t worker = static_cast<int64_t>(blockIdx.x) * per + (threadIdx.x >> 5);
+        if constexpr (EP)
+            ep_zero_pad_rows_warp(a, worker, static_cast<int64_t>(a.zero_blocks) * per);
+        else
+            zero_pad_rows_warp(a.send, a.pad_mask, a.rows_max, a.V, worker, static_cast<int64_t>(a.zero_blocks) * per);
         return;
     }
     const int groups = PERMUTE_THREADS / a.group;
@@ -92,14 +130,33 @@ __global__ void __launch_bounds__(PERMUTE_THREADS) permute_kernel(PermuteArgs a)
             atomicOr(a.status, MOE_DEV_ROW_RANGE);
             d = -1;
         }
-        s_dest[g][gt] = d;
+        if constexpr (EP) {
+            uint4 *dst = nullptr;
+            if (d >= 0) {
+                const int32_t q = __ldg(a.phys_idx + t * a.k + gt);
+                const int64_t r = q >= 0 && q < a.E
+                                      ? static_cast<int64_t>(__ldg(a.ep_base + q)) + d - __ldg(a.ep_offsets + q)
+                                      : -1;
+                if (r < 0 || r >= a.recv_max)
+                    atomicOr(a.status, MOE_DEV_ROW_RANGE);
+                else
+                    dst = a.ep_peers[q / a.E_loc] + r * a.V;
+            }
+            s_dest[g][gt] = dst;
+        } else {
+            s_dest[g][gt] = d;
+        }
     }
     __syncthreads();
     if (!active)
         return;
     bool any = false; // a token whose every slot was dropped is not read at all
-    for (int j = 0; j < a.k; ++j)
-        any |= s_dest[g][j] >= 0;
+    for (int j = 0; j < a.k; ++j) {
+        if constexpr (EP)
+            any |= s_dest[g][j] != nullptr;
+        else
+            any |= s_dest[g][j] >= 0;
+    }
     if (!any)
         return;
     const int32_t c0 = piece * (a.group * PERMUTE_CHUNKS) + gt;
@@ -112,10 +169,17 @@ __global__ void __launch_bounds__(PERMUTE_THREADS) permute_kernel(PermuteArgs a)
             v[c] = ld_stream_u4(src + idx);
     }
     for (int j = 0; j < a.k; ++j) {
-        const int32_t d = s_dest[g][j];
-        if (d < 0)
-            continue;
-        uint4 *dst = a.send + static_cast<int64_t>(d) * a.V;
+        uint4 *dst;
+        if constexpr (EP) {
+            dst = s_dest[g][j];
+            if (dst == nullptr)
+                continue;
+        } else {
+            const int32_t d = s_dest[g][j];
+            if (d < 0)
+                continue;
+            dst = a.send + static_cast<int64_t>(d) * a.V;
+        }
 #pragma unroll
         for (int c = 0; c < PERMUTE_CHUNKS; ++c) {
             const int32_t idx = c0 + c * a.group;

@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-#define MOE_RT_ABI_VERSION 4
+#define MOE_RT_ABI_VERSION 5
 
 /* Every entry point is exported; everything else in the library is hidden. */
 #if defined(__GNUC__)
@@ -332,6 +332,72 @@ MOE_API int moe_dedup_combine_local(const moe_problem_t *problem, const moe_layo
  *   partial [recv_max, H] bf16; out [N, H] bf16 */
 MOE_API int moe_dedup_combine(const moe_problem_t *problem, const moe_dedup_t *dedup, const uint16_t *partial,
                               uint16_t *out, void *stream);
+
+/*
+ * Expert-parallel exchange between R ranks ([Megatron MoE] all-to-all token
+ * dispatcher: every rank's permuted rows go to the rank owning their expert,
+ * which orders what it received by local expert; [Megatron MORI]: dispatch
+ * writes into the receivers' buffers with the permute fused in, and combine
+ * reads the expert outputs back). Every rank runs moe_dispatch_layout on its own
+ * tokens with the same problem (tp_size 1); the ranks' receive buffers are given
+ * as device arrays of R device pointers, which may point into other GPUs' memory
+ * mapped into this process (peer access) or, on one GPU, to separate buffers.
+ * Receive layout of rank r: its experts ascending; within an expert the source
+ * ranks ascending; each source's rows for that expert in its own send-buffer
+ * order, its padding rows (capacity / alignment) included as zeros. Rows past a
+ * rank's num_recv are left untouched. The caller orders the steps across ranks:
+ * every rank's plan before its dispatch, every dispatch into a buffer before that
+ * buffer's experts run, the experts before the combines that read them.
+ * Pinned reading: the receive order above is the plainest one the pages' all-to-all
+ * plus sort-by-local-expert gives (sources ascending within an expert).
+ */
+#define MOE_MAX_EP_RANKS 64
+
+/* Rows of one rank's receive buffer: R x (rows one source can send to one rank:
+ * E_loc*ceil(C/T) with a capacity, else N*k + E_loc*(row_align-1), at most rows_max).
+ * Negative MOE_ERR_* for an invalid problem, MOE_ERR_UNSUPPORTED for tp_size > 1
+ * or R > MOE_MAX_EP_RANKS. Host only. */
+MOE_API int64_t moe_ep_recv_rows_max(const moe_problem_t *problem);
+
+/*
+ * Plan of the exchange for source rank src_rank, one small launch:
+ *   offsets_all          [R][E+1] int32: every rank's layout expert_offsets (the
+ *                        caller gathers them, e.g. with an all-gather)
+ *   base                 [E] int32 out: the receive row on expert q's owner where
+ *                        this rank's rows for q start
+ *   recv_expert_offsets  [E_loc+1] int32 out: this rank's receive layout by local expert
+ *   num_recv             [1] int32 out: rows this rank receives
+ *   status               [1] MOE_DEV_* bits (MOE_DEV_ROW_RANGE if a receive buffer
+ *                        of moe_ep_recv_rows_max rows cannot hold the exchange)
+ * Limit: E <= 4096 physical experts.
+ */
+MOE_API int moe_ep_plan(const moe_problem_t *problem, const int32_t *offsets_all, int32_t src_rank, int32_t *base,
+                        int32_t *recv_expert_offsets, int32_t *num_recv, uint32_t *status, void *stream);
+
+/*
+ * Dispatch with the exchange fused in: for every kept slot (t, j) of expert q,
+ * peer_recv[q / E_loc][base[q] + dest_row[t,j] - expert_offsets[q]] = hidden[t];
+ * this rank's padding rows of every expert are zeroed there.
+ *   layout     this rank's layout (phys_idx, dest_row, expert_offsets, tokens_per_expert, status)
+ *   base       [E] from moe_ep_plan for this rank
+ *   hidden     [N, H] bf16; peer_recv: device array of R device pointers, each a
+ *              [moe_ep_recv_rows_max, H] bf16 receive buffer
+ */
+MOE_API int moe_ep_dispatch(const moe_problem_t *problem, const moe_layout_t *layout, const int32_t *base,
+                            const uint16_t *hidden, uint16_t *const *peer_recv, void *stream);
+
+/*
+ * Combine with the exchange fused in: out[t] = bf16_rn( fp32 fmaf chain over
+ * ascending kept j of p[t,j] * y_r[base[q] + dest_row[t,j] - expert_offsets[q]] ),
+ * q = phys_idx[t,j], r = q / E_loc: the same result as moe_combine over this
+ * rank's own send-buffer order, bit for bit.
+ *   peer_expert_out  device array of R device pointers, rank r's expert output
+ *                    in its receive-buffer order
+ *   topk_probs [N, k] fp32 or NULL (unit weights); out [N, H] bf16
+ */
+MOE_API int moe_ep_combine(const moe_problem_t *problem, const moe_layout_t *layout, const int32_t *base,
+                           const uint16_t *const *peer_expert_out, const float *topk_probs, uint16_t *out,
+                           void *stream);
 
 /*
  * Backward of permute ([Megatron MORI]: dispatch backward sums the row

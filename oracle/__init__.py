@@ -15,6 +15,7 @@ from .oracle import (
     permute,
     combine,
     restore_combined,
+    ep_exchange,
     dedup_layout,
     dedup_combine_local,
     permute_backward,
@@ -33,6 +34,7 @@ __all__ = [
     "permute",
     "combine",
     "restore_combined",
+    "ep_exchange",
     "dedup_layout",
     "dedup_combine_local",
     "permute_backward",

@@ -358,6 +358,42 @@ def restore_combined(expert_outs, dest_rows, topk_probs: Optional[np.ndarray]) -
     return out
 
 
+def ep_exchange(layouts, sends, R: int):
+    """The expert-parallel exchange between R ranks ([Megatron MoE] all-to-all token
+    dispatcher: each rank's permuted rows go to the rank owning their expert, which
+    then sorts what it received by local expert; [Megatron MORI] dispatch into the
+    receivers' buffers, combine reading the expert outputs back).
+
+    ``layouts[s]`` / ``sends[s]``: source rank s's layout (``expert_offsets``,
+    ``tokens_per_expert``) and send buffer. Rank r receives, for each of its experts
+    q in ascending order and within q for each source s in ascending order, the rows
+    that s holds for q (its padding rows included, as zeros).
+
+    Returns ``recv`` (per rank: [rows, H]), ``recv_expert_offsets`` (per rank:
+    [E_loc + 1], where each local expert's rows start) and ``base`` (per source:
+    [E], the receive row on q's owner where source s's rows for q start).
+    """
+    S = len(layouts)
+    E = len(layouts[0]["expert_offsets"]) - 1
+    E_loc = E // R
+    H = sends[0].shape[1]
+    recv, recv_off = [], []
+    base = [np.zeros(E, np.int64) for _ in range(S)]
+    for r in range(R):
+        blocks, offs, pos = [], [], 0
+        for q in range(r * E_loc, (r + 1) * E_loc):
+            offs.append(pos)
+            for s in range(S):
+                lo, hi = int(layouts[s]["expert_offsets"][q]), int(layouts[s]["expert_offsets"][q + 1])
+                base[s][q] = pos
+                blocks.append(sends[s][lo:hi])
+                pos += hi - lo
+        offs.append(pos)
+        recv.append(np.concatenate(blocks, axis=0) if blocks else np.zeros((0, H), np.uint16))
+        recv_off.append(np.asarray(offs, np.int64))
+    return recv, recv_off, base
+
+
 def permute_backward(grad_send: np.ndarray, dest_row: np.ndarray) -> np.ndarray:
     grad_send = _c(grad_send, np.uint16)
     dest_row = _c(dest_row, np.int32)

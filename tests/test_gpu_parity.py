@@ -438,3 +438,49 @@ def test_dedup_path(case):
     assert np.array_equal(host(out), oracle.combine(exp_partial, D["token_rank_row"], None))
     assert G.status() == 0 and V.status() == 0
 
+
+# ------------------------------------------------- expert-parallel exchange
+
+EP_CASES = [
+    # R, N, H, k, E_log, C, replicas, row_align
+    (2, 300, 64, 2, 8, 0, 0, 0),
+    (4, 1000, 136, 4, 16, 0, 0, 0),
+    (4, 2000, 264, 4, 16, 80, 0, 0),  # capacity: drops and padding rows
+    (4, 1500, 72, 4, 16, 0, 4, 0),  # reroute: one replica slot per rank
+    (4, 1200, 40, 3, 16, 0, 0, 8),  # alignment padding, k = 3
+    (8, 2048, 1024, 8, 64, 0, 0, 0),  # 8 ranks, top-8
+]
+
+
+@pytest.mark.parametrize("case", EP_CASES, ids=[f"R{c[0]}_N{c[1]}_H{c[2]}_k{c[3]}_C{c[5]}_rep{c[6]}_A{c[7]}"
+                                                for c in EP_CASES])
+def test_ep_exchange(case):
+    """R ranks' dispatch into each other's receive buffers and the combine back, against the oracle."""
+    R, N, H, k, E_log, C, reps, A = case
+    p = moe.Problem(N=N, H=H, k=k, E_log=E_log, R=R, capacity=C, num_replicas=reps, row_align=A)
+    srcs = [_small_case(N, H, k, E_log, R, C, reps, 0.05, seed=1000 * R + s, zipf=1.3) for s in range(R)]
+    layouts = [moe.moe_dispatch_layout(p, dev(idx), dev(probs)) for idx, probs, _ in srcs]
+    offsets_all = torch.stack([G["expert_offsets"] for G in layouts])
+    plans = [moe.moe_ep_plan(p, offsets_all, s) for s in range(R)]
+    RR = moe.moe_ep_recv_rows_max(p)
+    canary = torch.tensor(0x7F7F, dtype=torch.int16).view(torch.bfloat16).item()
+    recv = [torch.full((RR, H), canary, dtype=torch.bfloat16, device="cuda") for _ in range(R)]
+    table = moe.peer_table(recv)
+    for s, (_, _, hidden) in enumerate(srcs):
+        moe.moe_ep_dispatch(p, layouts[s], plans[s], dev(hidden), table)
+    outs = [moe.moe_ep_combine(p, layouts[s], plans[s], table, dev(srcs[s][1])) for s in range(R)]  # identity experts
+    torch.cuda.synchronize()
+    L_or = [oracle.layout(idx, probs, E_log=E_log, R=R, C=C, num_replicas=reps, align=A) for idx, probs, _ in srcs]
+    sends = [oracle.permute(h, L["dest_row"], L["rows_max"]) for (_, _, h), L in zip(srcs, L_or)]
+    rv, roff, base = oracle.ep_exchange(L_or, sends, R)
+    for r in range(R):
+        n = len(rv[r])
+        got = host(recv[r])
+        assert int(host(plans[r].num_recv)[0]) == n
+        assert np.array_equal(host(plans[r].recv_expert_offsets), roff[r])
+        assert np.array_equal(got[:n], rv[r])
+        assert np.all(got[n:] == 0x7F7F)  # rows past num_recv are left alone
+    for s in range(R):
+        assert np.array_equal(host(plans[s].base), base[s])
+        assert np.array_equal(host(outs[s]), oracle.combine(sends[s], L_or[s]["dest_row"], srcs[s][1]))
+        assert layouts[s].status() == 0 and int(host(plans[s].status)[0]) == 0
