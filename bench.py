@@ -318,6 +318,106 @@ class Step:
         return out
 
 
+class EpStep:
+    """One step of the expert-parallel exchange between R ranks simulated on this GPU.
+
+    The workload's N tokens are split evenly over the R ranks. Every rank routes
+    and lays out its own tokens; the layouts write their expert_offsets straight
+    into the rows of one [R, E+1] table (on several GPUs: an all-gather); every
+    rank plans, dispatches into the owners' receive buffers, and (identity experts)
+    combines from them. Calls of the same kind share a name in the per-call table."""
+
+    def __init__(self, w, moe, native, torch, sets, device):
+        self.w = w
+        self.torch = torch
+        self.lib = native.lib()
+        R, H, k, E = w.R, w.H, w.k, w.E
+        if w.N % R:
+            raise ValueError("the EP workload needs N divisible by R")
+        n = w.N // R
+        self.n = n
+        p = moe.Problem(N=n, H=H, k=k, E_log=w.E_log, R=R, capacity=w.capacity, num_replicas=w.num_replicas,
+                        row_align=w.row_align)
+        self.problem = p
+        self.offsets_all = torch.zeros((R, E + 1), dtype=torch.int32, device=device)
+        self.layouts = []
+        for r in range(R):
+            G = moe.Layout.allocate(p, device)
+            G.tensors["expert_offsets"] = self.offsets_all[r]  # the layout writes its row of the table
+            self.layouts.append(G)
+        self.plans = [moe.EpPlan.allocate(p, device) for _ in range(R)]
+        RR = moe.moe_ep_recv_rows_max(p)
+        self.recv = [torch.empty((RR, H), dtype=torch.bfloat16, device=device) for _ in range(R)]
+        self.table = moe.peer_table(self.recv)
+        self.sets = sets
+        self.idx = torch.empty((w.N, k), dtype=torch.int32, device=device)
+        self.probs = torch.empty((w.N, k), dtype=torch.float32, device=device)
+        self.out = torch.empty((w.N, H), dtype=torch.bfloat16, device=device)
+        self._p = p.c_struct()
+        self._Ls = [G.c_struct() for G in self.layouts]
+        self.stream = torch.cuda.current_stream(device)
+        self._s = ctypes.c_void_p(self.stream.cuda_stream)
+        vp = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+        P = ctypes.byref(self._p)
+        lib = self.lib
+        self.calls = []
+        for st in sets:
+            rows = [slice(r * n, (r + 1) * n) for r in range(R)]
+            c = [("route", lib.moe_route_topk, (vp(st["logits"][rows[r]]), None, n, w.E_log, k,
+                                                vp(self.idx[rows[r]]), vp(self.probs[rows[r]]), self._s))
+                 for r in range(R)]
+            c += [("layout", lib.moe_dispatch_layout,
+                   (P, vp(self.idx[rows[r]]), vp(self.probs[rows[r]]), ctypes.byref(self._Ls[r]),
+                    vp(self.layouts[r].workspace), self.layouts[r].workspace.numel(), self._s)) for r in range(R)]
+            c += [("ep_plan", lib.moe_ep_plan,
+                   (P, vp(self.offsets_all), r, vp(self.plans[r].base), vp(self.plans[r].recv_expert_offsets),
+                    vp(self.plans[r].num_recv), vp(self.plans[r].status), self._s)) for r in range(R)]
+            c += [("ep_dispatch", lib.moe_ep_dispatch,
+                   (P, ctypes.byref(self._Ls[r]), vp(self.plans[r].base), vp(st["hidden"][rows[r]]),
+                    vp(self.table), self._s)) for r in range(R)]
+            c += [("ep_combine", lib.moe_ep_combine,
+                   (P, ctypes.byref(self._Ls[r]), vp(self.plans[r].base), vp(self.table),
+                    vp(self.probs[rows[r]]), vp(self.out[rows[r]]), self._s)) for r in range(R)]
+            self.calls.append(c)
+        self.kernel_names = [name for name, _, _ in self.calls[0]]
+
+    def run(self, i, events=None):
+        for n, (name, fn, args) in enumerate(self.calls[i % len(self.calls)]):
+            if events is not None:
+                events[n][0].record(self.stream)
+            rc = fn(*args)
+            if rc != 0:
+                raise RuntimeError(f"{name} returned {rc}")
+            if events is not None:
+                events[n][1].record(self.stream)
+
+    def status(self) -> int:
+        st = 0
+        for G in self.layouts:
+            st |= G.status()
+        for pl in self.plans:
+            st |= int(pl.status.item())
+        return st
+
+    def algorithmic_bytes(self) -> dict:
+        """Bytes per call (the mean over the R ranks), each row moved once."""
+        w, R, n = self.w, self.w.R, self.n
+        H, k, E = w.H, w.k, w.E
+        row, NK, RM = 2 * H, n * k, self.problem.rows_max
+        kept = [int(G["counters"][1].item()) for G in self.layouts]
+        read = [int((G["dest_row"] >= 0).any(dim=1).sum().item()) for G in self.layouts]
+        rows = [int(G["num_rows"].item()) for G in self.layouts]
+        mean = lambda v: sum(v) / len(v)  # noqa: E731
+        layout_bytes = NK * 8 + NK * (4 + 4 + 4 + 1) + RM * (4 * 4 + 1) + R * NK * 4
+        return {
+            "route": n * w.E_log * 4 + NK * 8,
+            "layout": layout_bytes,
+            "ep_plan": R * (E + 1) * 4 + E * 4 + (E // R + 2) * 4,
+            "ep_dispatch": round(mean([read[r] * row + rows[r] * row + NK * 8 + E * 12 for r in range(R)])),
+            "ep_combine": round(mean([kept[r] * row + n * row + NK * 12 + E * 8 for r in range(R)])),
+        }
+
+
 def run_ours(args, ws, rank, local):
     import torch
     import torch.distributed as tdist
@@ -353,7 +453,7 @@ def run_ours(args, ws, rank, local):
         shift = (s * 7919) % max(w.N, 1)
         sets.append({key: torch.roll(v, shifts=shift, dims=0).contiguous() for key, v in base.items()})
     del base
-    step = Step(w, moe, _native, torch, sets, device)
+    step = (EpStep if w.ep else Step)(w, moe, _native, torch, sets, device)
 
     def barrier():
         if ws > 1:
@@ -430,7 +530,7 @@ def run_ours(args, ws, rank, local):
         with torch.cuda.stream(comp_s):
             for b in range(2):
                 dset = {key: torch.empty_like(step.sets[0][key]) for key in pin}
-                pipes.append(Step(w, moe, _native, torch, [dset], device))
+                pipes.append((EpStep if w.ep else Step)(w, moe, _native, torch, [dset], device))
         views = [{key: (q.sets[0][key].view(torch.int16) if q.sets[0][key].dtype == torch.bfloat16
                         else q.sets[0][key]) for key in pin} for q in pipes]
         h2d = sum(t.numel() * t.element_size() for t in pin.values())
@@ -502,6 +602,7 @@ def run_ours(args, ws, rank, local):
         avg_ms = statistics.mean(per_kernel_ms[name])
         qs = statistics.quantiles(per_kernel_ms[name], n=10) if len(per_kernel_ms[name]) > 1 else [avg_ms] * 9
         kernels[name] = {
+            "calls_per_step": step.kernel_names.count(name),
             "us": round(avg_ms * 1e3, 2),
             "median_us": round(statistics.median(per_kernel_ms[name]) * 1e3, 2),
             "p10_us": round(qs[0] * 1e3, 2),
@@ -529,7 +630,8 @@ def run_ours(args, ws, rank, local):
         "config": {
             **w.describe(),
             "parallelism": f"dp{ws}: independent batch per GPU, no collective on the data path",
-            "step": "+".join(step.kernel_names),
+            "step": "+".join(dict.fromkeys(
+                f"{n}x{step.kernel_names.count(n)}" if step.kernel_names.count(n) > 1 else n for n in step.kernel_names)),
             "l2": f"inputs rotated over {nsets} buffer sets ({nsets * set_bytes / 2**20:.0f} MiB > 126 MB L2), no flush",
         },
         "effective_gbs": round(path_bytes / (ms_step * 1e-3) / 1e9, 1),

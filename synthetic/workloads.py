@@ -55,6 +55,7 @@ class Workload:
     row_align: int = 0
     tp_size: int = 0
     dedup: bool = False
+    ep: bool = False  # the N tokens are split evenly over the R ranks, which exchange rows
     seed: int = 0x5EED0000
     note: str = field(default="", compare=False)
 
@@ -87,6 +88,7 @@ class Workload:
             row_align=self.row_align,
             tp_size=self.tp_size,
             dedup=self.dedup,
+            ep=self.ep,
             seed=self.seed,
             note=self.note,
         )
@@ -114,6 +116,8 @@ class Workload:
             d["tp_size"] = self.tp_size
         if self.dedup:
             d["dedup"] = True
+        if self.ep:
+            d["ep_exchange"] = f"{self.R} ranks x {self.N // self.R} tokens, simulated on one GPU"
         return d
 
 
@@ -155,6 +159,9 @@ WORKLOADS = {
         # the same shape through the DeepEP-style path: each token sent once per rank,
         # receiver-side partials, sender-side sum over ranks
         Workload("ht_dedup", N=4096, H=7168, E_log=256, k=8, R=4, dedup=True, seed=0x5EED0002),
+        # the same 4096 tokens held by 4 ranks (1024 each) that exchange rows: every
+        # rank dispatches into the owners' receive buffers and combines from them
+        Workload("ht_ep4", N=4096, H=7168, E_log=256, k=8, R=4, ep=True, seed=0x5EED0002),
     ]
 }
 
