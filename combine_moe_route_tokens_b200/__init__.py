@@ -65,6 +65,7 @@ __all__ = [
     "moe_ep_plan",
     "moe_ep_dispatch",
     "moe_ep_combine",
+    "moe_ep_combine_backward",
     "moe_dedup_layout",
     "moe_dedup_dispatch",
     "moe_dedup_combine_local",
@@ -568,6 +569,31 @@ def moe_ep_combine(problem: Problem, layout: Layout, plan: EpPlan, peer_expert_o
         ctypes.byref(p), ctypes.byref(L), _ptr(plan.base), _ptr(table), _ptr(topk_probs), _ptr(out),
         _stream(stream)))
     return out
+
+
+def moe_ep_combine_backward(problem: Problem, layout: Layout, plan: EpPlan, grad_out: torch.Tensor,
+                            peer_expert_out, topk_probs: torch.Tensor, peer_grad_expert_out,
+                            grad_probs: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """grad_y rows written into the owners' gradient buffers; returns grad_probs [N, k] fp32.
+
+    The backward of moe_ep_dispatch is moe_ep_combine(..., topk_probs=None) over the
+    gradient buffers.
+    """
+    _need(grad_out, "grad_out", torch.bfloat16, (problem.N, problem.H), layout.device)
+    _need(topk_probs, "topk_probs", torch.float32, (problem.N, problem.k), layout.device)
+    ty = _table(peer_expert_out, layout.device)
+    tg = _table(peer_grad_expert_out, layout.device)
+    if ty.numel() != problem.R or tg.numel() != problem.R:
+        raise ValueError("one expert-output and one gradient buffer per rank")
+    if grad_probs is None:
+        grad_probs = torch.empty((problem.N, problem.k), dtype=torch.float32, device=layout.device)
+    _need(grad_probs, "grad_probs", torch.float32, (problem.N, problem.k), layout.device)
+    p = problem.c_struct()
+    L = layout.c_struct()
+    _native.check("moe_ep_combine_backward", _native.lib().moe_ep_combine_backward(
+        ctypes.byref(p), ctypes.byref(L), _ptr(plan.base), _ptr(grad_out), _ptr(ty), _ptr(topk_probs), _ptr(tg),
+        _ptr(grad_probs), _stream(stream)))
+    return grad_probs
 
 
 def moe_permute_backward(problem: Problem, layout: Layout, grad_send: torch.Tensor,

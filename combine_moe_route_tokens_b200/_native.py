@@ -131,6 +131,7 @@ _SIGNATURES = {
     "moe_ep_plan": (ctypes.c_int, [_PP, _VP, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP]),
     "moe_ep_dispatch": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP]),
     "moe_ep_combine": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP, _VP]),
+    "moe_ep_combine_backward": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "moe_dedup_rows_max": (ctypes.c_int64, [_PP]),
     "moe_dedup_workspace_bytes": (ctypes.c_int, [_PP, ctypes.POINTER(ctypes.c_size_t)]),
     "moe_dedup_layout": (ctypes.c_int, [_PP, _PL, _VP, _PD, _VP, ctypes.c_size_t, _VP]),

@@ -277,6 +277,16 @@ struct CombineBwdArgs {
     int32_t k;
     int32_t V;
     int32_t zero_blocks; // trailing CTAs that zero pad rows of grad_y
+    // expert-parallel exchange: y and grad_y rows live in the owners' buffers
+    // (receive order), row ep_base[q] + d - ep_offsets[q] of owner q / E_loc
+    const uint4 *const *ep_peer_y; // [R] device pointers
+    uint4 *const *ep_peer_gy;      // [R] device pointers
+    const int32_t *phys_idx;       // [N, k]
+    const int32_t *ep_base;        // [E]
+    const int32_t *ep_offsets;     // [E + 1]
+    const int32_t *ep_tokens;      // [E]
+    int64_t recv_max;
+    int32_t E, E_loc, R;
 };
 
 __device__ __forceinline__ float dot8(float s, const uint4 &g, const uint4 &y)
@@ -317,17 +327,24 @@ __device__ __forceinline__ float cta_sum_fixed(float v, float *s_red)
     return total;
 }
 
-template <int K>
+// EP: y and grad_y rows are in the owners' buffers of the exchange.
+template <int K, bool EP = false>
 __global__ void __launch_bounds__(COMBINE_BWD_THREADS) combine_backward_kernel(CombineBwdArgs a)
 {
     __shared__ float s_red[COMBINE_BWD_THREADS / 32];
     __shared__ float s_part[COMBINE_BWD_THREADS / 32][K > 0 ? K : 1];
+    __shared__ const uint4 *s_py[EP ? MOE_MAX_EP_RANKS : 1];
+    __shared__ uint4 *s_pg[EP ? MOE_MAX_EP_RANKS : 1];
     pdl_trigger();
     pdl_wait();
     if (blockIdx.x >= a.N) {
         const int64_t workers = static_cast<int64_t>(a.zero_blocks) * (COMBINE_BWD_THREADS / 32);
         const int64_t worker = (blockIdx.x - a.N) * (COMBINE_BWD_THREADS / 32) + (threadIdx.x >> 5);
-        zero_pad_rows_warp(a.grad_y, a.pad_mask, a.rows_max, a.V, worker, workers);
+        if constexpr (EP)
+            ep_zero_pads_warp(a.ep_peer_gy, a.ep_base, a.ep_offsets, a.ep_tokens, a.E, a.E_loc, a.V, a.recv_max,
+                              a.status, worker, workers);
+        else
+            zero_pad_rows_warp(a.grad_y, a.pad_mask, a.rows_max, a.V, worker, workers);
         return;
     }
     const int64_t t = blockIdx.x;
@@ -336,15 +353,50 @@ __global__ void __launch_bounds__(COMBINE_BWD_THREADS) combine_backward_kernel(C
     int32_t d;
     float p;
     load_slot_meta(a.dest_row, a.probs, t, k, a.rows_max, a.status, d, p);
+    // EP: lane j's slot row in its owner's buffers (row in d, owner in own), -1 if none
+    int32_t own = 0;
+    if constexpr (EP) {
+        if (threadIdx.x < a.R) {
+            s_py[threadIdx.x] = a.ep_peer_y[threadIdx.x];
+            s_pg[threadIdx.x] = a.ep_peer_gy[threadIdx.x];
+        }
+        if (d >= 0) {
+            const int32_t q = __ldg(a.phys_idx + t * k + lane);
+            const int64_t r = q >= 0 && q < a.E
+                                  ? static_cast<int64_t>(__ldg(a.ep_base + q)) + d - __ldg(a.ep_offsets + q)
+                                  : -1;
+            if (r < 0 || r >= a.recv_max) {
+                atomicOr(a.status, MOE_DEV_ROW_RANGE);
+                d = -1;
+            } else {
+                d = static_cast<int32_t>(r);
+                own = q / a.E_loc;
+            }
+        }
+        __syncthreads();
+    }
+    auto y_row = [&](int32_t row, int32_t owner) -> const uint4 * {
+        if constexpr (EP)
+            return s_py[owner] + static_cast<int64_t>(row) * a.V;
+        else
+            return a.y + static_cast<int64_t>(row) * a.V;
+    };
+    auto gy_row = [&](int32_t row, int32_t owner) -> uint4 * {
+        if constexpr (EP)
+            return s_pg[owner] + static_cast<int64_t>(row) * a.V;
+        else
+            return a.grad_y + static_cast<int64_t>(row) * a.V;
+    };
     const uint4 *g_row = a.grad_out + t * a.V;
 
     if constexpr (K > 0) {
-        int32_t dj[K];
+        int32_t dj[K], oj[K];
         float pj[K];
         float part[K];
 #pragma unroll
         for (int j = 0; j < K; ++j) {
             dj[j] = __shfl_sync(0xffffffffu, d, j);
+            oj[j] = EP ? __shfl_sync(0xffffffffu, own, j) : 0;
             pj[j] = __shfl_sync(0xffffffffu, p, j);
             part[j] = 0.0f;
         }
@@ -354,11 +406,11 @@ __global__ void __launch_bounds__(COMBINE_BWD_THREADS) combine_backward_kernel(C
 #pragma unroll
             for (int j = 0; j < K; ++j)
                 if (dj[j] >= 0)
-                    yj[j] = ld_stream_u4(a.y + static_cast<int64_t>(dj[j]) * a.V + v);
+                    yj[j] = ld_stream_u4(y_row(dj[j], oj[j]) + v);
 #pragma unroll
             for (int j = 0; j < K; ++j)
                 if (dj[j] >= 0) {
-                    st_u4(a.grad_y + static_cast<int64_t>(dj[j]) * a.V + v, scale8(pj[j], g));
+                    st_u4(gy_row(dj[j], oj[j]) + v, scale8(pj[j], g));
                     part[j] = dot8(part[j], g, yj[j]);
                 }
         }
@@ -374,7 +426,7 @@ __global__ void __launch_bounds__(COMBINE_BWD_THREADS) combine_backward_kernel(C
                 s_part[warp][j] = part[j];
         }
         __syncthreads();
-        if (threadIdx.x < K) { // lane j of warp 0 holds slot j's own dest_row in d
+        if (threadIdx.x < K) { // lane j of warp 0 holds slot j's own row in d
             const int j = threadIdx.x;
             float total = 0.0f;
             for (int w = 0; w < COMBINE_BWD_THREADS / 32; ++w)
@@ -384,13 +436,14 @@ __global__ void __launch_bounds__(COMBINE_BWD_THREADS) combine_backward_kernel(C
     } else {
         for (int j = 0; j < k; ++j) {
             const int32_t dj = __shfl_sync(0xffffffffu, d, j);
+            const int32_t oj = EP ? __shfl_sync(0xffffffffu, own, j) : 0;
             const float pj = __shfl_sync(0xffffffffu, p, j);
             float part = 0.0f;
             if (dj >= 0) {
                 for (int v = threadIdx.x; v < a.V; v += COMBINE_BWD_THREADS) {
                     const uint4 g = __ldg(g_row + v);
-                    const uint4 y = ld_stream_u4(a.y + static_cast<int64_t>(dj) * a.V + v);
-                    st_u4(a.grad_y + static_cast<int64_t>(dj) * a.V + v, scale8(pj, g));
+                    const uint4 y = ld_stream_u4(y_row(dj, oj) + v);
+                    st_u4(gy_row(dj, oj) + v, scale8(pj, g));
                     part = dot8(part, g, y);
                 }
             }

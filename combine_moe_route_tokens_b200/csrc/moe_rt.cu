@@ -925,6 +925,73 @@ int moe_ep_combine(const moe_problem_t *problem, const moe_layout_t *layout, con
     return launch_combine_args<SRC_EP>(a, problem->k, stream);
 }
 
+int moe_ep_combine_backward(const moe_problem_t *problem, const moe_layout_t *layout, const int32_t *base,
+                            const uint16_t *grad_out, const uint16_t *const *peer_expert_out, const float *topk_probs,
+                            uint16_t *const *peer_grad_expert_out, float *grad_probs, void *stream)
+{
+    Dims d;
+    int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    const int64_t recv_max = moe_ep_recv_rows_max(problem);
+    if (recv_max < 0)
+        return static_cast<int>(recv_max);
+    if ((rc = check_layout(layout, d, false)) != MOE_OK)
+        return rc;
+    if (layout->expert_offsets == nullptr || layout->tokens_per_expert == nullptr || base == nullptr ||
+        peer_expert_out == nullptr || peer_grad_expert_out == nullptr || (d.NK > 0 && layout->phys_idx == nullptr))
+        return MOE_ERR_INVALID;
+    if (problem->N == 0)
+        return MOE_OK;
+    if (grad_out == nullptr || !aligned16(grad_out) || topk_probs == nullptr || grad_probs == nullptr)
+        return MOE_ERR_INVALID;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev)) != MOE_OK)
+        return rc;
+    CombineBwdArgs a = {};
+    a.grad_out = reinterpret_cast<const uint4 *>(grad_out);
+    a.dest_row = layout->dest_row;
+    a.probs = topk_probs;
+    a.grad_probs = grad_probs;
+    a.status = layout->status;
+    a.N = problem->N;
+    a.rows_max = d.rows_max;
+    a.k = problem->k;
+    a.V = problem->H / 8;
+    a.ep_peer_y = reinterpret_cast<const uint4 *const *>(peer_expert_out);
+    a.ep_peer_gy = reinterpret_cast<uint4 *const *>(peer_grad_expert_out);
+    a.phys_idx = layout->phys_idx;
+    a.ep_base = base;
+    a.ep_offsets = layout->expert_offsets;
+    a.ep_tokens = layout->tokens_per_expert;
+    a.recv_max = recv_max;
+    a.E = d.E;
+    a.E_loc = d.E_loc;
+    a.R = problem->R;
+    // this rank's padding rows in the owners' gradient buffers: one warp per expert
+    const bool pads = problem->capacity > 0 || d.A > 1;
+    const int64_t zb = pads ? (d.E + COMBINE_BWD_THREADS / 32 - 1) / (COMBINE_BWD_THREADS / 32) : 0;
+    a.zero_blocks = static_cast<int32_t>(zb < 2 * dev.sms ? zb : 2 * dev.sms);
+    const int64_t blocks = problem->N + a.zero_blocks;
+    if (blocks > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    const dim3 grid(static_cast<unsigned>(blocks)), block(COMBINE_BWD_THREADS);
+    switch (problem->k) {
+    case 1:
+        return launch(combine_backward_kernel<1, true>, grid, block, 0, stream, false, a);
+    case 2:
+        return launch(combine_backward_kernel<2, true>, grid, block, 0, stream, false, a);
+    case 4:
+        return launch(combine_backward_kernel<4, true>, grid, block, 0, stream, false, a);
+    case 6:
+        return launch(combine_backward_kernel<6, true>, grid, block, 0, stream, false, a);
+    case 8:
+        return launch(combine_backward_kernel<8, true>, grid, block, 0, stream, false, a);
+    default:
+        return launch(combine_backward_kernel<0, true>, grid, block, 0, stream, false, a);
+    }
+}
+
 int moe_combine_backward(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *grad_out,
                          const uint16_t *expert_out, const float *topk_probs, uint16_t *grad_expert_out,
                          float *grad_probs, void *stream)
@@ -946,7 +1013,7 @@ int moe_combine_backward(const moe_problem_t *problem, const moe_layout_t *layou
     DeviceInfo dev;
     if ((rc = device_info(&dev)) != MOE_OK)
         return rc;
-    CombineBwdArgs a;
+    CombineBwdArgs a = {};
     a.grad_out = reinterpret_cast<const uint4 *>(grad_out);
     a.y = reinterpret_cast<const uint4 *>(expert_out);
     a.dest_row = layout->dest_row;

@@ -58,24 +58,29 @@ struct PermuteArgs {
 };
 
 // Expert-parallel exchange: zero this source's padding rows of every expert in
-// the owners' receive buffers; one warp per expert at a time.
-__device__ __forceinline__ void ep_zero_pad_rows_warp(const PermuteArgs &a, int64_t worker, int64_t nworkers)
+// the owners' buffers (receive buffers, or gradient buffers in the same order);
+// one warp per expert at a time. Row i of expert q (tokens[q] <= i < its rows)
+// sits at base[q] + i in the buffer of q's owner.
+__device__ __forceinline__ void ep_zero_pads_warp(uint4 *const *peers, const int32_t *base, const int32_t *offsets,
+                                                  const int32_t *tokens, int32_t E, int32_t E_loc, int32_t V,
+                                                  int64_t recv_max, uint32_t *status, int64_t worker,
+                                                  int64_t nworkers)
 {
     const int lane = threadIdx.x & 31;
     const uint4 z = make_uint4(0, 0, 0, 0);
-    for (int64_t q = worker; q < a.E; q += nworkers) {
-        const int32_t rows = __ldg(a.ep_offsets + q + 1) - __ldg(a.ep_offsets + q);
-        const int32_t first = __ldg(a.ep_tokens + q);
-        const int64_t b = __ldg(a.ep_base + q);
-        if (b < 0 || b + rows > a.recv_max) {
+    for (int64_t q = worker; q < E; q += nworkers) {
+        const int32_t rows = __ldg(offsets + q + 1) - __ldg(offsets + q);
+        const int32_t first = __ldg(tokens + q);
+        const int64_t b = __ldg(base + q);
+        if (b < 0 || b + rows > recv_max) {
             if (lane == 0 && rows > first)
-                atomicOr(a.status, MOE_DEV_ROW_RANGE);
+                atomicOr(status, MOE_DEV_ROW_RANGE);
             continue;
         }
-        uint4 *dst = a.ep_peers[q / a.E_loc];
+        uint4 *dst = peers[q / E_loc];
         for (int32_t i = first; i < rows; ++i)
-            for (int32_t c = lane; c < a.V; c += 32)
-                st_u4(dst + (b + i) * a.V + c, z);
+            for (int32_t c = lane; c < V; c += 32)
+                st_u4(dst + (b + i) * V + c, z);
     }
 }
 
@@ -112,7 +117,8 @@ __global__ void __launch_bounds__(PERMUTE_THREADS) permute_kernel(PermuteArgs a)
         const int64_t per = PERMUTE_THREADS / 32;
         const int64_t worker = static_cast<int64_t>(blockIdx.x) * per + (threadIdx.x >> 5);
         if constexpr (EP)
-            ep_zero_pad_rows_warp(a, worker, static_cast<int64_t>(a.zero_blocks) * per);
+            ep_zero_pads_warp(a.ep_peers, a.ep_base, a.ep_offsets, a.ep_tokens, a.E, a.E_loc, a.V, a.recv_max,
+                              a.status, worker, static_cast<int64_t>(a.zero_blocks) * per);
         else
             zero_pad_rows_warp(a.send, a.pad_mask, a.rows_max, a.V, worker, static_cast<int64_t>(a.zero_blocks) * per);
         return;

@@ -400,6 +400,23 @@ MOE_API int moe_ep_combine(const moe_problem_t *problem, const moe_layout_t *lay
                            void *stream);
 
 /*
+ * Backward of moe_ep_combine ([Megatron MORI]: combine backward with
+ * receiver-side probs): for every kept slot (t, j) of expert q, at row
+ * w = base[q] + dest_row[t,j] - expert_offsets[q] of owner r = q / E_loc:
+ *   peer_grad_expert_out[r][w] = bf16_rn( fp32(p[t,j] * grad_out[t]) ),
+ *   grad_probs[t,j] = fp32 dot( grad_out[t], peer_expert_out[r][w] ) (0 for a dropped slot),
+ * with the same arithmetic as moe_combine_backward; this rank's padding rows in the
+ * owners' gradient buffers are zeroed. The backward of moe_ep_dispatch is
+ * moe_ep_combine with unit weights (topk_probs NULL) over the gradient buffers.
+ *   peer_expert_out, peer_grad_expert_out: device arrays of R device pointers
+ *   grad_out [N, H] bf16; topk_probs [N, k] fp32; grad_probs [N, k] fp32 out
+ */
+MOE_API int moe_ep_combine_backward(const moe_problem_t *problem, const moe_layout_t *layout, const int32_t *base,
+                                    const uint16_t *grad_out, const uint16_t *const *peer_expert_out,
+                                    const float *topk_probs, uint16_t *const *peer_grad_expert_out,
+                                    float *grad_probs, void *stream);
+
+/*
  * Backward of permute ([Megatron MORI]: dispatch backward sums the row
  * gradients back per token with receiver-side indices): combine with unit
  * weights, grad_hidden[t] = bf16_rn( fp32 sum over ascending kept j of

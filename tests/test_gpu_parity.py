@@ -484,3 +484,33 @@ def test_ep_exchange(case):
         assert np.array_equal(host(plans[s].base), base[s])
         assert np.array_equal(host(outs[s]), oracle.combine(sends[s], L_or[s]["dest_row"], srcs[s][1]))
         assert layouts[s].status() == 0 and int(host(plans[s].status)[0]) == 0
+
+    # backward through the exchange: combine backward into the owners' gradient buffers,
+    # then the dispatch backward (the EP combine with unit weights over them)
+    rng = np.random.default_rng(R * 7 + N)
+    grads = [bf16_bits_from_f32(rng.standard_normal((N, H)).astype(np.float32)) for _ in range(R)]
+    gbufs = [torch.full((RR, H), canary, dtype=torch.bfloat16, device="cuda") for _ in range(R)]
+    gtable = moe.peer_table(gbufs)
+    gps = [moe.moe_ep_combine_backward(p, layouts[s], plans[s], dev(grads[s]), table, dev(srcs[s][1]), gtable)
+           for s in range(R)]
+    torch.cuda.synchronize()
+    ghs = [moe.moe_ep_combine(p, layouts[s], plans[s], gtable, None) for s in range(R)]
+    torch.cuda.synchronize()
+    exp_gy = []
+    for s in range(R):
+        gy, gp = oracle.combine_backward(grads[s], sends[s], L_or[s]["dest_row"], L_or[s]["row_token"],
+                                         L_or[s]["row_prob"])
+        exp_gy.append(gy)
+        # same arithmetic as the one-buffer backward: grad_probs bit for bit
+        _, gp_local = moe.moe_combine_backward(p, layouts[s], dev(grads[s]), dev(sends[s]), dev(srcs[s][1]))
+        torch.cuda.synchronize()
+        assert np.array_equal(host(gps[s]).view(np.uint32), host(gp_local).view(np.uint32))
+        assert np.allclose(host(gps[s]), gp, rtol=1e-4, atol=1e-4 * np.sqrt(H))
+        assert np.array_equal(host(ghs[s]), oracle.permute_backward(gy, L_or[s]["dest_row"]))
+    g_rv, _, _ = oracle.ep_exchange(L_or, exp_gy, R)
+    for r in range(R):
+        n = len(g_rv[r])
+        got = host(gbufs[r])
+        assert np.array_equal(got[:n], g_rv[r])
+        assert np.all(got[n:] == 0x7F7F)
+    assert all(G.status() == 0 for G in layouts)
