@@ -87,17 +87,44 @@ __device__ __forceinline__ uint32_t lanemask_lt()
     return m;
 }
 
-// Hot set and greedy placement for the reroute (warp 0; every block computes
-// the same result from the same totals). Hot experts: num_replicas rounds of
-// a warp arg-max over (count desc, id asc). Placement, per hot expert in that
-// order: the least-loaded rank (lowest id on ties) among the ranks other than
-// the master's that still have a free replica slot, else the master's own
-// rank; then floor(c/2) of load moves from the master's rank to it.
-__device__ void layout_placement(const LayoutArgs &a, const int32_t *s_cnt, int32_t *s_repl, int32_t *s_hot)
+// Hot set with the counts held in registers (E_log <= 32 * CPL): lane l holds
+// experts l, l + 32, ...; each round takes the warp's largest count (equal
+// counts: the lowest id, from a second reduction) and clears it.
+template <int CPL>
+__device__ __forceinline__ void layout_hot_set_regs(const LayoutArgs &a, const int32_t *s_cnt, int32_t *s_hot)
 {
     const int lane = threadIdx.x & 31;
-    if (threadIdx.x >= 32)
-        return;
+    uint32_t c[CPL];
+#pragma unroll
+    for (int u = 0; u < CPL; ++u) {
+        const int e = u * 32 + lane;
+        c[u] = e < a.E_log ? static_cast<uint32_t>(s_cnt[e]) + 1u : 0u; // +1: 0 marks "none"
+    }
+    for (int h = 0; h < a.num_replicas; ++h) {
+        uint32_t best = 0;
+        int bu = 0;
+#pragma unroll
+        for (int u = 0; u < CPL; ++u) {
+            const bool better = c[u] > best;
+            best = better ? c[u] : best;
+            bu = better ? u : bu;
+        }
+        const uint32_t wmax = __reduce_max_sync(0xffffffffu, best);
+        const uint32_t cand = (best == wmax && best != 0u) ? ~static_cast<uint32_t>(bu * 32 + lane) : 0u;
+        const int e = static_cast<int>(~__reduce_max_sync(0xffffffffu, cand));
+        const bool mine = (e & 31) == lane;
+#pragma unroll
+        for (int u = 0; u < CPL; ++u)
+            c[u] = (mine && u == (e >> 5)) ? 0u : c[u];
+        if (lane == 0)
+            s_hot[h] = e;
+    }
+}
+
+// Hot set for any E_log <= 2048: the counts are read from shared memory each round.
+__device__ __forceinline__ void layout_hot_set_smem(const LayoutArgs &a, const int32_t *s_cnt, int32_t *s_hot)
+{
+    const int lane = threadIdx.x & 31;
     uint64_t taken = 0; // bit u: expert lane + 32u already chosen (E_log <= 2048)
     for (int h = 0; h < a.num_replicas; ++h) {
         uint32_t best = 0;
@@ -117,6 +144,28 @@ __device__ void layout_placement(const LayoutArgs &a, const int32_t *s_cnt, int3
         if (lane == 0)
             s_hot[h] = e;
     }
+}
+
+// Hot experts and their replica placement, by warp 0 (readings of the UltraEP
+// page): the num_replicas largest logical counts, lowest id on ties; in that
+// order: the least-loaded rank (lowest id on ties) among the ranks other than
+// the master's that still have a free replica slot, else the master's own
+// rank; then floor(c/2) of load moves from the master's rank to it.
+__device__ void layout_placement(const LayoutArgs &a, const int32_t *s_cnt, int32_t *s_repl, int32_t *s_hot)
+{
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x >= 32)
+        return;
+    if (a.E_log <= 32)
+        layout_hot_set_regs<1>(a, s_cnt, s_hot);
+    else if (a.E_log <= 64)
+        layout_hot_set_regs<2>(a, s_cnt, s_hot);
+    else if (a.E_log <= 128)
+        layout_hot_set_regs<4>(a, s_cnt, s_hot);
+    else if (a.E_log <= 256)
+        layout_hot_set_regs<8>(a, s_cnt, s_hot);
+    else
+        layout_hot_set_smem(a, s_cnt, s_hot);
     __syncwarp();
     // lane owns ranks lane and lane + 32
     uint32_t load0 = 0, load1 = 0;
@@ -127,9 +176,27 @@ __device__ void layout_placement(const LayoutArgs &a, const int32_t *s_cnt, int3
     if (lane + 32 < a.R)
         for (int i = 0; i < a.M; ++i)
             load1 += static_cast<uint32_t>(s_cnt[(lane + 32) * a.M + i]);
+    // lane h < 32 holds hot expert h, its home rank and the load it moves, so each
+    // round's dependent chain starts at the reductions
+    int hot_e = 0, hot_home = 0;
+    uint32_t hot_moved = 0;
+    if (lane < a.num_replicas) {
+        hot_e = s_hot[lane];
+        hot_home = hot_e / a.M;
+        hot_moved = static_cast<uint32_t>(s_cnt[hot_e]) / 2u;
+    }
     for (int h = 0; h < a.num_replicas; ++h) {
-        const int e = s_hot[h];
-        const int home = e / a.M;
+        int e, home;
+        uint32_t moved;
+        if (h < 32) { // uniform over the warp
+            e = __shfl_sync(0xffffffffu, hot_e, h);
+            home = __shfl_sync(0xffffffffu, hot_home, h);
+            moved = __shfl_sync(0xffffffffu, hot_moved, h);
+        } else {
+            e = s_hot[h];
+            home = e / a.M;
+            moved = static_cast<uint32_t>(s_cnt[e]) / 2u;
+        }
         const uint32_t c0 = (lane < a.R && free0 > 0 && lane != home) ? load0 : 0xFFFFFFFFu;
         const uint32_t c1 = (lane + 32 < a.R && free1 > 0 && lane + 32 != home) ? load1 : 0xFFFFFFFFu;
         const uint32_t m = __reduce_min_sync(0xffffffffu, min(c0, c1));
@@ -143,7 +210,6 @@ __device__ void layout_placement(const LayoutArgs &a, const int32_t *s_cnt, int3
         }
         const int owner_free = __shfl_sync(0xffffffffu, best < 32 ? free0 : free1, best & 31);
         const int slot = a.S - owner_free;
-        const uint32_t moved = static_cast<uint32_t>(s_cnt[e]) / 2u;
         if (lane == (best & 31)) {
             if (best < 32) {
                 free0 -= 1;
@@ -499,6 +565,9 @@ __global__ void __launch_bounds__(LAYOUT_THREADS, 1) layout_kernel(LayoutArgs a)
 
     // ---- phase 2d: per-assignment outputs. `in_block` = rank of the assignment
     // among the earlier ones of its block with the same logical id.
+    // without capacity or alignment the kept rows are dense ([0, num_rows)): 2d writes
+    // their expert, and 2e needs no search
+    const bool rows_dense = a.C == 0 && a.A == 1;
     auto emit = [&](int64_t i, int32_t e, float p, int32_t in_block) {
         int32_t q = -1, ord = -1, dest = -1;
         uint8_t drop = 0;
@@ -530,6 +599,8 @@ __global__ void __launch_bounds__(LAYOUT_THREADS, 1) layout_kernel(LayoutArgs a)
             o.row_token[dest] = t;
             o.row_slot[dest] = static_cast<int32_t>(i) - t * a.k;
             o.row_prob[dest] = p;
+            if (rows_dense) // no padding inside the buffer: the row's expert is known here
+                o.row_local_expert[dest] = q - (q / a.E_loc) * a.E_loc;
         }
         if (o.local_topk != nullptr) {
             const int owner = dest >= 0 ? q / a.E_loc : -1;
@@ -560,11 +631,23 @@ __global__ void __launch_bounds__(LAYOUT_THREADS, 1) layout_kernel(LayoutArgs a)
     }
 
     // ---- phase 2e: per-row outputs that depend on the row index only, written
-    // in row order: the owning expert (capacity slot, or a binary search of the
-    // offsets), pad_mask, the rank-local expert id, and 0 / -1 / 0 in pad rows.
+    // in row order: pad_mask and 0 / -1 / 0 in pad rows; with padding inside the
+    // buffer also the owning expert (capacity slot, or a binary search of the
+    // offsets) and the rank-local expert id (dense rows got theirs in 2d).
     const int64_t stride = static_cast<int64_t>(a.G) * LAYOUT_THREADS;
     const int32_t num_rows = s_off[E];
     for (int64_t row = static_cast<int64_t>(b) * LAYOUT_THREADS + tid; row < a.rows_max; row += stride) {
+        if (rows_dense) {
+            const bool tail = row >= num_rows;
+            o.pad_mask[row] = tail ? 1 : 0;
+            if (tail) {
+                o.row_local_expert[row] = -1;
+                o.row_token[row] = -1;
+                o.row_slot[row] = -1;
+                o.row_prob[row] = 0.0f;
+            }
+            continue;
+        }
         int32_t q;
         bool pad;
         if (a.C > 0) {

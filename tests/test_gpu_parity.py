@@ -514,3 +514,52 @@ def test_ep_exchange(case):
         assert np.array_equal(got[:n], g_rv[r])
         assert np.all(got[n:] == 0x7F7F)
     assert all(G.status() == 0 for G in layouts)
+
+
+# ------------------------------------------------- randomized sweep
+
+
+def _sweep_cases(n=40, seed=20261202):
+    rng = np.random.default_rng(seed)
+    cases = []
+    while len(cases) < n:
+        R = int(rng.choice([1, 2, 3, 4, 8]))
+        E_log = R * int(rng.integers(1, 9))
+        k = int(rng.integers(1, min(E_log, 10) + 1))
+        reps = R * int(rng.integers(0, 2)) if E_log > R else 0
+        reps = min(reps, E_log)
+        N = int(rng.choice([1, 2, 31, 33, 257, 1000, 3001]))
+        H = 8 * int(rng.choice([1, 3, 16, 33, 130]))
+        C = int(rng.choice([0, 0, 1, 7, 40]))
+        A = int(rng.choice([0, 0, 2, 8])) if C == 0 else 0
+        if C and A:
+            continue
+        neg = float(rng.choice([0.0, 0.1]))
+        cases.append((N, H, k, E_log, R, C, reps, A, neg, int(rng.integers(1 << 30))))
+    return cases
+
+
+@pytest.mark.parametrize("case", _sweep_cases(), ids=lambda c: "N{}_H{}_k{}_E{}_R{}_C{}_rep{}_A{}".format(*c[:8]))
+def test_random_sweep_full_path(case):
+    """Random small problems (every option mixed) through layout, permute, combine and both backwards."""
+    N, H, k, E_log, R, C, reps, A, neg, seed = case
+    idx, probs, hidden = _small_case(N, H, k, E_log, R, C, reps, neg, seed=seed, zipf=1.3)
+    L = oracle.layout(idx, probs, E_log=E_log, R=R, C=C, num_replicas=reps, align=A)
+    p = moe.Problem(N=N, H=H, k=k, E_log=E_log, R=R, capacity=C, num_replicas=reps, row_align=A)
+    G = moe.moe_dispatch_layout(p, dev(idx), dev(probs))
+    send = moe.moe_permute(p, G, dev(hidden))
+    out = moe.moe_combine(p, G, send, dev(probs))
+    rng = np.random.default_rng(seed + 1)
+    g = bf16_bits_from_f32(rng.standard_normal((N, H)).astype(np.float32))
+    gy, gp = moe.moe_combine_backward(p, G, dev(g), send, dev(probs))
+    gh = moe.moe_permute_backward(p, G, gy)
+    torch.cuda.synchronize()
+    assert_layout_equal(G, L)
+    exp_send = oracle.permute(hidden, L["dest_row"], L["rows_max"])
+    assert np.array_equal(host(send), exp_send)
+    assert np.array_equal(host(out), oracle.combine(exp_send, L["dest_row"], probs))
+    exp_gy, exp_gp = oracle.combine_backward(g, exp_send, L["dest_row"], L["row_token"], L["row_prob"])
+    assert np.array_equal(host(gy), exp_gy)
+    assert np.allclose(host(gp), exp_gp, rtol=1e-4, atol=1e-4 * np.sqrt(H))
+    assert np.array_equal(host(gh), oracle.permute_backward(exp_gy, L["dest_row"]))
+    assert G.status() == 0
