@@ -8,7 +8,10 @@ router top-k -> dispatch layout -> permute -> (identity experts) -> combine,
 plus combine-backward and permute-backward for workloads that train
 (``ultraep``). Inputs are resident in HBM when the timed region starts and
 rotate over several buffer sets whose total size exceeds the 126 MB L2, so no
-step reads inputs that a previous step left in L2.
+step reads inputs that a previous step left in L2. Each set's step is captured once
+into a CUDA graph (the same C-ABI calls) and replayed in the timed region
+(``--eager``: the calls themselves); per-call times come from a second, eager pass
+with CUDA events around every call.
 
 N > 1 (torchrun, one process per GPU): each rank processes its own batch
 (data-parallel, independent seeds, no collective on the data path); timing is
@@ -453,7 +456,10 @@ def run_ours(args, ws, rank, local):
         shift = (s * 7919) % max(w.N, 1)
         sets.append({key: torch.roll(v, shifts=shift, dims=0).contiguous() for key, v in base.items()})
     del base
-    step = (EpStep if w.ep else Step)(w, moe, _native, torch, sets, device)
+    # a stream of our own (not the legacy default stream), so that steps can be captured
+    work_stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(work_stream):
+        step = (EpStep if w.ep else Step)(w, moe, _native, torch, sets, device)
 
     def barrier():
         if ws > 1:
@@ -464,6 +470,25 @@ def run_ours(args, ws, rank, local):
         step.run(i)
     torch.cuda.synchronize()
     abytes = step.algorithmic_bytes()
+
+    # one CUDA graph per buffer set, captured from the same C-ABI calls (the launches
+    # keep their programmatic-dependent-launch edges) and replayed in the timed
+    # region; --eager times the calls themselves
+    run_step = step.run
+    if not args.eager:
+        graphs = []
+        for i in range(len(step.calls)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=work_stream):
+                step.run(i)
+            graphs.append(g)
+        def run_step(i, events=None):
+            with torch.cuda.stream(work_stream):  # replay where the events are recorded
+                graphs[i % len(graphs)].replay()
+
+        for i in range(args.warmup):
+            run_step(i)
+        torch.cuda.synchronize()
 
     nk = len(step.kernel_names)
     t0 = torch.cuda.Event(enable_timing=True)
@@ -476,7 +501,7 @@ def run_ours(args, ws, rank, local):
     with sampler:
         t0.record(step.stream)
         for i in range(args.steps):
-            step.run(args.warmup + i)
+            run_step(args.warmup + i)
         t1.record(step.stream)
         torch.cuda.synchronize()
     barrier()
@@ -489,7 +514,7 @@ def run_ours(args, ws, rank, local):
     torch.cuda.synchronize()
     h0.record(step.stream)
     for i in range(args.steps):
-        step.run(0)
+        run_step(0)
     h1.record(step.stream)
     torch.cuda.synchronize()
     barrier()
@@ -648,7 +673,9 @@ def run_ours(args, ws, rank, local):
             "traffic": stored_traffic(dominant, w.name),
         },
         "gpu_launches": args.steps * len(step.kernel_names),
-        "kernel_timing": "per-kernel CUDA events in a second pass of the same K steps",
+        "kernel_timing": "per-kernel CUDA events in a second pass of the same K steps (launched eagerly)",
+        "launch": "eager C-ABI calls, programmatic dependent launch" if args.eager else
+                  "one CUDA graph per buffer set (captured C-ABI calls, programmatic dependent launch), replayed",
         "hot_l2": {
             "ms_per_step": round(hot_ms / args.steps, 4),
             "value": round(w.N * args.steps * ws / (hot_ms / 1e3), 1),
@@ -812,6 +839,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--tokens", type=int, default=0, help="run the workload with this many tokens (profiling)")
+    ap.add_argument("--eager", action="store_true",
+                    help="time eager C-ABI calls instead of replaying one captured CUDA graph per buffer set")
     ap.add_argument("--calibrate", action="store_true",
                     help="print the device's copy and fill bandwidth at the permute's size, then exit")
     ap.add_argument("--no-cpu-baseline", action="store_true")

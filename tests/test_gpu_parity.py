@@ -563,3 +563,38 @@ def test_random_sweep_full_path(case):
     assert np.allclose(host(gp), exp_gp, rtol=1e-4, atol=1e-4 * np.sqrt(H))
     assert np.array_equal(host(gh), oracle.permute_backward(exp_gy, L["dest_row"]))
     assert G.status() == 0
+
+
+def _sweep_next_cases(n=36, seed=20261203):
+    rng = np.random.default_rng(seed)
+    cases = []
+    while len(cases) < n:
+        mode = ("tp", "dedup", "ep")[len(cases) % 3]
+        R = int(rng.choice([1, 2, 3, 4, 8])) if mode != "ep" else int(rng.choice([2, 3, 4, 8]))
+        E_log = R * int(rng.integers(1, 9))
+        k = int(rng.integers(1, min(E_log, 10) + 1))
+        reps = R if (E_log > R and rng.random() < 0.4) else 0
+        N = int(rng.choice([1, 33, 257, 1000, 3001]))
+        H = 8 * int(rng.choice([1, 3, 16, 33]))
+        C = int(rng.choice([0, 0, 8, 40]))
+        A = int(rng.choice([0, 0, 2, 8]))
+        if C and A and C % A:
+            continue
+        T = int(rng.choice([2, 3, 4])) if mode == "tp" else 0
+        if mode == "tp" and C and A and (-(-C // T)) % A:
+            continue
+        cases.append((mode, N, H, k, E_log, R, C, reps, A, T))
+    return cases
+
+
+@pytest.mark.parametrize("case", _sweep_next_cases(),
+                         ids=lambda c: "{}_N{}_H{}_k{}_E{}_R{}_C{}_rep{}_A{}_T{}".format(*c))
+def test_random_sweep_next_rows(case):
+    """Random small problems through the TP-fold restore, the dedup view or the EP exchange."""
+    mode, N, H, k, E_log, R, C, reps, A, T = case
+    if mode == "tp":
+        test_tp_fold_layout_permute_restore((N, H, k, E_log, R, C, reps, A, T))
+    elif mode == "dedup":
+        test_dedup_path((N, H, k, E_log, R, C, reps, A, T))
+    else:
+        test_ep_exchange((R, N, H, k, E_log, C, reps, A))
