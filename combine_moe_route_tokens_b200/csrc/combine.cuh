@@ -42,6 +42,7 @@ struct CombineArgs {
     int32_t k;
     int32_t V;       // 16-byte chunks per row (H / 8)
     int32_t nchunks; // CTAs per token
+    int32_t last_first; // 1: tokens are taken last first (see combine_kernel)
     // restore after TP folding: T peer buffers and row maps (y / dest_row unused)
     int32_t T;
     const uint4 *ys[MOE_MAX_TP];
@@ -167,8 +168,12 @@ __global__ void __launch_bounds__(COMBINE_THREADS, 4) combine_kernel(CombineArgs
 {
     pdl_trigger();
     pdl_wait();
-    const int64_t t = blockIdx.x / a.nchunks;
-    const int c = static_cast<int>(blockIdx.x - t * a.nchunks);
+    // With last_first, tokens are taken last first: the rows a preceding token-ordered
+    // pass (the permute) wrote last are the ones still in L2 when this kernel starts.
+    // Each output row has one writer, so the order changes no result.
+    const int64_t tb = blockIdx.x / a.nchunks;
+    const int c = static_cast<int>(blockIdx.x - tb * a.nchunks);
+    const int64_t t = a.last_first ? a.N - 1 - tb : tb;
     const int v = c * blockDim.x + threadIdx.x;
     const int k = K > 0 ? K : a.k;
 

@@ -352,8 +352,10 @@ __global__ void __launch_bounds__(256, 4) dedup_combine_local_kernel(DedupCombin
                         (gridDim.x - a.token_blocks) * blockDim.x);
         return;
     }
-    const int64_t t = blockIdx.x / a.nchunks;
-    const int c = static_cast<int>(blockIdx.x - t * a.nchunks);
+    // tokens last first: the send rows the permute wrote last are still in L2
+    const int64_t tb = blockIdx.x / a.nchunks;
+    const int c = static_cast<int>(blockIdx.x - tb * a.nchunks);
+    const int64_t t = a.N - 1 - tb;
     const int v = c * blockDim.x + threadIdx.x;
     const int lane = threadIdx.x & 31;
     const int k = K > 0 ? K : a.k;

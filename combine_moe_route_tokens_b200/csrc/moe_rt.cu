@@ -489,6 +489,7 @@ int launch_combine(const moe_problem_t *problem, const moe_layout_t *layout, con
     a.k = problem->k;
     a.V = problem->H / 8;
     a.T = 1;
+    a.last_first = 1; // right after a permute, its last rows are still in L2
     return launch_combine_args<SRC_LOCAL>(a, problem->k, stream);
 }
 
@@ -538,6 +539,7 @@ int moe_restore_combined(const moe_problem_t *problem, const moe_layout_t *peer_
         a.ys[q] = reinterpret_cast<const uint4 *>(peer_expert_out[q]);
         a.dests[q] = peer_layouts[q].dest_row;
     }
+    a.last_first = 1;
     return launch_combine_args<SRC_TP_PEERS>(a, problem->k, stream);
 }
 
@@ -784,6 +786,7 @@ int moe_dedup_combine(const moe_problem_t *problem, const moe_dedup_t *dedup, co
     a.k = problem->R;
     a.V = problem->H / 8;
     a.T = 1;
+    a.last_first = 0; // the receiver pass wrote its partials last first: read them first first
     return launch_combine_args<SRC_LOCAL>(a, problem->R, stream);
 }
 
@@ -922,6 +925,7 @@ int moe_ep_combine(const moe_problem_t *problem, const moe_layout_t *layout, con
     a.recv_max = recv_max;
     a.E = d.E;
     a.E_loc = d.E_loc;
+    a.last_first = 1;
     return launch_combine_args<SRC_EP>(a, problem->k, stream);
 }
 
