@@ -598,3 +598,20 @@ def test_random_sweep_next_rows(case):
         test_dedup_path((N, H, k, E_log, R, C, reps, A, T))
     else:
         test_ep_exchange((R, N, H, k, E_log, C, reps, A))
+
+
+def test_grid_barrier_ticket_wraps():
+    """The layout's single-word grid barrier adds 2^20 per launch and wraps modulo 2^32
+    after 4096 launches on one workspace; 4200 launches in a row must all complete."""
+    N, k, E_log, R = 4096, 2, 16, 4  # 8192 assignments: 16 blocks meet at the barrier
+    idx, probs, _ = _small_case(N, 8, k, E_log, R, seed=99)
+    p = moe.Problem(N=N, H=8, k=k, E_log=E_log, R=R)
+    G = moe.Layout.allocate(p)
+    d_idx, d_probs = dev(idx), dev(probs)
+    for _ in range(4200):
+        moe.moe_dispatch_layout(p, d_idx, d_probs, layout=G)
+    torch.cuda.synchronize()
+    assert G.status() == 0
+    assert_layout_equal(G, oracle.layout(idx, probs, E_log=E_log, R=R))
+    word = int(G.workspace[:4].view(torch.int32).item()) & 0xFFFFFFFF
+    assert word == (4200 << 20) & 0xFFFFFFFF  # every launch added exactly 2^20
