@@ -324,11 +324,15 @@ class Step:
 class EpStep:
     """One step of the expert-parallel exchange between R ranks simulated on this GPU.
 
-    The workload's N tokens are split evenly over the R ranks. Every rank routes
-    and lays out its own tokens; the layouts write their expert_offsets straight
-    into the rows of one [R, E+1] table (on several GPUs: an all-gather); every
-    rank plans, dispatches into the owners' receive buffers, and (identity experts)
-    combines from them. Calls of the same kind share a name in the per-call table."""
+    The workload's N tokens are split evenly over the R ranks, and each rank's calls
+    run on a stream of its own, as the ranks would on GPUs of their own. Every rank
+    routes and lays out its own tokens (its layout writes its expert_offsets straight
+    into row r of one [R, E+1] table: the stand-in for the all-gather); after all
+    layouts every rank plans and dispatches into the owners' receive buffers; after
+    all dispatches every rank combines from them (identity experts). The step then
+    joins the ranks' streams. Calls of the same kind share a name in the per-call table."""
+
+    PHASES = ("route", "layout", "ep_plan", "ep_dispatch", "ep_combine")
 
     def __init__(self, w, moe, native, torch, sets, device):
         self.w = w
@@ -359,40 +363,64 @@ class EpStep:
         self._p = p.c_struct()
         self._Ls = [G.c_struct() for G in self.layouts]
         self.stream = torch.cuda.current_stream(device)
-        self._s = ctypes.c_void_p(self.stream.cuda_stream)
+        self.rank_streams = [torch.cuda.Stream(device) for _ in range(R)]
+        self._rs = [ctypes.c_void_p(st.cuda_stream) for st in self.rank_streams]
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        self._start = ev()
+        self._phase_done = [[ev() for _ in range(R)] for _ in self.PHASES]
         vp = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
         P = ctypes.byref(self._p)
         lib = self.lib
-        self.calls = []
+        self.calls = []  # per set: {phase: [(name, fn, args) for each rank]}
         for st in sets:
             rows = [slice(r * n, (r + 1) * n) for r in range(R)]
-            c = [("route", lib.moe_route_topk, (vp(st["logits"][rows[r]]), None, n, w.E_log, k,
-                                                vp(self.idx[rows[r]]), vp(self.probs[rows[r]]), self._s))
-                 for r in range(R)]
-            c += [("layout", lib.moe_dispatch_layout,
-                   (P, vp(self.idx[rows[r]]), vp(self.probs[rows[r]]), ctypes.byref(self._Ls[r]),
-                    vp(self.layouts[r].workspace), self.layouts[r].workspace.numel(), self._s)) for r in range(R)]
-            c += [("ep_plan", lib.moe_ep_plan,
-                   (P, vp(self.offsets_all), r, vp(self.plans[r].base), vp(self.plans[r].recv_expert_offsets),
-                    vp(self.plans[r].num_recv), vp(self.plans[r].status), self._s)) for r in range(R)]
-            c += [("ep_dispatch", lib.moe_ep_dispatch,
-                   (P, ctypes.byref(self._Ls[r]), vp(self.plans[r].base), vp(st["hidden"][rows[r]]),
-                    vp(self.table), self._s)) for r in range(R)]
-            c += [("ep_combine", lib.moe_ep_combine,
-                   (P, ctypes.byref(self._Ls[r]), vp(self.plans[r].base), vp(self.table),
-                    vp(self.probs[rows[r]]), vp(self.out[rows[r]]), self._s)) for r in range(R)]
-            self.calls.append(c)
-        self.kernel_names = [name for name, _, _ in self.calls[0]]
+            ph = {
+                "route": [("route", lib.moe_route_topk,
+                           (vp(st["logits"][rows[r]]), None, n, w.E_log, k, vp(self.idx[rows[r]]),
+                            vp(self.probs[rows[r]]), self._rs[r])) for r in range(R)],
+                "layout": [("layout", lib.moe_dispatch_layout,
+                            (P, vp(self.idx[rows[r]]), vp(self.probs[rows[r]]), ctypes.byref(self._Ls[r]),
+                             vp(self.layouts[r].workspace), self.layouts[r].workspace.numel(), self._rs[r]))
+                           for r in range(R)],
+                "ep_plan": [("ep_plan", lib.moe_ep_plan,
+                             (P, vp(self.offsets_all), r, vp(self.plans[r].base),
+                              vp(self.plans[r].recv_expert_offsets), vp(self.plans[r].num_recv),
+                              vp(self.plans[r].status), self._rs[r])) for r in range(R)],
+                "ep_dispatch": [("ep_dispatch", lib.moe_ep_dispatch,
+                                 (P, ctypes.byref(self._Ls[r]), vp(self.plans[r].base), vp(st["hidden"][rows[r]]),
+                                  vp(self.table), self._rs[r])) for r in range(R)],
+                "ep_combine": [("ep_combine", lib.moe_ep_combine,
+                                (P, ctypes.byref(self._Ls[r]), vp(self.plans[r].base), vp(self.table),
+                                 vp(self.probs[rows[r]]), vp(self.out[rows[r]]), self._rs[r])) for r in range(R)],
+            }
+            self.calls.append(ph)
+        self.kernel_names = [name for phase in self.PHASES for name, _, _ in self.calls[0][phase]]
 
     def run(self, i, events=None):
-        for n, (name, fn, args) in enumerate(self.calls[i % len(self.calls)]):
-            if events is not None:
-                events[n][0].record(self.stream)
-            rc = fn(*args)
-            if rc != 0:
-                raise RuntimeError(f"{name} returned {rc}")
-            if events is not None:
-                events[n][1].record(self.stream)
+        """Fork to the ranks' streams; join where a phase needs every rank's previous one."""
+        R = self.w.R
+        ph = self.calls[i % len(self.calls)]
+        self._start.record(self.stream)
+        for st in self.rank_streams:
+            st.wait_event(self._start)
+        n = 0
+        for p_i, phase in enumerate(self.PHASES):
+            if phase in ("ep_plan", "ep_combine"):  # needs every rank's layout / dispatch
+                for st in self.rank_streams:
+                    for e in self._phase_done[p_i - 1]:
+                        st.wait_event(e)
+            for r, (name, fn, args) in enumerate(ph[phase]):
+                if events is not None:
+                    events[n][0].record(self.rank_streams[r])
+                rc = fn(*args)
+                if rc != 0:
+                    raise RuntimeError(f"{name} returned {rc}")
+                if events is not None:
+                    events[n][1].record(self.rank_streams[r])
+                self._phase_done[p_i][r].record(self.rank_streams[r])
+                n += 1
+        for r in range(R):
+            self.stream.wait_event(self._phase_done[-1][r])
 
     def status(self) -> int:
         st = 0

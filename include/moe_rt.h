@@ -192,6 +192,9 @@ MOE_API int moe_route_topk(const float *logits, const uint8_t *token_mask, int64
  *   layout      every pointer except local_topk must be non-NULL
  *   workspace   moe_layout_workspace_bytes() bytes, zero-filled before first use
  * Limits: E_log <= 2048, k <= 32, R <= 64 when num_replicas > 0.
+ * The launch is cooperative (one CTA per SM, up to 128 CTAs): layouts enqueued on
+ * several streams at once must together fit the GPU's SMs, else their bounded
+ * barrier reports MOE_DEV_TIMEOUT.
  */
 MOE_API int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, const float *topk_probs,
                         const moe_layout_t *layout, void *workspace, size_t workspace_bytes, void *stream);
