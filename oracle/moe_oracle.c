@@ -520,9 +520,9 @@ void oracle_permute(const oracle_problem *p, int32_t H, const int32_t *dest_row,
  * into [num_tokens, H] one top-k slot at a time, in ascending slot order, so
  * the accumulation order per token is fixed. [Megatron MoE] combine.
  *
- * Precision (the spec of this build; the page itself accumulates in the
- * activation dtype): fp32 accumulator starting at +0, one fused multiply-add
- * per kept slot in ascending j, one rounding to bf16 at the end.
+ * Precision (a reading; the page itself accumulates in the activation dtype):
+ * fp32 accumulator starting at +0, one fused multiply-add per kept slot in
+ * ascending j, one rounding to bf16 at the end.
  *   out[t,h] = bf16( fma(p[t,k-1], y[.,h], ... fma(p[t,0], y[.,h], +0) ... ) )
  * A NULL prob array means unit weights.
  */
