@@ -11,7 +11,10 @@
 #include <cstdint>
 #include <cstdio>
 #include <atomic>
+#include <cstdlib>
 #include <mutex>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "moe_rt.h"
 
@@ -50,6 +53,34 @@ LayoutKernel layout_kernel_for(int ipl)
 }
 
 constexpr int LAYOUT_IPLS[] = {0, 1, 2, 4, 8};
+
+// NVTX ranges around the enqueuing entry points, for profilers' timelines: on
+// when the environment variable MOE_RT_NVTX is set to a non-empty value other
+// than "0" (read once); off, a range costs one cached flag test.
+bool nvtx_on()
+{
+    static const bool on = [] {
+        const char *v = std::getenv("MOE_RT_NVTX");
+        return v != nullptr && v[0] != '\0' && !(v[0] == '0' && v[1] == '\0');
+    }();
+    return on;
+}
+
+struct NvtxRange {
+    const bool on;
+    explicit NvtxRange(const char *name) : on(nvtx_on())
+    {
+        if (on)
+            nvtxRangePushA(name);
+    }
+    ~NvtxRange()
+    {
+        if (on)
+            nvtxRangePop();
+    }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 // Programmatic dependent launch is used unless the driver refuses it for a
 // kind of launch; then that kind falls back to ordinary stream order.
@@ -300,6 +331,7 @@ int moe_layout_workspace_bytes(const moe_problem_t *problem, size_t *bytes)
 int moe_route_topk(const float *logits, const uint8_t *token_mask, int64_t N, int32_t E, int32_t k,
                    int32_t *topk_idx, float *topk_probs, void *stream)
 {
+    NvtxRange nvtx_range("moe_route_topk");
     if (N < 0 || E < 1 || k < 1 || k > E)
         return MOE_ERR_INVALID;
     if (k > 32 || E > 1024)
@@ -334,6 +366,7 @@ int moe_route_topk(const float *logits, const uint8_t *token_mask, int64_t N, in
 int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, const float *topk_probs,
                         const moe_layout_t *layout, void *workspace, size_t workspace_bytes, void *stream)
 {
+    NvtxRange nvtx_range("moe_dispatch_layout");
     Dims d;
     int rc = check_problem(problem, &d);
     if (rc != MOE_OK)
@@ -396,6 +429,7 @@ int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, c
 int moe_permute(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *hidden, uint16_t *send,
                 void *stream)
 {
+    NvtxRange nvtx_range("moe_permute");
     Dims d;
     int rc = check_problem(problem, &d);
     if (rc != MOE_OK)
@@ -498,18 +532,21 @@ int launch_combine(const moe_problem_t *problem, const moe_layout_t *layout, con
 int moe_combine(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *expert_out,
                 const float *topk_probs, uint16_t *out, void *stream)
 {
+    NvtxRange nvtx_range("moe_combine");
     return launch_combine(problem, layout, expert_out, topk_probs, out, stream);
 }
 
 int moe_permute_backward(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *grad_send,
                          uint16_t *grad_hidden, void *stream)
 {
+    NvtxRange nvtx_range("moe_permute_backward");
     return launch_combine(problem, layout, grad_send, nullptr, grad_hidden, stream);
 }
 
 int moe_restore_combined(const moe_problem_t *problem, const moe_layout_t *peer_layouts,
                          const uint16_t *const *peer_expert_out, const float *topk_probs, uint16_t *out, void *stream)
 {
+    NvtxRange nvtx_range("moe_restore_combined");
     Dims d;
     int rc = check_problem(problem, &d);
     if (rc != MOE_OK)
@@ -567,6 +604,7 @@ int moe_dedup_workspace_bytes(const moe_problem_t *problem, size_t *bytes)
 int moe_dedup_layout(const moe_problem_t *problem, const moe_layout_t *layout, const float *topk_probs,
                      const moe_dedup_t *dedup, void *workspace, size_t workspace_bytes, void *stream)
 {
+    NvtxRange nvtx_range("moe_dedup_layout");
     Dims d;
     int rc = check_problem(problem, &d);
     if (rc != MOE_OK)
@@ -654,6 +692,7 @@ int moe_dedup_layout(const moe_problem_t *problem, const moe_layout_t *layout, c
 int moe_dedup_dispatch(const moe_problem_t *problem, const moe_dedup_t *dedup, const uint16_t *hidden,
                        uint16_t *recv_x, void *stream)
 {
+    NvtxRange nvtx_range("moe_dedup_dispatch");
     Dims d;
     int rc = check_problem(problem, &d);
     if (rc != MOE_OK)
@@ -696,6 +735,7 @@ int moe_dedup_dispatch(const moe_problem_t *problem, const moe_dedup_t *dedup, c
 int moe_dedup_combine_local(const moe_problem_t *problem, const moe_layout_t *layout, const moe_dedup_t *dedup,
                             const uint16_t *expert_out, const float *topk_probs, uint16_t *partial, void *stream)
 {
+    NvtxRange nvtx_range("moe_dedup_combine_local");
     Dims d;
     int rc = check_problem(problem, &d);
     if (rc != MOE_OK)
@@ -762,6 +802,7 @@ int moe_dedup_combine_local(const moe_problem_t *problem, const moe_layout_t *la
 int moe_dedup_combine(const moe_problem_t *problem, const moe_dedup_t *dedup, const uint16_t *partial,
                       uint16_t *out, void *stream)
 {
+    NvtxRange nvtx_range("moe_dedup_combine");
     Dims d;
     int rc = check_problem(problem, &d);
     if (rc != MOE_OK)
@@ -809,6 +850,7 @@ int64_t moe_ep_recv_rows_max(const moe_problem_t *problem)
 int moe_ep_plan(const moe_problem_t *problem, const int32_t *offsets_all, int32_t src_rank, int32_t *base,
                 int32_t *recv_expert_offsets, int32_t *num_recv, uint32_t *status, void *stream)
 {
+    NvtxRange nvtx_range("moe_ep_plan");
     Dims d;
     int rc = check_problem(problem, &d);
     if (rc != MOE_OK)
@@ -841,6 +883,7 @@ int moe_ep_plan(const moe_problem_t *problem, const int32_t *offsets_all, int32_
 int moe_ep_dispatch(const moe_problem_t *problem, const moe_layout_t *layout, const int32_t *base,
                     const uint16_t *hidden, uint16_t *const *peer_recv, void *stream)
 {
+    NvtxRange nvtx_range("moe_ep_dispatch");
     Dims d;
     int rc = check_problem(problem, &d);
     if (rc != MOE_OK)
@@ -892,6 +935,7 @@ int moe_ep_dispatch(const moe_problem_t *problem, const moe_layout_t *layout, co
 int moe_ep_combine(const moe_problem_t *problem, const moe_layout_t *layout, const int32_t *base,
                    const uint16_t *const *peer_expert_out, const float *topk_probs, uint16_t *out, void *stream)
 {
+    NvtxRange nvtx_range("moe_ep_combine");
     Dims d;
     int rc = check_problem(problem, &d);
     if (rc != MOE_OK)
@@ -933,6 +977,7 @@ int moe_ep_combine_backward(const moe_problem_t *problem, const moe_layout_t *la
                             const uint16_t *grad_out, const uint16_t *const *peer_expert_out, const float *topk_probs,
                             uint16_t *const *peer_grad_expert_out, float *grad_probs, void *stream)
 {
+    NvtxRange nvtx_range("moe_ep_combine_backward");
     Dims d;
     int rc = check_problem(problem, &d);
     if (rc != MOE_OK)
@@ -1000,6 +1045,7 @@ int moe_combine_backward(const moe_problem_t *problem, const moe_layout_t *layou
                          const uint16_t *expert_out, const float *topk_probs, uint16_t *grad_expert_out,
                          float *grad_probs, void *stream)
 {
+    NvtxRange nvtx_range("moe_combine_backward");
     Dims d;
     int rc = check_problem(problem, &d);
     if (rc != MOE_OK)
@@ -1103,6 +1149,7 @@ int scratch_address(void **out)
 extern "C" int moe_dispatch_layout_noalloc(const moe_problem_t *problem, const int32_t *topk_idx,
                                            const float *topk_probs, const moe_layout_t *layout, void *stream)
 {
+    NvtxRange nvtx_range("moe_dispatch_layout_noalloc");
     Dims d;
     int rc = check_problem(problem, &d);
     if (rc != MOE_OK)

@@ -615,3 +615,17 @@ def test_grid_barrier_ticket_wraps():
     assert_layout_equal(G, oracle.layout(idx, probs, E_log=E_log, R=R))
     word = int(G.workspace[:4].view(torch.int32).item()) & 0xFFFFFFFF
     assert word == (4200 << 20) & 0xFFFFFFFF  # every launch added exactly 2^20
+
+
+def test_nvtx_ranges_on():
+    """With MOE_RT_NVTX=1 every entry point opens and closes an NVTX range; the path is unchanged."""
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, MOE_RT_NVTX="1")
+    r = subprocess.run([sys.executable, "-c", "import __graft_entry__ as g; g.smoke()"], cwd=root, env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
+    assert "smoke: ok" in r.stdout
