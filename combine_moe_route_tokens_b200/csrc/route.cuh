@@ -77,25 +77,86 @@ __device__ __forceinline__ void route_select(const float (&v)[VPL], int E, int k
 
     int my_id = -1;
     uint32_t my_key = 0;
-    for (int j = 0; j < k; ++j) {
-        uint32_t best = 0;
-        int bi = 0;
+    bool done = false;
+    if constexpr (VPL >= 4) {
+        // Candidates first. Every lane holds a key (E > 64), so the k-th largest of
+        // the 32 lane maxima, t0, is reached by k distinct keys, and the k-th largest
+        // key overall is >= t0: every key the k rounds below can pick, ties included,
+        // is >= t0, and any key < t0 is below all of them. When no lane holds more
+        // than two keys >= t0 (the usual case), the rounds run over those two
+        // registers per lane; otherwise over all of them. Same picks either way.
+        if (k <= 16) {
+            uint32_t lm = key[0];
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-            const bool better = key[i] > best;
-            best = better ? key[i] : best;
-            bi = better ? i : bi;
+            for (int i = 1; i < VPL; ++i)
+                lm = max(lm, key[i]);
+            uint32_t t0 = 0;
+            for (int j = 0; j < k; ++j) { // remove one lane maximum per round, largest first
+                const uint32_t w = __reduce_max_sync(0xffffffffu, lm);
+                const uint32_t holders = __ballot_sync(0xffffffffu, lm == w);
+                if (lane == __ffs(holders) - 1)
+                    lm = 0;
+                t0 = w;
+            }
+            int c = 0;
+#pragma unroll
+            for (int i = 0; i < VPL; ++i)
+                c += key[i] >= t0 ? 1 : 0;
+            if (t0 != 0u && __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(c)) <= 2u) {
+                uint32_t k0 = 0, k1 = 0; // this lane's candidates in ascending index
+                int i0 = 0, i1 = 0;
+#pragma unroll
+                for (int i = VPL - 1; i >= 0; --i) {
+                    const bool in = key[i] >= t0;
+                    k1 = in ? k0 : k1;
+                    i1 = in ? i0 : i1;
+                    k0 = in ? key[i] : k0;
+                    i0 = in ? i : i0;
+                }
+                for (int j = 0; j < k; ++j) {
+                    const bool second = k1 > k0; // equal keys: the lower index (slot 0)
+                    const uint32_t best = second ? k1 : k0;
+                    const int bi = second ? i1 : i0;
+                    const uint32_t wmax = __reduce_max_sync(0xffffffffu, best);
+                    const uint32_t cand =
+                        (best == wmax && best != 0u) ? ~static_cast<uint32_t>(bi * 32 + lane) : 0u;
+                    const int e = static_cast<int>(~__reduce_max_sync(0xffffffffu, cand));
+                    if ((e & 31) == lane) {
+                        if (second)
+                            k1 = 0;
+                        else
+                            k0 = 0;
+                    }
+                    if (lane == j) {
+                        my_id = e;
+                        my_key = wmax;
+                    }
+                }
+                done = true;
+            }
         }
-        const uint32_t wmax = __reduce_max_sync(0xffffffffu, best);
-        const uint32_t cand = (best == wmax && best != 0u) ? ~static_cast<uint32_t>(bi * 32 + lane) : 0u;
-        const int e = static_cast<int>(~__reduce_max_sync(0xffffffffu, cand));
-        const bool mine = (e & 31) == lane;
+    }
+    if (!done) {
+        for (int j = 0; j < k; ++j) {
+            uint32_t best = 0;
+            int bi = 0;
 #pragma unroll
-        for (int i = 0; i < VPL; ++i)
-            key[i] = (mine && i == (e >> 5)) ? 0u : key[i];
-        if (lane == j) {
-            my_id = e;
-            my_key = wmax;
+            for (int i = 0; i < VPL; ++i) {
+                const bool better = key[i] > best;
+                best = better ? key[i] : best;
+                bi = better ? i : bi;
+            }
+            const uint32_t wmax = __reduce_max_sync(0xffffffffu, best);
+            const uint32_t cand = (best == wmax && best != 0u) ? ~static_cast<uint32_t>(bi * 32 + lane) : 0u;
+            const int e = static_cast<int>(~__reduce_max_sync(0xffffffffu, cand));
+            const bool mine = (e & 31) == lane;
+#pragma unroll
+            for (int i = 0; i < VPL; ++i)
+                key[i] = (mine && i == (e >> 5)) ? 0u : key[i];
+            if (lane == j) {
+                my_id = e;
+                my_key = wmax;
+            }
         }
     }
     id = lane < k ? my_id : -1;

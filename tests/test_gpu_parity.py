@@ -629,3 +629,27 @@ def test_nvtx_ranges_on():
                        capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
     assert "smoke: ok" in r.stdout
+
+
+@pytest.mark.parametrize("kind", ["ties_spread", "ties_dense", "one_lane_heavy"])
+def test_route_candidate_paths(kind):
+    """The router's candidate fast path (at most two keys per lane at or above the k-th
+    lane maximum) and its fallback must pick the same ids, ties at the threshold included."""
+    rng = np.random.default_rng(11)
+    N, E, k = 300, 256, 8
+    logits = (rng.standard_normal((N, E)) - 3.0).astype(np.float32)
+    if kind == "ties_spread":  # ten equal maxima on ten different lanes: fast path, ties at t0
+        hot = [1, 34, 67, 100, 133, 166, 199, 232, 9, 42]
+        logits[:, hot] = 5.0
+    elif kind == "ties_dense":  # equal maxima three per lane: the fallback
+        hot = [3, 35, 67, 99, 4, 36, 68, 100, 5]
+        logits[:, hot] = 5.0
+    else:  # one lane holds all the large keys
+        hot = [7, 39, 71, 103, 135, 167, 199, 231]
+        logits[:, hot] = 4.0 + rng.random((N, len(hot))).astype(np.float32)
+    gi, gp = moe.moe_route_topk(dev(logits), k)
+    idx, probs = oracle.route_topk(logits, k)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(gi), idx)
+    tol = route_prob_tolerance(logits, idx) * probs.astype(np.float64)
+    assert np.all(np.abs(host(gp).astype(np.float64) - probs.astype(np.float64)) <= tol)
