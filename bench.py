@@ -462,7 +462,10 @@ def run_ours(args, ws, rank, local):
                                  device_id=torch.device("cuda", local))
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    build()
+    if local == 0:  # one build per node; the other ranks wait for it
+        build()
+    if ws > 1:
+        tdist.barrier()
     moe.load_library()
 
     w = get_workload(args.workload)

@@ -60,13 +60,17 @@ def build(force: bool = False, verbose: bool = False) -> str:
     """Compile csrc/moe_rt.cu into combine_moe_route_tokens_b200/libmoert.so (if stale)."""
     if not force and not is_stale():
         return LIB_PATH
-    tmp = LIB_PATH + ".tmp"
+    tmp = f"{LIB_PATH}.tmp.{os.getpid()}"  # several processes may build at once: each renames a whole file
     cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, os.path.join(CSRC, "moe_rt.cu")]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), file=sys.stderr)
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB_PATH)
+    try:
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, LIB_PATH)
+    finally:
+        if os.path.exists(tmp):
+            os.remove(tmp)
     return LIB_PATH
 
 
