@@ -682,6 +682,7 @@ def run_ours(args, ws, rank, local):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
+        "accumulate": "fp32 (combine and backward)",
         "data": "synthetic",
         "config": {
             **w.describe(),
