@@ -506,13 +506,22 @@ def run_ours(args, ws, rank, local):
     # keep their programmatic-dependent-launch edges) and replayed in the timed
     # region; --eager times the calls themselves
     run_step = step.run
+    launch_mode = "eager C-ABI calls, programmatic dependent launch"
     if not args.eager:
         graphs = []
-        for i in range(len(step.calls)):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=work_stream):
-                step.run(i)
-            graphs.append(g)
+        try:
+            for i in range(len(step.calls)):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=work_stream):
+                    step.run(i)
+                graphs.append(g)
+        except Exception as exc:  # a driver without capture support: time the calls themselves
+            graphs = []
+            torch.cuda.synchronize()
+            launch_mode += f" (graph capture failed: {type(exc).__name__})"
+    if not args.eager and graphs:
+        launch_mode = "one CUDA graph per buffer set (captured C-ABI calls, programmatic dependent launch), replayed"
+
         def run_step(i, events=None):
             with torch.cuda.stream(work_stream):  # replay where the events are recorded
                 graphs[i % len(graphs)].replay()
@@ -706,8 +715,7 @@ def run_ours(args, ws, rank, local):
         },
         "gpu_launches": args.steps * len(step.kernel_names),
         "kernel_timing": "per-kernel CUDA events in a second pass of the same K steps (launched eagerly)",
-        "launch": "eager C-ABI calls, programmatic dependent launch" if args.eager else
-                  "one CUDA graph per buffer set (captured C-ABI calls, programmatic dependent launch), replayed",
+        "launch": launch_mode,
         "hot_l2": {
             "ms_per_step": round(hot_ms / args.steps, 4),
             "value": round(w.N * args.steps * ws / (hot_ms / 1e3), 1),
