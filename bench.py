@@ -44,6 +44,7 @@ from synthetic import get_workload, make_inputs  # noqa: E402
 
 METRIC = "dispatch+combine tokens/s and effective HBM GB/s (% of B200 peak), 1 GPU"
 L2_BYTES = 126 * 1024 * 1024
+E2E_DEPTH = 3  # device buffer sets the end-to-end pipeline rotates over
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -579,21 +580,22 @@ def run_ours(args, ws, rank, local):
     elapsed_ms = max_over_ranks(elapsed_ms, device)
 
     # end to end through the public API: every step copies its inputs in from pinned host
-    # memory and its combined output back out. Two pipelines of device buffers alternate, so
-    # step i's copy-out (one copy engine) overlaps step i+1's copy-in (the other) and its
+    # memory and its combined output back out. E2E_DEPTH sets of device buffers rotate, so
+    # step i's copy-out (one copy engine) overlaps the next steps' copy-in (the other) and
     # kernels; each step waits for the copy-in of its own inputs, and a buffer is written
     # again only after its previous copy-out finished.
     e2e = None
     if not args.no_e2e:
         pin = {key: torch.from_numpy(v if v.dtype != np.uint16 else v.view(np.int16)).pin_memory()
                for key, v in host.items()}
-        outs_host = [torch.empty((w.N, w.H), dtype=torch.int16).pin_memory() for _ in range(2)]
+        depth = E2E_DEPTH
+        outs_host = [torch.empty((w.N, w.H), dtype=torch.int16).pin_memory() for _ in range(depth)]
         h2d_s = torch.cuda.Stream(device)
         d2h_s = torch.cuda.Stream(device)
         comp_s = torch.cuda.Stream(device)
         pipes = []
         with torch.cuda.stream(comp_s):
-            for b in range(2):
+            for b in range(depth):
                 dset = {key: torch.empty_like(step.sets[0][key]) for key in pin}
                 pipes.append((EpStep if w.ep else Step)(w, moe, _native, torch, [dset], device))
         views = [{key: (q.sets[0][key].view(torch.int16) if q.sets[0][key].dtype == torch.bfloat16
@@ -601,11 +603,11 @@ def run_ours(args, ws, rank, local):
         h2d = sum(t.numel() * t.element_size() for t in pin.values())
         d2h = outs_host[0].numel() * outs_host[0].element_size()
         ev = lambda: torch.cuda.Event()  # noqa: E731
-        in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
-        started = [False, False]
+        in_done, comp_done, out_done = ([ev() for _ in range(depth)] for _ in range(3))
+        started = [False] * depth
 
         def e2e_step(i):
-            b = i % 2
+            b = i % depth
             if started[b]:
                 h2d_s.wait_event(comp_done[b])  # the kernels of step i-2 finished reading these inputs
             with torch.cuda.stream(h2d_s):
@@ -634,7 +636,7 @@ def run_ours(args, ws, rank, local):
         comp_s.wait_event(e0)
         for i in range(args.steps):
             e2e_step(i)
-        for b in range(2):  # the timed region ends when the last output is on the host
+        for b in range(depth):  # the timed region ends when the last output is on the host
             d2h_s.wait_event(out_done[b])
         e1.record(d2h_s)
         torch.cuda.synchronize()
@@ -651,7 +653,7 @@ def run_ours(args, ws, rank, local):
             "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
             "ms_per_step": round(e_ms / args.steps, 4),
-            "pipelining": "2 device buffer sets; copy-in, kernels and copy-out on three streams",
+            "pipelining": f"{depth} device buffer sets; copy-in, kernels and copy-out on three streams",
         }
         del pipes
 
