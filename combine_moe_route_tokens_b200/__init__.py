@@ -529,10 +529,17 @@ def moe_ep_plan(problem: Problem, offsets_all: torch.Tensor, src_rank: int, plan
     return plan
 
 
-def _table(peers, device) -> torch.Tensor:
+def _table(peers, device, problem: Optional[Problem] = None) -> torch.Tensor:
+    """A peer table as given (int64 device addresses), or built from R buffers after checking
+    that each is a [moe_ep_recv_rows_max, H] bf16 tensor."""
     if isinstance(peers, torch.Tensor) and peers.dtype == torch.int64:
         return peers
-    return peer_table(list(peers), device)
+    peers = list(peers)
+    if problem is not None:
+        rows = moe_ep_recv_rows_max(problem)
+        for r, b in enumerate(peers):
+            _need(b, f"buffer of rank {r}", torch.bfloat16, (rows, problem.H))
+    return peer_table(peers, device)
 
 
 def moe_ep_dispatch(problem: Problem, layout: Layout, plan: EpPlan, hidden: torch.Tensor, peer_recv,
@@ -543,7 +550,7 @@ def moe_ep_dispatch(problem: Problem, layout: Layout, plan: EpPlan, hidden: torc
     their ``peer_table``.
     """
     _need(hidden, "hidden", torch.bfloat16, (problem.N, problem.H), layout.device)
-    table = _table(peer_recv, layout.device)
+    table = _table(peer_recv, layout.device, problem)
     if table.numel() != problem.R:
         raise ValueError("peer_recv needs one buffer per rank")
     p = problem.c_struct()
@@ -555,7 +562,7 @@ def moe_ep_dispatch(problem: Problem, layout: Layout, plan: EpPlan, hidden: torc
 def moe_ep_combine(problem: Problem, layout: Layout, plan: EpPlan, peer_expert_out, topk_probs: Optional[torch.Tensor],
                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """out[t] = bf16(fp32 sum over ascending kept j of p[t,j] * (row of slot j on its expert's owner))."""
-    table = _table(peer_expert_out, layout.device)
+    table = _table(peer_expert_out, layout.device, problem)
     if table.numel() != problem.R:
         raise ValueError("peer_expert_out needs one buffer per rank")
     if topk_probs is not None:
@@ -581,8 +588,8 @@ def moe_ep_combine_backward(problem: Problem, layout: Layout, plan: EpPlan, grad
     """
     _need(grad_out, "grad_out", torch.bfloat16, (problem.N, problem.H), layout.device)
     _need(topk_probs, "topk_probs", torch.float32, (problem.N, problem.k), layout.device)
-    ty = _table(peer_expert_out, layout.device)
-    tg = _table(peer_grad_expert_out, layout.device)
+    ty = _table(peer_expert_out, layout.device, problem)
+    tg = _table(peer_grad_expert_out, layout.device, problem)
     if ty.numel() != problem.R or tg.numel() != problem.R:
         raise ValueError("one expert-output and one gradient buffer per rank")
     if grad_probs is None:
