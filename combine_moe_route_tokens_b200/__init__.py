@@ -51,6 +51,7 @@ COUNTER_NAMES = (
 __all__ = [
     "Problem",
     "Layout",
+    "CountsPrefetch",
     "MoeError",
     "moe_route_topk",
     "moe_dispatch_layout",
@@ -169,6 +170,22 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None, device=Non
 
 
 @dataclass
+class CountsPrefetch:
+    """Counts on their way to pinned host memory (Layout.prefetch_counts)."""
+
+    host: Dict[str, torch.Tensor]
+    event: "torch.cuda.Event"
+
+    def ready(self) -> bool:
+        return self.event.query()
+
+    def get(self) -> Dict[str, torch.Tensor]:
+        """The host tensors, waiting for the copies if they have not landed yet."""
+        self.event.synchronize()
+        return self.host
+
+
+@dataclass
 class Layout:
     """Device buffers of every dispatch-layout output plus the layout workspace."""
 
@@ -232,6 +249,24 @@ class Layout:
     def reset_workspace(self) -> None:
         """Zero the layout workspace (needed again only after a MOE_DEV_TIMEOUT)."""
         self.workspace.zero_()
+
+    def prefetch_counts(self, stream=None) -> "CountsPrefetch":
+        """Copy the per-expert and per-rank counts to pinned host memory without waiting.
+
+        The copies are enqueued after the work already on ``stream`` (the layout call),
+        so the host can read them later, off the critical path, instead of forcing a
+        synchronisation when it needs them (Megatron MORI: deferred count reads)."""
+        st = torch.cuda.current_stream(self.device) if stream is None else stream
+        keys = ("tokens_per_expert", "expert_offsets", "input_splits", "output_splits", "num_rows", "counters")
+        host = {}
+        with torch.cuda.stream(st):
+            for key in keys:
+                buf = torch.empty(self.tensors[key].shape, dtype=self.tensors[key].dtype, pin_memory=True)
+                buf.copy_(self.tensors[key], non_blocking=True)
+                host[key] = buf
+            done = torch.cuda.Event()
+            done.record(st)
+        return CountsPrefetch(host=host, event=done)
 
     def counters(self) -> Dict[str, int]:
         """dispatch_counters as a dict. Synchronises."""

@@ -653,3 +653,15 @@ def test_route_candidate_paths(kind):
     assert np.array_equal(host(gi), idx)
     tol = route_prob_tolerance(logits, idx) * probs.astype(np.float64)
     assert np.all(np.abs(host(gp).astype(np.float64) - probs.astype(np.float64)) <= tol)
+
+
+def test_counts_prefetch_to_host():
+    """Layout.prefetch_counts: pinned host copies of the counts, readable after the layout without a sync point."""
+    w, d, idx, probs, L = workload_case("capacity")
+    G = moe.moe_dispatch_layout(problem_of(w), dev(idx), dev(probs))
+    pf = G.prefetch_counts()
+    got = pf.get()
+    for key in ("tokens_per_expert", "expert_offsets", "input_splits", "output_splits", "num_rows", "counters"):
+        assert got[key].is_pinned()
+        assert np.array_equal(got[key].numpy().reshape(-1), np.asarray(L[key]).reshape(-1)), key
+    assert pf.ready()
