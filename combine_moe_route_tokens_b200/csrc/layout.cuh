@@ -9,8 +9,8 @@
 //            per-warp exclusive prefixes and publishes its per-expert total;
 //   barrier  bounded grid barrier (acquire/release atomics; co-residency is
 //            guaranteed by the cooperative launch);
-//   phase 2  every block reads all block totals in one batch of loads, so it
-//            knows per logical expert the total count and the count in
+//   phase 2  every block reads all block totals (16-byte loads, up to eight in
+//            flight per thread), so it knows per logical expert the total count and the count in
 //            earlier blocks; it derives the hot-expert placement, physical
 //            counts, capacity, the exclusive scan and the rank splits (block 0
 //            publishes them); then, with no further global reads, it writes

@@ -4,7 +4,8 @@
 // Every entry point validates on the host, then enqueues its kernel(s) on the
 // caller's stream and returns; nothing here synchronises with the device or
 // reads device memory. The only host state is a per-device cache of
-// attributes (SM count, shared-memory limit) and kernel attribute setup.
+// attributes (SM count, shared-memory limit) with the kernel attribute setup,
+// the programmatic-launch fallback flags and the NVTX switch.
 
 #include <cuda_runtime.h>
 
