@@ -85,14 +85,24 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source without comments and whitespace (what the compiler sees as code)."""
+    import re
+
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return "".join(text.split())
+
+
 def source_digest():
-    """Digest of the kernel sources, to tell whether a stored ncu capture still applies."""
+    """Digest of the kernel sources' code (comments and layout ignored), to tell whether a
+    stored ncu capture still applies."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "combine_moe_route_tokens_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode())
-            h.update(f.read())
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
