@@ -119,10 +119,13 @@ int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, void *s
     cfg.numAttrs = n;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
     if (e != cudaSuccess && n > n_base) {
+        // retry without the programmatic attribute; only if that launch succeeds was the
+        // attribute the cause, and only then is it dropped for later launches of this kind
         (void)cudaGetLastError();
-        pdl_ok.store(false, std::memory_order_relaxed);
         cfg.numAttrs = n_base;
         e = cudaLaunchKernelEx(&cfg, kernel, args...);
+        if (e == cudaSuccess)
+            pdl_ok.store(false, std::memory_order_relaxed);
     }
     if (e != cudaSuccess) {
         (void)cudaGetLastError();
