@@ -10,7 +10,9 @@
 // streaming loads in flight per thread), then accumulated in fp32 with one
 // fmaf per kept slot in ascending j from +0, and rounded once to bf16
 // (cvt.rn.bf16x2). No atomics: every output element has one writer. A warp
-// covers 512 contiguous bytes of each source row.
+// covers 512 contiguous bytes of each source row. Short rows with one or two
+// slots take combine_rows_kernel: several tokens per CTA, four chunks per
+// thread, the same arithmetic.
 //
 // Combine backward: one CTA per token walks the row in 16-byte chunks,
 // writes grad_y[dest_row[t,j]] = bf16(fp32(p[t,j] * g)) and accumulates the
@@ -266,6 +268,64 @@ __global__ void __launch_bounds__(COMBINE_THREADS, 4) combine_kernel(CombineArgs
             return;
     }
     st_u4(a.out + t * a.V + v, pack8(acc));
+}
+
+// Combine of short rows with one or two slots (one buffer). With one 16-byte
+// chunk per thread such a token gives a CTA at most 32 bytes to load per
+// thread, too little in flight to cover the memory latency, and tokens whose
+// slots were all dropped only load their metadata and store zeros. Here a
+// token's row is covered by V / COMBINE_ROW_CPT threads (whole warps), each
+// owning COMBINE_ROW_CPT chunks a row-quarter apart, and a CTA holds several
+// tokens: every load of every chunk is issued before the first multiply-add.
+// The arithmetic per element is the one of combine_kernel (fma chain in
+// ascending j from +0, one bf16 rounding). The host takes this kernel for k <= 2
+// and V in {128, 256, 512, 1024}, so COMBINE_THREADS is a multiple of the
+// threads per token.
+constexpr int COMBINE_ROW_CPT = 4;
+
+template <int K>
+__global__ void __launch_bounds__(COMBINE_THREADS, 4) combine_rows_kernel(CombineArgs a)
+{
+    pdl_trigger();
+    pdl_wait();
+    const int tpt = a.V / COMBINE_ROW_CPT; // threads per token: 32, 64, 128 or 256
+    const int u = static_cast<int>(threadIdx.x) / tpt, l = static_cast<int>(threadIdx.x) - u * tpt;
+    const int64_t tb = static_cast<int64_t>(blockIdx.x) * (COMBINE_THREADS / tpt) + u;
+    if (tb >= a.N) // whole warps: tpt is a multiple of 32
+        return;
+    const int64_t t = a.last_first ? a.N - 1 - tb : tb;
+    int32_t d;
+    float p;
+    load_slot_meta(a.dest_row, a.probs, t, K, a.rows_max, a.status, d, p);
+    int32_t dj[K];
+    float pj[K];
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+        dj[j] = __shfl_sync(0xffffffffu, d, j);
+        pj[j] = __shfl_sync(0xffffffffu, p, j);
+    }
+    uint4 yj[K][COMBINE_ROW_CPT];
+#pragma unroll
+    for (int j = 0; j < K; ++j)
+        if (dj[j] >= 0) {
+            const uint4 *row = a.y + static_cast<int64_t>(dj[j]) * a.V + l;
+#pragma unroll
+            for (int i = 0; i < COMBINE_ROW_CPT; ++i)
+                yj[j][i] = ld_stream_u4(row + i * tpt);
+        }
+    uint4 *out = a.out + t * a.V + l;
+#pragma unroll
+    for (int i = 0; i < COMBINE_ROW_CPT; ++i) {
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            acc[e] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < K; ++j)
+            if (dj[j] >= 0)
+                fma8(acc, pj[j], yj[j][i]);
+        st_u4(out + i * tpt, pack8(acc));
+    }
 }
 
 struct CombineBwdArgs {

@@ -479,6 +479,19 @@ namespace {
 extern "C++" template <int SRC>
 int launch_combine_args(CombineArgs a, int k, void *stream)
 {
+    if constexpr (SRC == SRC_LOCAL) {
+        // short rows with one or two slots: several tokens per CTA, four chunks per thread
+        if ((k == 1 || k == 2) && (a.V == 128 || a.V == 256 || a.V == 512 || a.V == 1024)) {
+            const int64_t per_cta = COMBINE_THREADS / (a.V / COMBINE_ROW_CPT);
+            const int64_t blocks = (a.N + per_cta - 1) / per_cta;
+            if (blocks > INT32_MAX)
+                return MOE_ERR_UNSUPPORTED;
+            const dim3 grid(static_cast<unsigned>(blocks)), block(COMBINE_THREADS);
+            if (k == 1)
+                return launch(combine_rows_kernel<1>, grid, block, 0, stream, false, a);
+            return launch(combine_rows_kernel<2>, grid, block, 0, stream, false, a);
+        }
+    }
     // the widest CTA (up to 256 threads) that splits the row into equal parts
     const int v32 = ((a.V + 31) / 32) * 32;
     const int threads = v32 % 256 == 0 ? 256 : (v32 % 128 == 0 ? 128 : (v32 % 64 == 0 ? 64 : 32));

@@ -397,6 +397,41 @@ def test_tp_fold_layout_permute_restore(case):
     assert all(G.status() == 0 for G in layouts)
 
 
+# ------------------------------------------- short rows with one or two slots
+
+ROW_CASES = [
+    # N, H, k, E_log, R, C, neg: k <= 2 with H / 8 in {128, 256, 512, 1024} takes the
+    # combine kernel that holds several tokens per CTA and four chunks per thread
+    (1, 1024, 1, 4, 2, 0, 0.0),  # a single token: one partly filled CTA
+    (1001, 1024, 2, 16, 2, 0, 0.1),  # eight tokens per CTA, ragged last CTA, -1 ids
+    (4099, 2048, 2, 64, 2, 60, 0.05),  # capacity: most tokens keep nothing, rows of zeros
+    (333, 4096, 1, 8, 4, 0, 0.2),  # two tokens per CTA
+    (77, 8192, 2, 32, 4, 3, 0.0),  # one token per CTA, heavy drops
+]
+
+
+@pytest.mark.parametrize("case", ROW_CASES, ids=[f"N{c[0]}_H{c[1]}_k{c[2]}_C{c[5]}" for c in ROW_CASES])
+def test_combine_short_rows(case):
+    N, H, k, E_log, R, C, neg = case
+    idx, probs, hidden = _small_case(N, H, k, E_log, R, C, 0, neg, seed=N + H, zipf=1.5)
+    L = oracle.layout(idx, probs, E_log=E_log, R=R, C=C)
+    p = moe.Problem(N=N, H=H, k=k, E_log=E_log, R=R, capacity=C)
+    G = moe.moe_dispatch_layout(p, dev(idx), dev(probs))
+    send = moe.moe_permute(p, G, dev(hidden))
+    exp_send = oracle.permute(hidden, L["dest_row"], L["rows_max"])
+    assert np.array_equal(host(send), exp_send)
+    for w in (probs, None):
+        out = moe.moe_combine(p, G, send, None if w is None else dev(w))
+        assert np.array_equal(host(out), oracle.combine(exp_send, L["dest_row"], w))
+    rng = np.random.default_rng(N)
+    g = bf16_bits_from_f32(rng.standard_normal((N, H)).astype(np.float32))
+    gy, _ = moe.moe_combine_backward(p, G, dev(g), send, dev(probs))
+    exp_gy, _ = oracle.combine_backward(g, exp_send, L["dest_row"], L["row_token"], L["row_prob"])
+    assert np.array_equal(host(gy), exp_gy)
+    assert np.array_equal(host(moe.moe_permute_backward(p, G, gy)), oracle.permute_backward(exp_gy, L["dest_row"]))
+    assert G.status() == 0
+
+
 # ------------------------------------------------------- DeepEP-style dedup
 
 
@@ -408,6 +443,7 @@ DEDUP_CASES = [
     (2049, 24, 8, 64, 8, 0, 8, 0, 2),  # reroute + TP folding (peer 0)
     (300, 16, 12, 48, 16, 0, 0, 0, 0),  # k > 8, E_loc not a multiple of 16
     (70000, 8, 1, 4, 2, 0, 0, 0, 0),  # many tokens, several per lane
+    (2500, 2048, 2, 16, 2, 0, 0, 0, 0),  # sender-side sum over two ranks on 4 KB rows
 ]
 
 
