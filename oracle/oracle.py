@@ -18,6 +18,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.c")
 _HDR = os.path.join(_HERE, "moe_oracle.h")
 _LIB = os.path.join(_HERE, "libmoe_oracle.so")
+# MOE_ORACLE_LIB names a prebuilt variant of the library to load instead; the
+# mutation tests build copies of moe_oracle.c with one planted mistake each and
+# check that the pins reject every one of them.
+_LIB_OVERRIDE = os.environ.get("MOE_ORACLE_LIB") or None
 
 COUNTER_NAMES = (
     "assignments_total",
@@ -32,11 +36,13 @@ COUNTER_NAMES = (
 
 
 def library_path() -> str:
-    return _LIB
+    return _LIB_OVERRIDE or _LIB
 
 
 def build(force: bool = False) -> str:
     """Compile the oracle into ``oracle/libmoe_oracle.so`` (gcc, no fast-math, no FP contraction)."""
+    if _LIB_OVERRIDE:  # a prebuilt variant: nothing to compile
+        return _LIB_OVERRIDE
     stale = (
         not os.path.exists(_LIB)
         or os.path.getmtime(_LIB) < max(os.path.getmtime(_SRC), os.path.getmtime(_HDR))
@@ -127,7 +133,7 @@ def _lib() -> ctypes.CDLL:
     global _lib_handle
     if _lib_handle is None:
         build()
-        lib = ctypes.CDLL(_LIB)
+        lib = ctypes.CDLL(library_path())
         lib.oracle_problem_valid.restype = ctypes.c_int
         lib.oracle_problem_valid.argtypes = [ctypes.POINTER(_Problem)]
         lib.oracle_rows_max.restype = ctypes.c_int64
