@@ -7,7 +7,8 @@ named beside it against that library (MOE_ORACLE_LIB) in a child pytest. The
 case passes when the child reports a failing test: some pin caught the mistake.
 A control build of the unmodified source must pass the same pins, so that a
 failure cannot come from the harness itself. Every planted mistake keeps all
-memory accesses inside their buffers.
+memory accesses inside their buffers. The numpy exchange (oracle.ep_exchange)
+is mutated the same way in a copy of its source, in this process.
 """
 
 import os
@@ -137,3 +138,61 @@ def test_pins_reject_planted_mistake(source, tmp_path, mutant):
     r = _run_pins(_build(source.replace(old, new), str(tmp_path), name), files)
     # 1 = some test failed; anything else (a crash, a collection error) is not a pin at work
     assert r.returncode == 1, f"{name}: the pins did not reject it (exit {r.returncode})\n{r.stdout[-2000:]}"
+
+
+# The expert-parallel exchange of the oracle is numpy (oracle.ep_exchange): its
+# planted mistakes are made in a copy of the function's source, and the exchange
+# pins of tests/test_oracle_ep.py run in this process against the copy.
+EP_MUTANTS = [
+    ("ep_sources_descending", "            for s in range(S):", "            for s in reversed(range(S)):"),
+    ("ep_experts_descending", "        for q in range(r * E_loc, (r + 1) * E_loc):",
+     "        for q in reversed(range(r * E_loc, (r + 1) * E_loc)):"),
+    ("ep_padding_rows_left_out",
+     'lo, hi = int(layouts[s]["expert_offsets"][q]), int(layouts[s]["expert_offsets"][q + 1])',
+     'lo = int(layouts[s]["expert_offsets"][q]); hi = lo + int(layouts[s]["tokens_per_expert"][q])'),
+    ("ep_base_after_the_rows", "                base[s][q] = pos\n                blocks.append(sends[s][lo:hi])\n"
+     "                pos += hi - lo\n",
+     "                blocks.append(sends[s][lo:hi])\n                pos += hi - lo\n                base[s][q] = pos\n"),
+    ("ep_expert_offsets_shifted", "            offs.append(pos)\n            for s in range(S):",
+     "            for s in range(S):\n                offs.append(pos) if s == S - 1 else None"),
+]
+
+
+def _ep_variant(old=None, new=None):
+    import inspect
+    import textwrap
+    import types
+
+    import numpy as np
+
+    import oracle
+
+    src = textwrap.dedent(inspect.getsource(oracle.oracle.ep_exchange))
+    if old is not None:
+        assert src.count(old) == 1, "the planted text must occur exactly once"
+        src = src.replace(old, new)
+    ns = {"np": np}
+    exec(compile(src, "<ep_exchange variant>", "exec"), ns)
+    return types.SimpleNamespace(layout=oracle.layout, permute=oracle.permute, combine=oracle.combine,
+                                 ep_exchange=ns["ep_exchange"])
+
+
+def _ep_pins_fail(lib):
+    import test_oracle_ep
+
+    for case in test_oracle_ep.CASES:
+        try:
+            test_oracle_ep.test_exchange_delivers_every_kept_assignment_once(lib, case)
+        except (AssertionError, ValueError, IndexError):  # a failed pin, as pytest would count it
+            return True
+    return False
+
+
+def test_ep_control_passes_the_pins():
+    assert not _ep_pins_fail(_ep_variant())
+
+
+@pytest.mark.parametrize("mutant", EP_MUTANTS, ids=[m[0] for m in EP_MUTANTS])
+def test_ep_pins_reject_planted_mistake(mutant):
+    name, old, new = mutant
+    assert _ep_pins_fail(_ep_variant(old, new)), f"{name}: the exchange pins did not reject it"
