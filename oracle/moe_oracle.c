@@ -169,7 +169,7 @@ void oracle_route_topk(const float *logits, const uint8_t *token_mask, int64_t N
  *  7. the per-rank DeepEP-contract view local_topk and dispatch_counters
  *     ([DeepSpeed EP] dispatch_counters).
  *
- * Readings where the pages are silent (see the design notes): first-come drop
+ * Readings where the pages are silent (taken here, not from the pages): first-come drop
  * in flattened order; hot set = the num_replicas largest logical counts,
  * equal counts to the lower id; greedy placement onto the least-loaded other
  * rank with a free slot; a hot expert's logical ordinal o goes to the master
