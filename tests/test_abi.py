@@ -116,6 +116,19 @@ def test_layout_requires_outputs_and_workspace(lib):
                                    ctypes.c_void_p(256), 1 << 20, None) == _native.MOE_ERR_INVALID
 
 
+def test_layout_rejects_undersized_or_misaligned_workspace(lib):
+    # every output pointer set (fake addresses: the checks run on the host, before any
+    # device work), so only the workspace decides
+    p = moe.Problem(N=4, H=8, k=2, E_log=4, R=2)
+    L = _native.MoeLayout(**{name: 4096 * (i + 1) for i, name in enumerate(_native.LAYOUT_FIELDS)})
+    need = p.workspace_bytes
+    f = lib.moe_dispatch_layout
+    args = (ctypes.byref(p.c_struct()), ctypes.c_void_p(1 << 20), None, ctypes.byref(L))
+    assert f(*args, ctypes.c_void_p(1 << 24), need - 1, None) == _native.MOE_ERR_INVALID  # one byte short
+    assert f(*args, ctypes.c_void_p((1 << 24) + 128), need, None) == _native.MOE_ERR_INVALID  # not 256-byte aligned
+    assert f(*args, None, need, None) == _native.MOE_ERR_INVALID
+
+
 def test_route_argument_checks(lib):
     f = lib.moe_route_topk
     assert f(None, None, 4, 8, 0, None, None, None) == _native.MOE_ERR_INVALID  # k = 0
