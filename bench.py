@@ -51,6 +51,11 @@ FALLBACK_HBM_GBS = 6650.0
 # ----------------------------------------------------------------- helpers
 
 
+# C-ABI calls that enqueue more than one kernel (the dedup layout: placement, then the
+# per-row fill); every other call is one kernel
+KERNELS_PER_CALL = {"dedup_layout": 2}
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -725,7 +730,7 @@ def run_ours(args, ws, rank, local):
             "frac": round(ach / peak, 3),
             "traffic": stored_traffic(dominant, w.name),
         },
-        "gpu_launches": args.steps * len(step.kernel_names),
+        "gpu_launches": args.steps * sum(KERNELS_PER_CALL.get(n, 1) for n in step.kernel_names),
         "kernel_timing": "per-kernel CUDA events in a second pass of the same K steps (launched eagerly)",
         "launch": launch_mode,
         "hot_l2": {
