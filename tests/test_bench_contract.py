@@ -1,0 +1,56 @@
+"""The benchmark's command-line contract on CPU: the reference arm's JSON line (the
+oracle timed on the host cores), its behaviour on ranks other than 0, and the
+warm-up floor. The GPU arm's line is produced only on a GPU machine.
+"""
+
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench(*args, env=None):
+    e = dict(os.environ)
+    for key in ("RANK", "LOCAL_RANK", "WORLD_SIZE"):
+        e.pop(key, None)
+    e.update(env or {})
+    return subprocess.run([sys.executable, "bench.py", *args], cwd=ROOT, env=e, capture_output=True, text=True,
+                          timeout=600)
+
+
+def _last_json(stdout):
+    lines = [line for line in stdout.splitlines() if line.startswith("{")]
+    assert len(lines) == 1, stdout
+    return json.loads(lines[0])
+
+
+def test_reference_arm_line():
+    r = _bench("--impl", "reference", "--workload", "tiny", "--steps", "3", "--warmup", "3")
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = _last_json(r.stdout)
+    assert d["impl"] == "reference"
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["steps"] == 3 and d["warmup"] == 3 and d["n_gpus"] == 1
+    assert d["unit"] == "tokens/s" and d["higher_is_better"] is True and d["value"] > 0
+    assert d["config"]["workload"] == "tiny" and "model" not in d["config"]
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] == d["value"] and cb["sample"]
+    e2e = d["e2e"]
+    assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    r = _bench("--impl", "reference", "--workload", "tiny", "--steps", "3", "--warmup", "3", "--gpus", "2",
+               env={"RANK": "1", "LOCAL_RANK": "1", "WORLD_SIZE": "2"})
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert not [line for line in r.stdout.splitlines() if line.startswith("{")]
+
+
+def test_warmup_floor():
+    r = _bench("--impl", "reference", "--workload", "tiny", "--steps", "3", "--warmup", "2")
+    assert r.returncode == 2 and "--warmup must be >= 3" in r.stderr
