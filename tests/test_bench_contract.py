@@ -54,3 +54,15 @@ def test_reference_arm_other_ranks_exit_without_work():
 def test_warmup_floor():
     r = _bench("--impl", "reference", "--workload", "tiny", "--steps", "3", "--warmup", "2")
     assert r.returncode == 2 and "--warmup must be >= 3" in r.stderr
+
+
+def test_traffic_digest_ignores_comments_and_layout_only():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    code = "__global__ void k(int *p)\n{\n    p[0] = 1; // one\n}\n"
+    same = "/* a new comment */\n__global__ void k(int *p) {\n  p[0] = 1;   // changed comment\n}\n"
+    other = "__global__ void k(int *p)\n{\n    p[0] = 2; // one\n}\n"
+    assert bench._code_only(code) == bench._code_only(same)
+    assert bench._code_only(code) != bench._code_only(other)
+    assert bench.stored_traffic("permute", "no_such_workload") is None
