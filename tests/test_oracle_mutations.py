@@ -48,6 +48,10 @@ MUTANTS = [
      "o->rank_offsets[r] = o->expert_offsets[r];", LAYOUT),
     ("layout_row_slot_transposed", "o->row_slot[row] = (int32_t)(a % k);", "o->row_slot[row] = (int32_t)(a / k);",
      LAYOUT),
+    ("layout_rows_not_aligned", "        while (rows % A != 0)\n            ++rows;\n", "", LAYOUT),
+    ("layout_capacity_rows_from_counts",
+     "int32_t rows = C > 0 ? oracle_local_capacity(p) : o->tokens_per_expert[e];",
+     "int32_t rows = o->tokens_per_expert[e];", LAYOUT),
     ("layout_local_id_not_rebased", "o->local_topk[(int64_t)r * NK + a] = keep ? q - r * E_loc : -1;",
      "o->local_topk[(int64_t)r * NK + a] = keep ? q : -1;", LAYOUT),
     ("layout_row_prob_of_slot_zero", "o->row_prob[row] = topk_probs ? topk_probs[a] : 0.0f;",
@@ -95,6 +99,8 @@ MUTANTS = [
     ("dedup_tokens_descending",
      "        for (int64_t t = 0; t < N; ++t) {\n            if (!o->is_token_in_rank[t * R + r]) {",
      "        for (int64_t t = N - 1; t >= 0; --t) {\n            if (!o->is_token_in_rank[t * R + r]) {", DEDUP),
+    ("dedup_weight_of_slot_zero", "float w = topk_probs ? topk_probs[t * k + j] : 0.0f;",
+     "float w = topk_probs ? topk_probs[t * k] : 0.0f;", DEDUP),
     ("dedup_multihot_not_set", "o->recv_routing_map[(int64_t)row * E_loc + local] = 1;",
      "o->recv_routing_map[(int64_t)row * E_loc + local] = 0;", DEDUP),
     ("dedup_partial_takes_next_rank_row", "if (d < rank_offsets[r] || d >= rank_offsets[r + 1])",
