@@ -7,6 +7,11 @@ imports nothing from the product.
 
 from .oracle import (
     build,
+    build_omp,
+    omp_threads,
+    omp_route_topk,
+    omp_permute,
+    omp_combine,
     library_path,
     rows_max,
     num_experts,
@@ -26,6 +31,11 @@ from .oracle import (
 
 __all__ = [
     "build",
+    "build_omp",
+    "omp_threads",
+    "omp_route_topk",
+    "omp_permute",
+    "omp_combine",
     "library_path",
     "rows_max",
     "num_experts",

@@ -18,6 +18,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.c")
 _HDR = os.path.join(_HERE, "moe_oracle.h")
 _LIB = os.path.join(_HERE, "libmoe_oracle.so")
+_OMP_SRC = os.path.join(_HERE, "moe_oracle_omp.c")
+_OMP_LIB = os.path.join(_HERE, "libmoe_oracle_omp.so")
 # MOE_ORACLE_LIB names a prebuilt variant of the library to load instead; the
 # mutation tests build copies of moe_oracle.c with one planted mistake each and
 # check that the pins reject every one of them.
@@ -65,6 +67,27 @@ def build(force: bool = False) -> str:
         subprocess.run(cmd, check=True)
         os.replace(_LIB + ".tmp", _LIB)
     return _LIB
+
+
+def build_omp(force: bool = False) -> str:
+    """Compile the all-cores variant ``oracle/libmoe_oracle_omp.so``: moe_oracle_omp.c (OpenMP over
+    tokens for route, permute and combine, calling the unchanged oracle functions) linked with its
+    own copy of moe_oracle.c, built with the same flags as the oracle plus -fopenmp."""
+    srcs = (_SRC, _HDR, _OMP_SRC)
+    stale = not os.path.exists(_OMP_LIB) or os.path.getmtime(_OMP_LIB) < max(os.path.getmtime(x) for x in srcs)
+    if force or stale:
+        # the first compiler that has an OpenMP runtime ($CC may be a toolchain without libgomp)
+        last = None
+        for cc in dict.fromkeys([os.environ.get("CC", "gcc"), "gcc", "/usr/bin/gcc"]):
+            cmd = [cc, "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
+                   "-Wall", "-o", _OMP_LIB + ".tmp", _OMP_SRC, _SRC, "-lm"]
+            last = subprocess.run(cmd, capture_output=True, text=True)
+            if last.returncode == 0:
+                break
+        if last.returncode != 0:
+            raise RuntimeError("no C compiler with OpenMP found: " + last.stderr[-500:])
+        os.replace(_OMP_LIB + ".tmp", _OMP_LIB)
+    return _OMP_LIB
 
 
 class _Problem(ctypes.Structure):
@@ -428,3 +451,64 @@ def combine_backward(grad_out: np.ndarray, expert_out: np.ndarray, dest_row: np.
     _lib().oracle_combine_backward(ctypes.byref(p), H, RM, _ptr(dest_row), _ptr(row_token), _ptr(row_prob),
                                    _ptr(grad_out), _ptr(expert_out), _ptr(gy), _ptr(gp))
     return gy, gp
+
+
+# ------------------------------------------------------------ all host cores
+# The token-independent steps through libmoe_oracle_omp.so: the same oracle functions, each
+# thread on a contiguous chunk of tokens (a timing baseline; results equal the serial calls).
+
+_omp_handle: Optional[ctypes.CDLL] = None
+
+
+def _omp() -> ctypes.CDLL:
+    global _omp_handle
+    if _omp_handle is None:
+        build_omp()
+        lib = ctypes.CDLL(_OMP_LIB)
+        lib.oracle_omp_threads.restype = ctypes.c_int
+        lib.oracle_omp_threads.argtypes = []
+        lib.oracle_omp_route_topk.restype = None
+        lib.oracle_omp_route_topk.argtypes = [_P, _P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P, _P]
+        lib.oracle_omp_permute.restype = None
+        lib.oracle_omp_permute.argtypes = [ctypes.POINTER(_Problem), ctypes.c_int32, _P, ctypes.c_int64, _P, _P]
+        lib.oracle_omp_combine.restype = None
+        lib.oracle_omp_combine.argtypes = [ctypes.POINTER(_Problem), ctypes.c_int32, _P, _P, _P, _P]
+        _omp_handle = lib
+    return _omp_handle
+
+
+def omp_threads() -> int:
+    """Threads the all-cores variant runs with (OMP_NUM_THREADS, else every host core)."""
+    return int(_omp().oracle_omp_threads())
+
+
+def omp_route_topk(logits: np.ndarray, k: int, token_mask: Optional[np.ndarray] = None):
+    logits = _c(logits, np.float32)
+    N, E = logits.shape
+    idx = np.empty((N, k), np.int32)
+    probs = np.empty((N, k), np.float32)
+    mask = None if token_mask is None else _c(token_mask, np.uint8)
+    _omp().oracle_omp_route_topk(_ptr(logits), _ptr(mask), N, E, k, _ptr(idx), _ptr(probs))
+    return idx, probs
+
+
+def omp_permute(hidden: np.ndarray, dest_row: np.ndarray, rows_max: int) -> np.ndarray:
+    hidden = _c(hidden, np.uint16)
+    dest_row = _c(dest_row, np.int32)
+    N, H = hidden.shape
+    p = _Problem(N=N, k=dest_row.shape[1], E_log=1, num_replicas=0, R=1, C=0)
+    send = np.empty((rows_max, H), np.uint16)
+    _omp().oracle_omp_permute(ctypes.byref(p), H, _ptr(dest_row), rows_max, _ptr(hidden), _ptr(send))
+    return send
+
+
+def omp_combine(expert_out: np.ndarray, dest_row: np.ndarray, topk_probs: Optional[np.ndarray]) -> np.ndarray:
+    expert_out = _c(expert_out, np.uint16)
+    dest_row = _c(dest_row, np.int32)
+    N, k = dest_row.shape
+    H = expert_out.shape[1]
+    probs = None if topk_probs is None else _c(topk_probs, np.float32)
+    p = _Problem(N=N, k=k, E_log=1, num_replicas=0, R=1, C=0)
+    out = np.empty((N, H), np.uint16)
+    _omp().oracle_omp_combine(ctypes.byref(p), H, _ptr(dest_row), _ptr(expert_out), _ptr(probs), _ptr(out))
+    return out
