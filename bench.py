@@ -4,7 +4,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ht] [--impl ours|reference]
 
 A step is one pass of the whole hot path over one batch of synthetic input:
-router top-k -> dispatch layout -> permute -> (identity experts) -> combine,
+router top-k -> dispatch (the layout and the permute, fused: moe_dispatch) ->
+(identity experts) -> combine,
 plus combine-backward and permute-backward for workloads that train
 (``ultraep``). Inputs are resident in HBM when the timed region starts and
 rotate over several buffer sets whose total size exceeds the 126 MB L2, so no
@@ -51,9 +52,15 @@ FALLBACK_HBM_GBS = 6650.0
 # ----------------------------------------------------------------- helpers
 
 
-# C-ABI calls that enqueue more than one kernel (the dedup layout: placement, then the
-# per-row fill); every other call is one kernel
-KERNELS_PER_CALL = {"dedup_layout": 2}
+# C-ABI calls that enqueue more than one kernel (the dispatch layout: count + look-back,
+# then the row-map fill; the fused dispatch: count + look-back, then fill + row copy; the
+# dedup layout: placement, then the per-row fill); every other call is one kernel
+KERNELS_PER_CALL = {"layout": 2, "dispatch": 2, "dedup_layout": 2}
+
+
+def kernels_per_call(name: str) -> int:
+    """Kernels one call enqueues; per-peer names such as 'layout.1' count as their base call."""
+    return KERNELS_PER_CALL.get(name.split(".")[0], 1)
 
 
 def dist_env():
@@ -140,10 +147,9 @@ class ClockSampler:
         0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.002):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.period = period_s
-        self.samples = []
-        self.reasons = 0
+        self.samples = []  # (time.perf_counter(), SM MHz, reason bits)
         self.max_mhz = None
         self._stop = threading.Event()
         self._thread = None
@@ -163,14 +169,16 @@ class ClockSampler:
         nv = self._nv
         while not self._stop.is_set():
             try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                bits = int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+                self.samples.append((time.perf_counter(), mhz, bits))
             except Exception:
                 pass
             time.sleep(self.period)
 
     def __enter__(self):
         if self.ok:
+            self._stop.clear()
             self._thread = threading.Thread(target=self._run, daemon=True)
             self._thread.start()
         return self
@@ -179,17 +187,43 @@ class ClockSampler:
         if self._thread is not None:
             self._stop.set()
             self._thread.join()
+            self._thread = None
 
-    def summary(self):
+    @staticmethod
+    def mark() -> float:
+        return time.perf_counter()
+
+    def summary(self, window=None):
+        """Median SM clock and the clock-event reasons over every sample taken while the
+        GPU ran the benchmark (warm-up, both timed passes, the other workloads), with the
+        sample count; the same for the samples inside the headline's timed region."""
         if not self.ok:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml_unavailable"]}
-        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
-        return {
-            "sm_mhz": statistics.median(self.samples) if self.samples else None,
+
+        def names(bits):
+            return [n for bit, n in self.REASONS.items() if bits & bit]
+
+        allbits = 0
+        for _, _, b in self.samples:
+            allbits |= b
+        out = {
+            "sm_mhz": statistics.median([m for _, m, _ in self.samples]) if self.samples else None,
             "sm_max_mhz": self.max_mhz,
-            "reasons": names,
+            "reasons": names(allbits),
             "samples": len(self.samples),
+            "sampled": "NVML every ~1 ms while the GPU ran the benchmark's steps",
         }
+        if window is not None:
+            inside = [(m, b) for t, m, b in self.samples if window[0] <= t <= window[1]]
+            wbits = 0
+            for _, b in inside:
+                wbits |= b
+            out["timed_region"] = {
+                "sm_mhz": statistics.median([m for m, _ in inside]) if inside else None,
+                "reasons": names(wbits),
+                "samples": len(inside),
+            }
+        return out
 
 
 # ------------------------------------------------------------- GPU arm
@@ -202,7 +236,7 @@ class Step:
     layout and the send buffer of every peer in turn (all on this GPU), and
     restores with one slot-ordered combine over the peers' buffers."""
 
-    def __init__(self, w, moe, native, torch, sets, device):
+    def __init__(self, w, moe, native, torch, sets, device, unfused=False):
         self.w = w
         self.torch = torch
         self.lib = native.lib()
@@ -257,6 +291,14 @@ class Step:
                     ("dedup_combine_local", self.lib.moe_dedup_combine_local,
                      (P, L, D, vp(self.send), vp(self.probs), vp(self.partial), self._s)),
                     ("dedup_combine", self.lib.moe_dedup_combine, (P, D, vp(self.partial), vp(self.out), self._s)),
+                ]
+            elif T == 1 and not unfused:
+                ws = self.layout.workspace
+                c += [
+                    ("dispatch", self.lib.moe_dispatch,
+                     (P, vp(self.idx), vp(self.probs), L, vp(ws), ws.numel(), vp(s["hidden"]), vp(self.send),
+                      self._s)),
+                    ("combine", self.lib.moe_combine, (P, L, vp(self.send), vp(self.probs), vp(self.out), self._s)),
                 ]
             elif T == 1:
                 ws = self.layout.workspace
@@ -319,6 +361,9 @@ class Step:
         if T == 1:
             out["layout"] = layout_bytes
             out["permute"] = read[0] * row + RM * row + NK * 4 + RM
+            # the fused call moves the layout's bytes and the row copy's, without the
+            # permute's re-read of the row map
+            out["dispatch"] = layout_bytes + read[0] * row + RM * row
             out["combine"] = kept[0] * row + N * row + NK * 8
         else:
             for r in range(T):
@@ -465,6 +510,150 @@ class EpStep:
         }
 
 
+def device_sets(w, host, torch, device):
+    """Input buffer sets resident in HBM: one generated batch plus token-rotated copies
+    of it (same distribution, different buffers and token order), together larger than
+    twice the 126 MB L2 so that no step reads inputs a previous step left in L2."""
+    set_bytes = sum(v.nbytes for v in host.values())
+    nsets = max(2, min(8, math.ceil(2 * L2_BYTES / set_bytes)))
+    base = {
+        "logits": torch.from_numpy(host["logits"]).to(device),
+        "hidden": torch.from_numpy(host["hidden"].view(np.int16)).to(device).view(torch.bfloat16),
+    }
+    if w.backward:
+        base["grad_out"] = torch.from_numpy(host["grad_out"].view(np.int16)).to(device).view(torch.bfloat16)
+    sets = []
+    for s in range(nsets):
+        shift = (s * 7919) % max(w.N, 1)
+        sets.append({key: torch.roll(v, shifts=shift, dims=0).contiguous() for key, v in base.items()})
+    return sets, nsets, set_bytes
+
+
+def measure(w, host, steps, warmup, eager, hot_l2, ctx):
+    """Times `steps` whole steps of workload `w` on this rank's GPU.
+
+    Timed region 1: the K steps back to back between two CUDA events on the launching
+    stream (each buffer set's step captured once into a CUDA graph and replayed, unless
+    `eager`), barrier and synchronize on both sides, max over ranks. Optionally the same
+    K steps on one buffer set (inputs in L2, for comparison). Timed region 2: the same K
+    steps launched eagerly with events around every call, for per-call durations."""
+    torch, moe, _native, device, barrier = ctx["torch"], ctx["moe"], ctx["native"], ctx["device"], ctx["barrier"]
+    sets, nsets, set_bytes = device_sets(w, host, torch, device)
+    # a stream of our own (not the legacy default stream), so that steps can be captured
+    work_stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(work_stream):
+        step = EpStep(w, moe, _native, torch, sets, device) if w.ep else \
+            Step(w, moe, _native, torch, sets, device, unfused=ctx.get("unfused", False))
+    for i in range(warmup):
+        step.run(i)
+    torch.cuda.synchronize()
+    abytes = step.algorithmic_bytes()
+
+    # one CUDA graph per buffer set, captured from the same C-ABI calls (the launches
+    # keep their programmatic-dependent-launch edges) and replayed in the timed region
+    run_step = step.run
+    launch_mode = "eager C-ABI calls, programmatic dependent launch"
+    graphs = []
+    if not eager:
+        try:
+            for i in range(len(step.calls)):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=work_stream):
+                    step.run(i)
+                graphs.append(g)
+        except Exception as exc:  # a driver without capture support: time the calls themselves
+            graphs = []
+            torch.cuda.synchronize()
+            launch_mode += f" (graph capture failed: {type(exc).__name__})"
+    if graphs:
+        launch_mode = "one CUDA graph per buffer set (captured C-ABI calls, programmatic dependent launch), replayed"
+
+        def run_step(i, events=None):
+            with torch.cuda.stream(work_stream):  # replay where the events are recorded
+                graphs[i % len(graphs)].replay()
+
+        for i in range(warmup):
+            run_step(i)
+        torch.cuda.synchronize()
+
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    tr0 = ctx["sampler"].mark()
+    t0.record(step.stream)
+    for i in range(steps):
+        run_step(warmup + i)
+    t1.record(step.stream)
+    torch.cuda.synchronize()
+    tr1 = ctx["sampler"].mark()
+    barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    hot_ms = None
+    if hot_l2:
+        h0 = torch.cuda.Event(enable_timing=True)
+        h1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        h0.record(step.stream)
+        for i in range(steps):
+            run_step(0)
+        h1.record(step.stream)
+        torch.cuda.synchronize()
+        barrier()
+        hot_ms = max_over_ranks(h0.elapsed_time(h1), device)
+    nk = len(step.kernel_names)
+    events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nk)]
+              for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        step.run(warmup + i, events[i])
+    torch.cuda.synchronize()
+    barrier()
+    per_kernel_ms = {name: [] for name in step.kernel_names}
+    for i in range(steps):
+        for n, name in enumerate(step.kernel_names):
+            per_kernel_ms[name].append(events[i][n][0].elapsed_time(events[i][n][1]))
+    status = step.status()
+    if status != 0:
+        raise RuntimeError(f"device status {status:#x} after the timed steps of '{w.name}'")
+    elapsed_ms = max_over_ranks(elapsed_ms, device)
+    del graphs
+    return {
+        "step": step, "abytes": abytes, "elapsed_ms": elapsed_ms, "hot_ms": hot_ms, "per_kernel_ms": per_kernel_ms,
+        "launch_mode": launch_mode, "nsets": nsets, "set_bytes": set_bytes, "timed_window": (tr0, tr1),
+    }
+
+
+def kernel_table(m, peak):
+    """Per-call figures of a measurement: mean / median / p10 / p90 µs, algorithmic bytes, GB/s, frac."""
+    step = m["step"]
+    kernels = {}
+    for name in step.kernel_names:
+        vals = m["per_kernel_ms"][name]
+        avg_ms = statistics.mean(vals)
+        qs = statistics.quantiles(vals, n=10) if len(vals) > 1 else [avg_ms] * 9
+        gbs = m["abytes"][name] / (avg_ms * 1e-3) / 1e9
+        kernels[name] = {
+            "calls_per_step": step.kernel_names.count(name),
+            "us": round(avg_ms * 1e3, 2),
+            "median_us": round(statistics.median(vals) * 1e3, 2),
+            "p10_us": round(qs[0] * 1e3, 2),
+            "p90_us": round(qs[8] * 1e3, 2),
+            "algorithmic_bytes": m["abytes"][name],
+            "gbs": round(gbs, 1),
+            "frac": round(gbs / peak, 3),
+        }
+    return kernels
+
+
+# The surveyed configurations timed beside the headline in the default run (parity cases
+# of the same path; each gets its step time, per-call figures and roofline fractions).
+EXTRA_WORKLOADS = ("tiny", "qwen3", "capacity", "ultraep")
+EXTRA_STEPS, EXTRA_WARMUP = 20, 3
+
+
 def run_ours(args, ws, rank, local):
     import torch
     import torch.distributed as tdist
@@ -484,115 +673,20 @@ def run_ours(args, ws, rank, local):
         tdist.barrier()
     moe.load_library()
 
-    w = get_workload(args.workload)
-    if args.tokens:  # a smaller batch of the same workload (profiling captures), named as such
-        w = w.scaled(args.tokens)
-    host = rank_inputs(w, rank)
-    set_bytes = sum(v.nbytes for v in host.values())
-    nsets = max(2, min(8, math.ceil(2 * L2_BYTES / set_bytes)))
-    # one generated batch; the other sets are token-rotated copies of it (same distribution,
-    # different buffers and different token order)
-    base = {
-        "logits": torch.from_numpy(host["logits"]).to(device),
-        "hidden": torch.from_numpy(host["hidden"].view(np.int16)).to(device).view(torch.bfloat16),
-    }
-    if w.backward:
-        base["grad_out"] = torch.from_numpy(host["grad_out"].view(np.int16)).to(device).view(torch.bfloat16)
-    sets = []
-    for s in range(nsets):
-        shift = (s * 7919) % max(w.N, 1)
-        sets.append({key: torch.roll(v, shifts=shift, dims=0).contiguous() for key, v in base.items()})
-    del base
-    # a stream of our own (not the legacy default stream), so that steps can be captured
-    work_stream = torch.cuda.Stream(device)
-    with torch.cuda.stream(work_stream):
-        step = (EpStep if w.ep else Step)(w, moe, _native, torch, sets, device)
-
     def barrier():
         if ws > 1:
             tdist.barrier()
 
-    # warm-up
-    for i in range(args.warmup):
-        step.run(i)
-    torch.cuda.synchronize()
-    abytes = step.algorithmic_bytes()
-
-    # one CUDA graph per buffer set, captured from the same C-ABI calls (the launches
-    # keep their programmatic-dependent-launch edges) and replayed in the timed
-    # region; --eager times the calls themselves
-    run_step = step.run
-    launch_mode = "eager C-ABI calls, programmatic dependent launch"
-    if not args.eager:
-        graphs = []
-        try:
-            for i in range(len(step.calls)):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=work_stream):
-                    step.run(i)
-                graphs.append(g)
-        except Exception as exc:  # a driver without capture support: time the calls themselves
-            graphs = []
-            torch.cuda.synchronize()
-            launch_mode += f" (graph capture failed: {type(exc).__name__})"
-    if not args.eager and graphs:
-        launch_mode = "one CUDA graph per buffer set (captured C-ABI calls, programmatic dependent launch), replayed"
-
-        def run_step(i, events=None):
-            with torch.cuda.stream(work_stream):  # replay where the events are recorded
-                graphs[i % len(graphs)].replay()
-
-        for i in range(args.warmup):
-            run_step(i)
-        torch.cuda.synchronize()
-
-    nk = len(step.kernel_names)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
+    w = get_workload(args.workload)
+    if args.tokens:  # a smaller batch of the same workload (profiling captures), named as such
+        w = w.scaled(args.tokens)
+    host = rank_inputs(w, rank)
     sampler = ClockSampler(local)
-    # timed region 1: K whole steps back to back (kernels launched with programmatic
-    # dependent launch overlap their launch with the previous kernel's tail)
-    barrier()
-    torch.cuda.synchronize()
+    ctx = {"torch": torch, "moe": moe, "native": _native, "device": device, "barrier": barrier, "sampler": sampler,
+           "unfused": args.unfused}
     with sampler:
-        t0.record(step.stream)
-        for i in range(args.steps):
-            run_step(args.warmup + i)
-        t1.record(step.stream)
-        torch.cuda.synchronize()
-    barrier()
-    elapsed_ms = t0.elapsed_time(t1)
-    # the same K steps on one buffer set, so that each step finds its inputs in L2
-    # (reported as hot_l2, for comparison only)
-    h0 = torch.cuda.Event(enable_timing=True)
-    h1 = torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    h0.record(step.stream)
-    for i in range(args.steps):
-        run_step(0)
-    h1.record(step.stream)
-    torch.cuda.synchronize()
-    barrier()
-    hot_ms = max_over_ranks(h0.elapsed_time(h1), device)
-    # timed region 2: the same K steps with CUDA events around every kernel on its
-    # stream, for the per-kernel durations and the roofline
-    events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nk)]
-              for _ in range(args.steps)]
-    barrier()
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        step.run(args.warmup + i, events[i])
-    torch.cuda.synchronize()
-    barrier()
-    per_kernel_ms = {name: [] for name in step.kernel_names}
-    for i in range(args.steps):
-        for n, name in enumerate(step.kernel_names):
-            per_kernel_ms[name].append(events[i][n][0].elapsed_time(events[i][n][1]))
-    status = step.status()
-    if status != 0:
-        raise RuntimeError(f"device status {status:#x} after the timed steps")
-    elapsed_ms = max_over_ranks(elapsed_ms, device)
+        m = measure(w, host, args.steps, args.warmup, args.eager, True, ctx)
+    step, abytes, elapsed_ms, hot_ms = m["step"], m["abytes"], m["elapsed_ms"], m["hot_ms"]
 
     # end to end through the public API: every step copies its inputs in from pinned host
     # memory and its combined output back out. E2E_DEPTH sets of device buffers rotate, so
@@ -601,76 +695,17 @@ def run_ours(args, ws, rank, local):
     # again only after its previous copy-out finished.
     e2e = None
     if not args.no_e2e:
-        pin = {key: torch.from_numpy(v if v.dtype != np.uint16 else v.view(np.int16)).pin_memory()
-               for key, v in host.items()}
-        depth = E2E_DEPTH
-        outs_host = [torch.empty((w.N, w.H), dtype=torch.int16).pin_memory() for _ in range(depth)]
-        h2d_s = torch.cuda.Stream(device)
-        d2h_s = torch.cuda.Stream(device)
-        comp_s = torch.cuda.Stream(device)
-        pipes = []
-        with torch.cuda.stream(comp_s):
-            for b in range(depth):
-                dset = {key: torch.empty_like(step.sets[0][key]) for key in pin}
-                pipes.append((EpStep if w.ep else Step)(w, moe, _native, torch, [dset], device))
-        views = [{key: (q.sets[0][key].view(torch.int16) if q.sets[0][key].dtype == torch.bfloat16
-                        else q.sets[0][key]) for key in pin} for q in pipes]
-        h2d = sum(t.numel() * t.element_size() for t in pin.values())
-        d2h = outs_host[0].numel() * outs_host[0].element_size()
-        ev = lambda: torch.cuda.Event()  # noqa: E731
-        in_done, comp_done, out_done = ([ev() for _ in range(depth)] for _ in range(3))
-        started = [False] * depth
+        e2e = measure_e2e(w, host, step, args, ws, ctx)
 
-        def e2e_step(i):
-            b = i % depth
-            if started[b]:
-                h2d_s.wait_event(comp_done[b])  # the kernels of step i-2 finished reading these inputs
-            with torch.cuda.stream(h2d_s):
-                for key in pin:
-                    views[b][key].copy_(pin[key], non_blocking=True)
-            in_done[b].record(h2d_s)
-            comp_s.wait_event(in_done[b])
-            if started[b]:
-                comp_s.wait_event(out_done[b])  # step i-2's output has left the device
-            pipes[b].run(0)
-            comp_done[b].record(comp_s)
-            d2h_s.wait_event(comp_done[b])
-            with torch.cuda.stream(d2h_s):
-                outs_host[b].copy_(pipes[b].out.view(torch.int16), non_blocking=True)
-            out_done[b].record(d2h_s)
-            started[b] = True
-
-        for i in range(max(2, min(args.warmup, 4))):
-            e2e_step(i)
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        barrier()
-        torch.cuda.synchronize()
-        e0.record(h2d_s)
-        comp_s.wait_event(e0)
-        for i in range(args.steps):
-            e2e_step(i)
-        for b in range(depth):  # the timed region ends when the last output is on the host
-            d2h_s.wait_event(out_done[b])
-        e1.record(d2h_s)
-        torch.cuda.synchronize()
-        barrier()
-        e_ms = max_over_ranks(e0.elapsed_time(e1), device)
-        st = 0
-        for q in pipes:
-            st |= q.status()
-        if st != 0:
-            raise RuntimeError(f"device status {st:#x} after the end-to-end steps")
-        e2e = {
-            "value": round(w.N * args.steps * ws / (e_ms / 1e3), 1),
-            "unit": "tokens/s",
-            "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h,
-            "ms_per_step": round(e_ms / args.steps, 4),
-            "pipelining": f"{depth} device buffer sets; copy-in, kernels and copy-out on three streams",
-        }
-        del pipes
+    # the other surveyed configurations, a short run each (default run only)
+    extra = {}
+    if not args.workload_given and not args.tokens and not args.no_extra:
+        with sampler:
+            for name in EXTRA_WORKLOADS:
+                wx = get_workload(name)
+                mx = measure(wx, rank_inputs(wx, rank), EXTRA_STEPS, EXTRA_WARMUP, args.eager, False, ctx)
+                extra[name] = mx
+                torch.cuda.empty_cache()
 
     if ws > 1:
         tdist.barrier()
@@ -679,23 +714,31 @@ def run_ours(args, ws, rank, local):
         return None
 
     peak, peak_kind = measured_peaks()
-    kernels = {}
-    for name in step.kernel_names:
-        avg_ms = statistics.mean(per_kernel_ms[name])
-        qs = statistics.quantiles(per_kernel_ms[name], n=10) if len(per_kernel_ms[name]) > 1 else [avg_ms] * 9
-        kernels[name] = {
-            "calls_per_step": step.kernel_names.count(name),
-            "us": round(avg_ms * 1e3, 2),
-            "median_us": round(statistics.median(per_kernel_ms[name]) * 1e3, 2),
-            "p10_us": round(qs[0] * 1e3, 2),
-            "p90_us": round(qs[8] * 1e3, 2),
-            "algorithmic_bytes": abytes[name],
-            "gbs": round(abytes[name] / (avg_ms * 1e-3) / 1e9, 1),
-        }
-    dominant = max(step.kernel_names, key=lambda n: kernels[n]["us"])
+    kernels = kernel_table(m, peak)
+    dominant = max(m["step"].kernel_names, key=lambda n: kernels[n]["us"])
     ach = kernels[dominant]["gbs"]
     ms_step = elapsed_ms / args.steps
-    path_bytes = sum(abytes[n] for n in step.kernel_names)
+    path_bytes = sum(abytes[n] for n in m["step"].kernel_names)
+    workloads = {}
+    for name, mx in extra.items():
+        kx = kernel_table(mx, peak)
+        msx = mx["elapsed_ms"] / EXTRA_STEPS
+        bx = sum(mx["abytes"][n] for n in mx["step"].kernel_names)
+        wx = mx["step"].w
+        dom = max(mx["step"].kernel_names, key=lambda n: kx[n]["us"])
+        workloads[name] = {
+            "config": wx.describe(),
+            "steps": EXTRA_STEPS,
+            "warmup": EXTRA_WARMUP,
+            "ms_per_step": round(msx, 4),
+            "tokens_per_s": round(wx.N * EXTRA_STEPS * ws / (mx["elapsed_ms"] / 1e3), 1),
+            "effective_gbs": round(bx / (msx * 1e-3) / 1e9, 1),
+            "effective_hbm_frac": round(bx / (msx * 1e-3) / 1e9 / peak, 3),
+            "dominant": dom,
+            "kernels": kx,
+            "l2": f"inputs rotated over {mx['nsets']} buffer sets ({mx['nsets'] * mx['set_bytes'] / 2**20:.0f} MiB)",
+            "launch": mx["launch_mode"],
+        }
     result = {
         "metric": METRIC,
         "value": round(w.N * args.steps * ws / (elapsed_ms / 1e3), 1),
@@ -714,8 +757,10 @@ def run_ours(args, ws, rank, local):
             **w.describe(),
             "parallelism": f"dp{ws}: independent batch per GPU, no collective on the data path",
             "step": "+".join(dict.fromkeys(
-                f"{n}x{step.kernel_names.count(n)}" if step.kernel_names.count(n) > 1 else n for n in step.kernel_names)),
-            "l2": f"inputs rotated over {nsets} buffer sets ({nsets * set_bytes / 2**20:.0f} MiB > 126 MB L2), no flush",
+                f"{n}x{m['step'].kernel_names.count(n)}" if m["step"].kernel_names.count(n) > 1 else n
+                for n in m["step"].kernel_names)),
+            "l2": f"inputs rotated over {m['nsets']} buffer sets ({m['nsets'] * m['set_bytes'] / 2**20:.0f} MiB "
+                  f"> 126 MB L2), no flush",
         },
         "effective_gbs": round(path_bytes / (ms_step * 1e-3) / 1e9, 1),
         "effective_hbm_frac": round(path_bytes / (ms_step * 1e-3) / 1e9 / peak, 3),
@@ -730,20 +775,97 @@ def run_ours(args, ws, rank, local):
             "frac": round(ach / peak, 3),
             "traffic": stored_traffic(dominant, w.name),
         },
-        "gpu_launches": args.steps * sum(KERNELS_PER_CALL.get(n, 1) for n in step.kernel_names),
+        "gpu_launches": args.steps * sum(kernels_per_call(n) for n in m["step"].kernel_names),
         "kernel_timing": "per-kernel CUDA events in a second pass of the same K steps (launched eagerly)",
-        "launch": launch_mode,
+        "launch": m["launch_mode"],
         "hot_l2": {
             "ms_per_step": round(hot_ms / args.steps, 4),
             "value": round(w.N * args.steps * ws / (hot_ms / 1e3), 1),
             "note": "the same K steps on one input set (inputs resident in L2); not the headline",
         },
-        "clocks": sampler.summary(),
+        "clocks": sampler.summary(m["timed_window"]),
         "e2e": e2e,
     }
+    if workloads:
+        result["workloads"] = workloads
     if not args.no_cpu_baseline and ws == 1:
         result["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
     return result
+
+
+def measure_e2e(w, host, step, args, ws, ctx):
+    """The headline metric end to end through the binding, host copies inside the timed region."""
+    torch, moe, _native, device, barrier = ctx["torch"], ctx["moe"], ctx["native"], ctx["device"], ctx["barrier"]
+    pin = {key: torch.from_numpy(v if v.dtype != np.uint16 else v.view(np.int16)).pin_memory()
+           for key, v in host.items()}
+    depth = E2E_DEPTH
+    outs_host = [torch.empty((w.N, w.H), dtype=torch.int16).pin_memory() for _ in range(depth)]
+    h2d_s = torch.cuda.Stream(device)
+    d2h_s = torch.cuda.Stream(device)
+    comp_s = torch.cuda.Stream(device)
+    pipes = []
+    with torch.cuda.stream(comp_s):
+        for b in range(depth):
+            dset = {key: torch.empty_like(step.sets[0][key]) for key in pin}
+            pipes.append(EpStep(w, moe, _native, torch, [dset], device) if w.ep else
+                         Step(w, moe, _native, torch, [dset], device, unfused=ctx.get("unfused", False)))
+    views = [{key: (q.sets[0][key].view(torch.int16) if q.sets[0][key].dtype == torch.bfloat16
+                    else q.sets[0][key]) for key in pin} for q in pipes]
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = outs_host[0].numel() * outs_host[0].element_size()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_done, comp_done, out_done = ([ev() for _ in range(depth)] for _ in range(3))
+    started = [False] * depth
+
+    def e2e_step(i):
+        b = i % depth
+        if started[b]:
+            h2d_s.wait_event(comp_done[b])  # the kernels of step i-depth finished reading these inputs
+        with torch.cuda.stream(h2d_s):
+            for key in pin:
+                views[b][key].copy_(pin[key], non_blocking=True)
+        in_done[b].record(h2d_s)
+        comp_s.wait_event(in_done[b])
+        if started[b]:
+            comp_s.wait_event(out_done[b])  # step i-depth's output has left the device
+        pipes[b].run(0)
+        comp_done[b].record(comp_s)
+        d2h_s.wait_event(comp_done[b])
+        with torch.cuda.stream(d2h_s):
+            outs_host[b].copy_(pipes[b].out.view(torch.int16), non_blocking=True)
+        out_done[b].record(d2h_s)
+        started[b] = True
+
+    for i in range(max(2, min(args.warmup, 4))):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(h2d_s)
+    comp_s.wait_event(e0)
+    for i in range(args.steps):
+        e2e_step(i)
+    for b in range(depth):  # the timed region ends when the last output is on the host
+        d2h_s.wait_event(out_done[b])
+    e1.record(d2h_s)
+    torch.cuda.synchronize()
+    barrier()
+    e_ms = max_over_ranks(e0.elapsed_time(e1), device)
+    st = 0
+    for q in pipes:
+        st |= q.status()
+    if st != 0:
+        raise RuntimeError(f"device status {st:#x} after the end-to-end steps")
+    return {
+        "value": round(w.N * args.steps * ws / (e_ms / 1e3), 1),
+        "unit": "tokens/s",
+        "h2d_bytes_per_step": h2d,
+        "d2h_bytes_per_step": d2h,
+        "ms_per_step": round(e_ms / args.steps, 4),
+        "pipelining": f"{depth} device buffer sets; copy-in, kernels and copy-out on three streams",
+    }
 
 
 # --------------------------------------------------------- CPU (oracle) arm
@@ -788,27 +910,60 @@ def sample_workload(w, target_s, oracle):
     return ws, make_inputs(ws, grad=w.backward)
 
 
+def oracle_step_all_cores(oracle, w, d):
+    """The path on every host core: route, permute and combine split over tokens with OpenMP
+    (the unchanged oracle functions on each chunk), the layout serial as defined."""
+    idx, probs = oracle.omp_route_topk(d["logits"], w.k)
+    L = oracle.layout(idx, probs, E_log=w.E_log, R=w.R, C=w.capacity, num_replicas=w.num_replicas,
+                      align=w.row_align, local_topk=True)
+    send = oracle.omp_permute(d["hidden"], L["dest_row"], L["rows_max"])
+    return oracle.omp_combine(send, L["dest_row"], probs)
+
+
+def _timed_median(fn, budget_s):
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while time.perf_counter() < t_end or len(times) < 3:
+        t = time.perf_counter()
+        fn()
+        times.append(time.perf_counter() - t)
+    return statistics.median(times), len(times)
+
+
 def cpu_baseline(w, budget_s=10.0):
+    """The oracle timed on this host: single-threaded as it stands (the headline baseline), and the
+    all-cores variant (OpenMP over tokens for route, permute and combine; the layout serial)."""
     import oracle
 
     oracle.build()
     ws, d = sample_workload(w, min(2.0, budget_s / 5), oracle)
-    times = []
-    t_end = time.perf_counter() + budget_s
-    while time.perf_counter() < t_end or not times:
-        t = time.perf_counter()
-        oracle_step(oracle, ws, d)
-        times.append(time.perf_counter() - t)
-    med = statistics.median(times)
-    return {
+    med, runs = _timed_median(lambda: oracle_step(oracle, ws, d), budget_s)
+    out = {
         "value": round(ws.N / med, 1),
         "unit": "tokens/s",
         "cores": 1,
         "kind": "oracle",
         "sample": f"first {ws.N} of {w.N} tokens of '{w.name}' (same H/E/k/R), whole path per run, "
-                  f"median of {len(times)} runs, single-threaded C oracle",
+                  f"median of {runs} runs, single-threaded C oracle",
         "host_cpus": os.cpu_count(),
     }
+    if not w.tp_size > 1 and not w.dedup and not w.ep and not w.backward:
+        try:
+            oracle.build_omp()
+            threads = oracle.omp_threads()
+            wa = w if w.N <= 4 * ws.N * threads else w.scaled(min(w.N, 4 * ws.N * threads))
+            da = d if wa.N == ws.N else make_inputs(wa)
+            med_a, runs_a = _timed_median(lambda: oracle_step_all_cores(oracle, wa, da), budget_s / 2)
+            out["all_cores"] = {
+                "value": round(wa.N / med_a, 1),
+                "unit": "tokens/s",
+                "cores": threads,
+                "kind": "oracle, OpenMP over tokens (route, permute, combine); layout serial",
+                "sample": f"first {wa.N} of {w.N} tokens of '{w.name}', whole path per run, median of {runs_a} runs",
+            }
+        except Exception as exc:  # no OpenMP toolchain on this host: the single-threaded figure stands
+            out["all_cores"] = {"unavailable": f"{type(exc).__name__}: {exc}"[:200]}
+    return out
 
 
 def run_reference(args, ws, rank):
@@ -915,8 +1070,13 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="ht",
-                    help="tiny | ht | qwen3 | capacity | ultraep | ht_align16 | ht_tp2 | ht_dedup")
+    ap.add_argument("--workload", default=None,
+                    help="tiny | ht | qwen3 | capacity | ultraep | ht_align16 | ht_tp2 | ht_dedup | ht_ep4 "
+                         "(default: ht as the headline, with tiny, qwen3, capacity and ultraep timed beside it)")
+    ap.add_argument("--unfused", action="store_true",
+                    help="call moe_dispatch_layout and moe_permute separately instead of the fused moe_dispatch")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only the headline workload (skip the other surveyed configurations)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--tokens", type=int, default=0, help="run the workload with this many tokens (profiling)")
@@ -927,6 +1087,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
+    args.workload_given = args.workload is not None
+    if args.workload is None:
+        args.workload = "ht"
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     ws, rank, local = dist_env()

@@ -6,6 +6,7 @@ functions keep the C names:
 
     moe_route_topk        router softmax + top-k
     moe_dispatch_layout   reroute, histogram, ordinals, capacity, scan, splits, row maps
+    moe_dispatch          the layout and the permute in one call (the permute fused into the layout's fill)
     moe_permute           send[dest_row[t, j]] = hidden[t]
     moe_combine           out[t] = bf16(sum_j p[t, j] * y[dest_row[t, j]]), fp32, ascending j
     moe_restore_combined  the same over the buffers of TP peers (after TP folding)
@@ -34,7 +35,7 @@ from ._native import (
     MOE_DEV_ROW_RANGE,
     MOE_DEV_TIMEOUT,
     MOE_FLAG_NONE,
-    MOE_FLAG_TEST_BARRIER_TIMEOUT,
+    MOE_FLAG_TEST_WAIT_TIMEOUT,
 )
 
 COUNTER_NAMES = (
@@ -56,6 +57,7 @@ __all__ = [
     "moe_route_topk",
     "moe_dispatch_layout",
     "moe_dispatch_layout_noalloc",
+    "moe_dispatch",
     "moe_permute",
     "moe_combine",
     "moe_restore_combined",
@@ -79,7 +81,7 @@ __all__ = [
     "MOE_DEV_ROW_RANGE",
     "MOE_DEV_TIMEOUT",
     "MOE_FLAG_NONE",
-    "MOE_FLAG_TEST_BARRIER_TIMEOUT",
+    "MOE_FLAG_TEST_WAIT_TIMEOUT",
 ]
 
 
@@ -192,6 +194,8 @@ class Layout:
     problem: Problem
     tensors: Dict[str, torch.Tensor] = field(default_factory=dict)
     workspace: Optional[torch.Tensor] = None
+    _pinned: Optional[Dict[str, torch.Tensor]] = field(default=None, repr=False)
+    _pinned_done: Optional["torch.cuda.Event"] = field(default=None, repr=False)
 
     @classmethod
     def allocate(cls, problem: Problem, device=None, local_topk: bool = True) -> "Layout":
@@ -246,27 +250,26 @@ class Layout:
     def clear_status(self) -> None:
         self.tensors["status"].zero_()
 
-    def reset_workspace(self) -> None:
-        """Zero the layout workspace (needed again only after a MOE_DEV_TIMEOUT)."""
-        self.workspace.zero_()
-
     def prefetch_counts(self, stream=None) -> "CountsPrefetch":
         """Copy the per-expert and per-rank counts to pinned host memory without waiting.
 
         The copies are enqueued after the work already on ``stream`` (the layout call),
         so the host can read them later, off the critical path, instead of forcing a
-        synchronisation when it needs them (Megatron MORI: deferred count reads)."""
+        synchronisation when it needs them (Megatron MORI: deferred count reads). The
+        pinned buffers are allocated on the first call and reused by every later one,
+        so later calls allocate nothing (a pinned allocation can synchronise the
+        device). Each call overwrites what the previous one copied."""
         st = torch.cuda.current_stream(self.device) if stream is None else stream
         keys = ("tokens_per_expert", "expert_offsets", "input_splits", "output_splits", "num_rows", "counters")
-        host = {}
+        if self._pinned is None:
+            self._pinned = {key: torch.empty(self.tensors[key].shape, dtype=self.tensors[key].dtype,
+                                             pin_memory=True) for key in keys}
+            self._pinned_done = torch.cuda.Event()
         with torch.cuda.stream(st):
             for key in keys:
-                buf = torch.empty(self.tensors[key].shape, dtype=self.tensors[key].dtype, pin_memory=True)
-                buf.copy_(self.tensors[key], non_blocking=True)
-                host[key] = buf
-            done = torch.cuda.Event()
-            done.record(st)
-        return CountsPrefetch(host=host, event=done)
+                self._pinned[key].copy_(self.tensors[key], non_blocking=True)
+            self._pinned_done.record(st)
+        return CountsPrefetch(host=self._pinned, event=self._pinned_done)
 
     def counters(self) -> Dict[str, int]:
         """dispatch_counters as a dict. Synchronises."""
@@ -418,7 +421,7 @@ def moe_route_topk(logits: torch.Tensor, k: int, token_mask: Optional[torch.Tens
 
 def moe_dispatch_layout(problem: Problem, topk_idx: torch.Tensor, topk_probs: Optional[torch.Tensor],
                         layout: Optional[Layout] = None, stream=None) -> Layout:
-    """Every dispatch-layout output in one launch; returns the (reusable) Layout."""
+    """Every dispatch-layout output (a count pass and a fill pass); returns the (reusable) Layout."""
     _need(topk_idx, "topk_idx", torch.int32, (problem.N, problem.k))
     if topk_probs is not None:
         _need(topk_probs, "topk_probs", torch.float32, (problem.N, problem.k), topk_idx.device)
@@ -432,6 +435,31 @@ def moe_dispatch_layout(problem: Problem, topk_idx: torch.Tensor, topk_probs: Op
                                            _ptr(layout.workspace), layout.workspace.numel(), _stream(stream))
     _native.check("moe_dispatch_layout", rc)
     return layout
+
+
+def moe_dispatch(problem: Problem, topk_idx: torch.Tensor, topk_probs: Optional[torch.Tensor], hidden: torch.Tensor,
+                 layout: Optional[Layout] = None, send: Optional[torch.Tensor] = None, stream=None):
+    """Dispatch layout and permute in one call; returns (layout, send).
+
+    Equals moe_dispatch_layout followed by moe_permute, bit for bit."""
+    _need(topk_idx, "topk_idx", torch.int32, (problem.N, problem.k))
+    if topk_probs is not None:
+        _need(topk_probs, "topk_probs", torch.float32, (problem.N, problem.k), topk_idx.device)
+    _need(hidden, "hidden", torch.bfloat16, (problem.N, problem.H), topk_idx.device)
+    if layout is None:
+        layout = Layout.allocate(problem, topk_idx.device)
+    elif layout.problem != problem:
+        raise ValueError("layout was allocated for a different problem")
+    if send is None:
+        send = torch.empty((problem.rows_max, problem.H), dtype=torch.bfloat16, device=topk_idx.device)
+    _need(send, "send", torch.bfloat16, (problem.rows_max, problem.H), topk_idx.device)
+    p = problem.c_struct()
+    L = layout.c_struct()
+    rc = _native.lib().moe_dispatch(ctypes.byref(p), _ptr(topk_idx), _ptr(topk_probs), ctypes.byref(L),
+                                    _ptr(layout.workspace), layout.workspace.numel(), _ptr(hidden), _ptr(send),
+                                    _stream(stream))
+    _native.check("moe_dispatch", rc)
+    return layout, send
 
 
 def moe_dispatch_layout_noalloc(problem: Problem, topk_idx: torch.Tensor, topk_probs: Optional[torch.Tensor],

@@ -31,9 +31,9 @@ MOE_DEV_TIMEOUT = 0x2
 MOE_DEV_ROW_RANGE = 0x4
 
 MOE_FLAG_NONE = 0
-MOE_FLAG_TEST_BARRIER_TIMEOUT = 0x80000000
+MOE_FLAG_TEST_WAIT_TIMEOUT = 0x80000000
 
-ABI_VERSION = 5
+ABI_VERSION = 6
 
 
 class MoeProblem(ctypes.Structure):
@@ -122,6 +122,7 @@ _SIGNATURES = {
     "moe_route_topk": (ctypes.c_int, [_VP, _VP, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _VP, _VP, _VP]),
     "moe_dispatch_layout": (ctypes.c_int, [_PP, _VP, _VP, _PL, _VP, ctypes.c_size_t, _VP]),
     "moe_dispatch_layout_noalloc": (ctypes.c_int, [_PP, _VP, _VP, _PL, _VP]),
+    "moe_dispatch": (ctypes.c_int, [_PP, _VP, _VP, _PL, _VP, ctypes.c_size_t, _VP, _VP, _VP]),
     "moe_permute": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP]),
     "moe_combine": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP]),
     "moe_restore_combined": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP]),

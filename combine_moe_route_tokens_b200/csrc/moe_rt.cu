@@ -22,6 +22,7 @@
 #include "ptx.cuh"
 #include "route.cuh"
 #include "layout.cuh"
+#include "dispatch.cuh"
 #include "permute.cuh"
 #include "combine.cuh"
 #include "dedup.cuh"
@@ -32,25 +33,41 @@ namespace {
 using namespace moert;
 
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;     // 1 s: every device-side wait gives up after this
-constexpr uint64_t TEST_WAIT_LIMIT_NS = 10000000ull;  // 10 ms for MOE_FLAG_TEST_BARRIER_TIMEOUT
-constexpr size_t WS_BARRIER_BYTES = 256;
+constexpr uint64_t TEST_WAIT_LIMIT_NS = 10000000ull;  // 10 ms for MOE_FLAG_TEST_WAIT_TIMEOUT
+constexpr size_t WS_BARRIER_BYTES = 256;  // dedup layout: grid barrier words
+constexpr size_t WS_TICKET_BYTES = 256;   // dispatch layout: the ticket word, then the look-back words
 
 using LayoutKernel = void (*)(LayoutArgs);
+using DispatchKernel = void (*)(DispatchArgs);
 
-LayoutKernel layout_kernel_for(int ipl)
+LayoutKernel layout_count_for(int ipl)
 {
     switch (ipl) {
     case 1:
-        return layout_kernel<1>;
+        return layout_count_kernel<1>;
     case 2:
-        return layout_kernel<2>;
+        return layout_count_kernel<2>;
     case 4:
-        return layout_kernel<4>;
+        return layout_count_kernel<4>;
     case 8:
-        return layout_kernel<8>;
+        return layout_count_kernel<8>;
     default:
-        return layout_kernel<0>;
+        return layout_count_kernel<0>;
     }
+}
+
+LayoutKernel layout_fill_for(bool reroute, bool dense)
+{
+    if (reroute)
+        return dense ? layout_fill_kernel<true, true> : layout_fill_kernel<true, false>;
+    return dense ? layout_fill_kernel<false, true> : layout_fill_kernel<false, false>;
+}
+
+DispatchKernel dispatch_for(bool reroute, bool dense)
+{
+    if (reroute)
+        return dense ? dispatch_kernel<true, true> : dispatch_kernel<true, false>;
+    return dense ? dispatch_kernel<false, true> : dispatch_kernel<false, false>;
 }
 
 constexpr int LAYOUT_IPLS[] = {0, 1, 2, 4, 8};
@@ -138,6 +155,7 @@ struct DeviceInfo {
     int sms = 0;
     int smem_optin = 0;
     int layout_dyn_max = 0; // dynamic shared memory the layout kernels may take (opt-in limit less their static part)
+    int tables_dyn_max = 0; // the same for the fill and fused dispatch kernels
     bool ready = false;
 };
 
@@ -161,15 +179,41 @@ int device_info(DeviceInfo *out)
         for (int ipl : LAYOUT_IPLS) {
             cudaFuncAttributes fa;
             if (e == cudaSuccess)
-                e = cudaFuncGetAttributes(&fa, layout_kernel_for(ipl));
+                e = cudaFuncGetAttributes(&fa, layout_count_for(ipl));
             if (e == cudaSuccess && static_cast<int>(fa.sharedSizeBytes) > static_max)
                 static_max = static_cast<int>(fa.sharedSizeBytes);
         }
         d.layout_dyn_max = d.smem_optin - static_max;
         for (int ipl : LAYOUT_IPLS)
             if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(layout_kernel_for(ipl), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                e = cudaFuncSetAttribute(layout_count_for(ipl), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          d.layout_dyn_max);
+        // the second pass's per-CTA tables (at most ~57 KB for E_log = 2048 with as many replicas)
+        int static2 = 0;
+        for (int rr = 0; rr < 2; ++rr)
+            for (int dn = 0; dn < 2; ++dn) {
+                cudaFuncAttributes fa1, fa2;
+                if (e == cudaSuccess)
+                    e = cudaFuncGetAttributes(&fa1, layout_fill_for(rr != 0, dn != 0));
+                if (e == cudaSuccess)
+                    e = cudaFuncGetAttributes(&fa2, dispatch_for(rr != 0, dn != 0));
+                if (e == cudaSuccess) {
+                    static2 = static_cast<int>(fa1.sharedSizeBytes) > static2 ? static_cast<int>(fa1.sharedSizeBytes)
+                                                                             : static2;
+                    static2 = static_cast<int>(fa2.sharedSizeBytes) > static2 ? static_cast<int>(fa2.sharedSizeBytes)
+                                                                             : static2;
+                }
+            }
+        d.tables_dyn_max = d.smem_optin - static2;
+        for (int rr = 0; rr < 2; ++rr)
+            for (int dn = 0; dn < 2; ++dn) {
+                if (e == cudaSuccess)
+                    e = cudaFuncSetAttribute(layout_fill_for(rr != 0, dn != 0),
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, d.tables_dyn_max);
+                if (e == cudaSuccess)
+                    e = cudaFuncSetAttribute(dispatch_for(rr != 0, dn != 0),
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, d.tables_dyn_max);
+            }
         if (e != cudaSuccess || d.layout_dyn_max <= 0)
             return MOE_ERR_CUDA;
         d.ready = true;
@@ -199,7 +243,7 @@ int check_problem(const moe_problem_t *p, Dims *d)
         return MOE_ERR_INVALID;
     if (p->E_log % p->R != 0 || p->num_replicas % p->R != 0 || p->num_replicas > p->E_log)
         return MOE_ERR_INVALID;
-    if ((p->flags & ~MOE_FLAG_TEST_BARRIER_TIMEOUT) != 0)
+    if ((p->flags & ~MOE_FLAG_TEST_WAIT_TIMEOUT) != 0)
         return MOE_ERR_INVALID;
     if (p->row_align < 0 || p->tp_size < 0 || p->tp_rank < 0)
         return MOE_ERR_INVALID;
@@ -249,30 +293,31 @@ int check_layout(const moe_layout_t *l, const Dims &d, bool need_rows)
 }
 
 struct LayoutGrid {
-    int32_t G;   // blocks
+    int32_t G;   // count blocks
     int32_t sub; // assignments per warp slice
     int32_t ipl; // assignments per lane kept in registers (1, 2, 4, 8), or 0 for longer slices
 };
 
-// About LAYOUT_ITEMS_PER_BLOCK assignments per block, at most LAYOUT_MAX_BLOCKS
-// blocks; slices of up to 8 items per lane stay in registers.
+// The fewest ids per lane (1, 2, 4 or 8, in registers) that keep the count grid
+// at LAYOUT_TARGET_BLOCKS blocks or fewer, so the look-back ends in one round;
+// larger problems take 8 per lane on up to LAYOUT_MAX_BLOCKS blocks, and beyond
+// that longer slices that are read twice.
 LayoutGrid layout_grid(int64_t NK)
 {
-    int64_t G = (NK + LAYOUT_ITEMS_PER_BLOCK - 1) / LAYOUT_ITEMS_PER_BLOCK;
-    G = G < 1 ? 1 : (G > LAYOUT_MAX_BLOCKS ? LAYOUT_MAX_BLOCKS : G);
-    int64_t ipl = (NK + G * LAYOUT_THREADS - 1) / (G * LAYOUT_THREADS);
-    if (ipl < 1)
-        ipl = 1;
-    int32_t kind = 0;
-    if (ipl <= LAYOUT_MAX_IPL) {
-        int64_t p2 = 1;
-        while (p2 < ipl)
-            p2 <<= 1;
-        ipl = p2;
-        kind = static_cast<int32_t>(ipl);
+    const int64_t per_block_ipl1 = static_cast<int64_t>(LAYOUT_THREADS);
+    int64_t ipl = 1;
+    while (ipl < LAYOUT_MAX_IPL && (NK + per_block_ipl1 * ipl - 1) / (per_block_ipl1 * ipl) > LAYOUT_TARGET_BLOCKS)
+        ipl <<= 1;
+    int64_t G = (NK + per_block_ipl1 * ipl - 1) / (per_block_ipl1 * ipl);
+    int32_t kind = static_cast<int32_t>(ipl);
+    int64_t sub = 32 * ipl;
+    if (G > LAYOUT_MAX_BLOCKS) { // slices longer than the registers hold
+        kind = 0;
+        const int64_t per_warp = (NK + static_cast<int64_t>(LAYOUT_MAX_BLOCKS) * LAYOUT_WARPS - 1) /
+                                 (static_cast<int64_t>(LAYOUT_MAX_BLOCKS) * LAYOUT_WARPS);
+        sub = ((per_warp + 31) / 32) * 32;
+        G = (NK + LAYOUT_WARPS * sub - 1) / (LAYOUT_WARPS * sub);
     }
-    const int64_t sub = 32 * ipl;
-    G = (NK + LAYOUT_WARPS * sub - 1) / (LAYOUT_WARPS * sub);
     if (G < 1)
         G = 1;
     return {static_cast<int32_t>(G), static_cast<int32_t>(sub), kind};
@@ -280,7 +325,7 @@ LayoutGrid layout_grid(int64_t NK)
 
 size_t layout_workspace_bytes(int32_t E_log)
 {
-    return WS_BARRIER_BYTES + static_cast<size_t>(LAYOUT_MAX_BLOCKS) * static_cast<size_t>(E_log) * 4;
+    return WS_TICKET_BYTES + static_cast<size_t>(LAYOUT_MAX_BLOCKS) * static_cast<size_t>(E_log) * 8;
 }
 
 } // namespace
@@ -367,11 +412,16 @@ int moe_route_topk(const float *logits, const uint8_t *token_mask, int64_t N, in
     return go(route_topk_kernel<32>);
 }
 
-int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, const float *topk_probs,
-                        const moe_layout_t *layout, void *workspace, size_t workspace_bytes, void *stream)
+} // extern "C"
+
+namespace {
+
+// Host checks and arguments of the dispatch layout, shared by moe_dispatch_layout
+// and moe_dispatch; nothing is enqueued.
+int prepare_layout(const moe_problem_t *problem, const int32_t *topk_idx, const float *topk_probs,
+                   const moe_layout_t *layout, void *workspace, size_t workspace_bytes, Dims &d, DeviceInfo &dev,
+                   LayoutGrid &lg, LayoutArgs &a)
 {
-    NvtxRange nvtx_range("moe_dispatch_layout");
-    Dims d;
     int rc = check_problem(problem, &d);
     if (rc != MOE_OK)
         return rc;
@@ -390,17 +440,12 @@ int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, c
     if (workspace == nullptr || workspace_bytes < layout_workspace_bytes(problem->E_log) ||
         (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return MOE_ERR_INVALID;
-    DeviceInfo dev;
     if ((rc = device_info(&dev)) != MOE_OK)
         return rc;
-    const LayoutGrid lg = layout_grid(d.NK);
-    if (lg.G > dev.sms)
+    lg = layout_grid(d.NK);
+    if (layout_count_smem_words(problem->E_log) * 4 > static_cast<size_t>(dev.layout_dyn_max) ||
+        layout_tables_smem_words(problem->E_log, d.E) * 4 > static_cast<size_t>(dev.tables_dyn_max))
         return MOE_ERR_UNSUPPORTED;
-    const size_t smem = layout_smem_words(problem->E_log, d.E) * 4;
-    if (smem > static_cast<size_t>(dev.layout_dyn_max))
-        return MOE_ERR_UNSUPPORTED;
-
-    LayoutArgs a;
     a.topk_idx = topk_idx;
     a.topk_probs = topk_probs;
     a.NK = d.NK;
@@ -420,14 +465,80 @@ int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, c
     a.C_local = d.C_local;
     a.sub = lg.sub;
     a.G = lg.G;
-    a.ws_barrier = static_cast<uint32_t *>(workspace);
-    a.ws_counts = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + WS_BARRIER_BYTES);
-    const bool test_timeout = (problem->flags & MOE_FLAG_TEST_BARRIER_TIMEOUT) != 0;
-    a.barrier_limit_ns = test_timeout ? TEST_WAIT_LIMIT_NS : WAIT_LIMIT_NS;
-    a.barrier_extra = test_timeout ? 1u : 0u;
+    a.ws_ticket = static_cast<unsigned long long *>(workspace);
+    a.ws_flags = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(workspace) + WS_TICKET_BYTES);
+    const bool test_timeout = (problem->flags & MOE_FLAG_TEST_WAIT_TIMEOUT) != 0;
+    a.wait_limit_ns = test_timeout ? TEST_WAIT_LIMIT_NS : WAIT_LIMIT_NS;
+    a.test_stall = test_timeout ? 1u : 0u;
     a.out = *l;
+    return MOE_OK;
+}
 
-    return launch(layout_kernel_for(lg.ipl), dim3(lg.G), dim3(LAYOUT_THREADS), smem, stream, true, a);
+} // namespace
+
+extern "C" {
+
+int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, const float *topk_probs,
+                        const moe_layout_t *layout, void *workspace, size_t workspace_bytes, void *stream)
+{
+    NvtxRange nvtx_range("moe_dispatch_layout");
+    Dims d;
+    DeviceInfo dev;
+    LayoutGrid lg;
+    LayoutArgs a;
+    int rc = prepare_layout(problem, topk_idx, topk_probs, layout, workspace, workspace_bytes, d, dev, lg, a);
+    if (rc != MOE_OK)
+        return rc;
+    const int64_t fill_items = d.NK > d.rows_max ? d.NK : d.rows_max;
+    const int64_t fill_blocks = fill_items > 0 ? (fill_items + FILL_THREADS - 1) / FILL_THREADS : 1;
+    if (fill_blocks > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    const bool reroute = problem->num_replicas > 0;
+    const bool dense = problem->capacity == 0 && d.A == 1;
+    rc = launch(layout_count_for(lg.ipl), dim3(lg.G), dim3(LAYOUT_THREADS), layout_count_smem_words(a.E_log) * 4,
+                stream, false, a);
+    if (rc != MOE_OK)
+        return rc;
+    return launch(layout_fill_for(reroute, dense), dim3(static_cast<unsigned>(fill_blocks)), dim3(FILL_THREADS),
+                  layout_tables_smem_words(a.E_log, a.E) * 4, stream, false, a);
+}
+
+int moe_dispatch(const moe_problem_t *problem, const int32_t *topk_idx, const float *topk_probs,
+                 const moe_layout_t *layout, void *workspace, size_t workspace_bytes, const uint16_t *hidden,
+                 uint16_t *send, void *stream)
+{
+    NvtxRange nvtx_range("moe_dispatch");
+    Dims d;
+    DeviceInfo dev;
+    LayoutGrid lg;
+    DispatchArgs da;
+    int rc = prepare_layout(problem, topk_idx, topk_probs, layout, workspace, workspace_bytes, d, dev, lg, da.L);
+    if (rc != MOE_OK)
+        return rc;
+    if ((problem->N > 0 && (hidden == nullptr || !aligned16(hidden))) ||
+        (d.rows_max > 0 && (send == nullptr || !aligned16(send))))
+        return MOE_ERR_INVALID;
+    da.hidden = reinterpret_cast<const uint4 *>(hidden);
+    da.send = reinterpret_cast<uint4 *>(send);
+    da.N = problem->N;
+    da.V = problem->H / 8;
+    da.group = da.V <= 32 * PERMUTE_CHUNKS ? 32 : (da.V <= 64 * PERMUTE_CHUNKS ? 64 : PERMUTE_THREADS);
+    da.pieces = (da.V + da.group * PERMUTE_CHUNKS - 1) / (da.group * PERMUTE_CHUNKS);
+    // row CTAs: one thread per row per pass, at most four CTAs per SM; CTA 0 writes the tables
+    const int64_t rb = (d.rows_max + PERMUTE_THREADS - 1) / PERMUTE_THREADS;
+    da.row_ctas = static_cast<int32_t>(rb < 1 ? 1 : (rb < 4 * dev.sms ? rb : 4 * dev.sms));
+    const int64_t groups = PERMUTE_THREADS / da.group;
+    const int64_t blocks = da.row_ctas + (problem->N * da.pieces + groups - 1) / groups;
+    if (blocks > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    const bool reroute = problem->num_replicas > 0;
+    const bool dense = problem->capacity == 0 && d.A == 1;
+    rc = launch(layout_count_for(lg.ipl), dim3(lg.G), dim3(LAYOUT_THREADS),
+                layout_count_smem_words(problem->E_log) * 4, stream, false, da.L);
+    if (rc != MOE_OK)
+        return rc;
+    return launch(dispatch_for(reroute, dense), dim3(static_cast<unsigned>(blocks)), dim3(PERMUTE_THREADS),
+                  layout_tables_smem_words(problem->E_log, d.E) * 4, stream, false, da);
 }
 
 int moe_permute(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *hidden, uint16_t *send,
@@ -1126,8 +1237,8 @@ int moe_combine_backward(const moe_problem_t *problem, const moe_layout_t *layou
 namespace {
 
 static_assert(MOE_NOALLOC_SCRATCH_BYTES ==
-                  WS_BARRIER_BYTES + static_cast<size_t>(LAYOUT_MAX_BLOCKS) * MOE_NOALLOC_MAX_E_LOG * 4,
-              "fixed scratch must hold the barrier words and LAYOUT_MAX_BLOCKS rows of per-expert counts");
+                  WS_TICKET_BYTES + static_cast<size_t>(LAYOUT_MAX_BLOCKS) * MOE_NOALLOC_MAX_E_LOG * 8,
+              "fixed scratch must hold the ticket word and LAYOUT_MAX_BLOCKS rows of look-back words");
 
 // Held by every device that loads the library, for the life of the process.
 static __device__ __align__(256) unsigned char g_layout_scratch[MOE_NOALLOC_SCRATCH_BYTES];
@@ -1139,12 +1250,12 @@ struct ScratchAddress {
 ScratchAddress g_scratch_address[MAX_DEVICES];
 std::mutex g_scratch_mutex;
 
-// Device address of g_layout_scratch on the current device, looked up once per
-// device (in host code the symbol is only a stand-in, not a device address).
-int scratch_address(void **out)
+// Device address of g_layout_scratch on device `dev`, looked up once per device
+// with that device current (in host code the symbol is only a stand-in, not a
+// device address).
+int scratch_address(int dev, void **out)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES)
+    if (dev < 0 || dev >= MAX_DEVICES)
         return MOE_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
     ScratchAddress &s = g_scratch_address[dev];
@@ -1186,20 +1297,21 @@ extern "C" int moe_dispatch_layout_noalloc(const moe_problem_t *problem, const i
     if (d.rows_max > 0 && (l->row_token == nullptr || l->row_slot == nullptr || l->row_local_expert == nullptr ||
                            l->row_prob == nullptr || l->pad_mask == nullptr))
         return MOE_ERR_INVALID;
-    DeviceInfo dev;
-    if ((rc = device_info(&dev)) != MOE_OK)
-        return rc;
-    if (layout_grid(d.NK).G > dev.sms)
-        return MOE_ERR_UNSUPPORTED;
-    void *scratch = nullptr;
-    if ((rc = scratch_address(&scratch)) != MOE_OK)
-        return rc;
-    // The grid barrier's arrival count and the error word must start at zero; a
-    // previous call that timed out may have left them set. The per-block counts
-    // are rewritten by every call before they are read.
-    if (cudaMemsetAsync(scratch, 0, WS_BARRIER_BYTES, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    // The scratch must be the array of the device that runs the call: the one that
+    // owns `stream`. Kernels launch on the current device, so the two must agree.
+    int cur = 0, owner = 0;
+    if (cudaGetDevice(&cur) != cudaSuccess || cudaStreamGetDevice(static_cast<cudaStream_t>(stream), &owner) !=
+                                                   cudaSuccess) {
         (void)cudaGetLastError();
         return MOE_ERR_CUDA;
     }
+    if (owner != cur)
+        return MOE_ERR_INVALID;
+    void *scratch = nullptr;
+    if ((rc = scratch_address(cur, &scratch)) != MOE_OK)
+        return rc;
+    // Nothing in the array has to be cleared between calls: every look-back word
+    // carries the epoch of the launch that wrote it, and the ticket word is
+    // rolled over by the last block of each launch (also after a timed-out one).
     return moe_dispatch_layout(problem, topk_idx, topk_probs, layout, scratch, MOE_NOALLOC_SCRATCH_BYTES, stream);
 }

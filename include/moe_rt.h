@@ -24,9 +24,12 @@
  *   full [max_tokens, ...] padded buffers and mask the tail). rows_max =
  *   E*ceil(capacity/T) when capacity > 0, else (N*k + E*(T-1))/T + E*(row_align - 1)
  *   (N*k without alignment or TP folding, T = tp_size). N*k and rows_max must be < 2^31.
- * Returns.  MOE_OK or a negative host-detected error; on error nothing is
- *   enqueued. Device-detected problems are OR-ed into *layout->status as
- *   MOE_DEV_* bits; read them when convenient (no call waits for them).
+ * Returns.  MOE_OK or a negative host-detected error; on MOE_ERR_INVALID,
+ *   MOE_ERR_UNSUPPORTED or MOE_ERR_SCRATCH_LIMIT nothing is enqueued (every
+ *   check comes before the first launch). MOE_ERR_CUDA means a launch failed;
+ *   a call that enqueues two kernels may then have enqueued the first.
+ *   Device-detected problems are OR-ed into *layout->status as MOE_DEV_* bits;
+ *   read them when convenient (no call waits for them).
  * Concurrency.  A layout / workspace pair backs one dispatch at a time
  *   ([Megatron MORI] review thread: one staging region per op means two calls
  *   of the same op must not be in flight together). Reusing the layout for
@@ -43,7 +46,7 @@
 extern "C" {
 #endif
 
-#define MOE_RT_ABI_VERSION 5
+#define MOE_RT_ABI_VERSION 6
 
 /* Every entry point is exported; everything else in the library is hidden. */
 #if defined(__GNUC__)
@@ -66,9 +69,10 @@ extern "C" {
 
 /* moe_problem_t.flags */
 #define MOE_FLAG_NONE 0u
-/* Test hook: the layout's grid barrier waits for one arrival that never comes,
- * with a ~10 ms limit, so the timeout path can be exercised without hanging. */
-#define MOE_FLAG_TEST_BARRIER_TIMEOUT 0x80000000u
+/* Test hook: in the dispatch layout the first block of the scan never publishes
+ * its counts, so the next block's look-back waits for a word that never comes,
+ * with a ~10 ms limit; the timeout path runs without hanging anything. */
+#define MOE_FLAG_TEST_WAIT_TIMEOUT 0x80000000u
 
 /* The problem statement ([DeepSpeed EP] RoutedAssignmentPayload; it follows the
  * pages' shapes: hidden [N,H] bf16, topk ids [N,k] int32, probs [N,k] fp32). */
@@ -147,10 +151,11 @@ MOE_API const char *moe_status_string(int code);
 MOE_API int64_t moe_rows_max(const moe_problem_t *problem);
 
 /*
- * Bytes of device scratch moe_dispatch_layout needs (per-block histograms and
- * a grid barrier). Host only. The scratch must be zero-filled before its first
- * use; afterwards every call leaves it ready for the next one, except a call
- * that reported MOE_DEV_TIMEOUT, after which it must be zero-filled again.
+ * Bytes of device scratch moe_dispatch_layout needs (a ticket word and the
+ * per-block look-back words of the scan). Host only. The scratch must be
+ * zero-filled once before its first use; afterwards every call leaves it ready
+ * for the next one, also a call that reported MOE_DEV_TIMEOUT (each look-back
+ * word carries the epoch of the launch that wrote it).
  * Returns MOE_OK and sets *bytes, or a negative MOE_ERR_*.
  */
 MOE_API int moe_layout_workspace_bytes(const moe_problem_t *problem, size_t *bytes);
@@ -173,7 +178,10 @@ MOE_API int moe_route_topk(const float *logits, const uint8_t *token_mask, int64
 /*
  * Dispatch layout: optional UltraEP reroute, histogram, stable ordinals,
  * capacity drop / pad, exclusive scan, rank splits, row maps and the local
- * view, in one cooperative launch.
+ * view, in two launches: a count pass whose blocks, ordered by an atomic
+ * ticket, scan the per-expert counts with a decoupled look-back (each block
+ * waits only for blocks that started before it, so any number of layouts may
+ * run at once on any streams), and a fill pass for the row maps.
  *   [UltraEP]: hot-expert replicas from the layer's actual load, tokens
  *     rerouted logical -> physical; router semantics stay logical.
  *   [DeepSpeed EP] assignment_ordinals_by_expert: stable ordinals per expert;
@@ -192,12 +200,29 @@ MOE_API int moe_route_topk(const float *logits, const uint8_t *token_mask, int64
  *   layout      every pointer except local_topk must be non-NULL
  *   workspace   moe_layout_workspace_bytes() bytes, zero-filled before first use
  * Limits: E_log <= 2048, k <= 32, R <= 64 when num_replicas > 0.
- * The launch is cooperative (one CTA per SM, up to 128 CTAs): layouts enqueued on
- * several streams at once must together fit the GPU's SMs, else their bounded
- * barrier reports MOE_DEV_TIMEOUT.
+ * The only device-side wait (a block for its predecessors' look-back words) is
+ * bounded by ~1 s; if it runs out, MOE_DEV_TIMEOUT is set and that call's
+ * outputs are invalid (destination rows stay inside [-1, rows_max)).
  */
 MOE_API int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, const float *topk_probs,
                         const moe_layout_t *layout, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Dispatch layout and permute in one call ([Megatron MORI]: the permute is
+ * fused into the dispatch node; [Megatron MoE] dispatch_postprocess: permuted
+ * tokens and tokens_per_expert). Computes exactly the outputs of
+ * moe_dispatch_layout followed by moe_permute (layout and send buffer, bit for
+ * bit) in two launches: the layout's count pass, then one kernel that finishes
+ * the layout and copies every kept token row to its send-buffer rows, zeroing
+ * pad and tail rows. Each token row is read once and can be read while the
+ * count pass runs; nothing passes through an intermediate row map in memory.
+ *   topk_idx, topk_probs, layout, workspace  as for moe_dispatch_layout
+ *   hidden [N, H] bf16; send [rows_max, H] bf16 (16-byte aligned, no overlap)
+ * Same limits as moe_dispatch_layout.
+ */
+MOE_API int moe_dispatch(const moe_problem_t *problem, const int32_t *topk_idx, const float *topk_probs,
+                         const moe_layout_t *layout, void *workspace, size_t workspace_bytes, const uint16_t *hidden,
+                         uint16_t *send, void *stream);
 
 /*
  * Dispatch layout for callers that cannot allocate device memory. The pages
@@ -215,17 +240,21 @@ MOE_API int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *top
  * Limits and rules:
  *  - E_log <= MOE_NOALLOC_MAX_E_LOG, else MOE_ERR_SCRATCH_LIMIT and nothing is enqueued;
  *    every other argument rule of moe_dispatch_layout applies.
+ *  - The current device must be the device that owns `stream` (the array used is
+ *    that device's); a stream of another device gives MOE_ERR_INVALID.
  *  - The first call on a device looks up the array's device address (once per
  *    device, with that device current). Make that first call before any stream
  *    capture begins.
  *  - All calls share the one array and it keeps what the last call left there.
- *    Each call first clears, in stream order, the words that must start at zero,
- *    so a call that ran out of time (MOE_DEV_TIMEOUT) does not affect the next.
+ *    Nothing in it has to start at zero after the first use: the scan's words
+ *    carry the epoch of the launch that wrote them and the ticket word is rolled
+ *    over by every launch, so a call that ran out of time (MOE_DEV_TIMEOUT) does
+ *    not affect the next and the call enqueues nothing but its two kernels.
  *    Calls whose executions overlap on the GPU (for example on two streams)
  *    race on the array and give wrong results: order them on one stream.
  */
 #define MOE_NOALLOC_MAX_E_LOG 512
-#define MOE_NOALLOC_SCRATCH_BYTES (256 + 128 * MOE_NOALLOC_MAX_E_LOG * 4)
+#define MOE_NOALLOC_SCRATCH_BYTES (256 + 128 * MOE_NOALLOC_MAX_E_LOG * 8)
 MOE_API int moe_dispatch_layout_noalloc(const moe_problem_t *problem, const int32_t *topk_idx,
                                         const float *topk_probs, const moe_layout_t *layout, void *stream);
 
@@ -244,7 +273,11 @@ MOE_API int moe_permute(const moe_problem_t *problem, const moe_layout_t *layout
  * top-k slot at a time in ascending slot order; [Megatron MoE] combine):
  *   out[t,h] = bf16_rn( fp32 chain acc = fmaf(p[t,j], y[dest_row[t,j], h], acc)
  *                       over ascending j with dest_row >= 0, from acc = +0 )
- * Deterministic, no atomics, bit-exact with the CPU definition.
+ * Deterministic, no atomics, bit-exact with the CPU definition, except for the
+ * bit pattern of a NaN: a NaN element (from a NaN input or an inf - inf sum) is
+ * a NaN exactly where the definition's is, but it is the canonical bf16 NaN that
+ * the hardware conversion produces, not the sign and payload the CPU definition
+ * keeps. Infinities and signed zeros follow IEEE fp32 and are bit-exact.
  *   expert_out [rows_max, H] bf16; topk_probs [N, k] fp32 or NULL (unit
  *   weights); out [N, H] bf16. Reads layout->dest_row.
  */

@@ -105,7 +105,7 @@ def test_unsupported_problems(lib, kw):
 
 def test_workspace_size(lib):
     p = moe.Problem(N=4096, H=7168, k=8, E_log=256, R=4)
-    assert p.workspace_bytes == 256 + 128 * 256 * 4
+    assert p.workspace_bytes == 256 + 128 * 256 * 8  # ticket word, then 64-bit look-back words per block and expert
 
 
 def test_layout_requires_outputs_and_workspace(lib):

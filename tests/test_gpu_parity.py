@@ -72,6 +72,25 @@ def assert_layout_equal(G, L):
             assert np.array_equal(got.astype(np.int64), exp.astype(np.int64)), key
 
 
+def check_dispatch(p, idx, probs, hidden, L):
+    """The fused dispatch (layout + permute in one call): its layout and its send buffer,
+    written over a canary, equal the oracle's, bit for bit."""
+    canary = torch.tensor(0x7F7F, dtype=torch.int16).view(torch.bfloat16).item()
+    send = torch.full((L["rows_max"], p.H), canary, dtype=torch.bfloat16, device="cuda")
+    G, send = moe.moe_dispatch(p, dev(idx), None if probs is None else dev(probs), dev(hidden), send=send)
+    torch.cuda.synchronize()
+    assert_layout_equal(G, L)
+    assert np.array_equal(host(send), oracle.permute(hidden, L["dest_row"], L["rows_max"]))
+    assert G.status() == 0
+    return G, send
+
+
+@pytest.mark.parametrize("name", WORKLOAD_NAMES)
+def test_dispatch_fused(name):
+    w, d, idx, probs, L = workload_case(name)
+    check_dispatch(problem_of(w), idx, probs, d["hidden"], L)
+
+
 @pytest.mark.parametrize("name", WORKLOAD_NAMES)
 def test_route(name):
     w, d, idx, probs, _ = workload_case(name)
@@ -106,6 +125,30 @@ def test_permute_combine(name):
     out1 = moe.moe_combine(p, G, send, None)
     assert np.array_equal(host(out1), oracle.combine(exp_send, L["dest_row"], None))
     assert G.status() == 0
+
+
+def test_combine_special_values():
+    """NaN, +-inf and signed zeros in the expert outputs: every non-NaN output is bit-exact; a NaN
+    output is NaN on both sides at the same places (the GPU's is the canonical bf16 NaN, the CPU
+    definition keeps sign and payload: the one documented exception to bit-exactness)."""
+    N, H, k, E_log, R = 300, 64, 4, 16, 2
+    idx, probs, hidden = _small_case(N, H, k, E_log, R, seed=21)
+    L = oracle.layout(idx, probs, E_log=E_log, R=R)
+    y = oracle.permute(hidden, L["dest_row"], L["rows_max"])
+    rng = np.random.default_rng(21)
+    specials = np.array([0x7FC0, 0xFFC1, 0x7F81, 0x7F80, 0xFF80, 0x8000, 0x0000], np.uint16)  # NaNs, +-inf, -0, +0
+    mask = rng.random(y.shape) < 0.02
+    y[mask] = specials[rng.integers(0, len(specials), mask.sum())]
+    p = moe.Problem(N=N, H=H, k=k, E_log=E_log, R=R)
+    G = moe.moe_dispatch_layout(p, dev(idx), dev(probs))
+    for pr in (probs, None):
+        got = host(moe.moe_combine(p, G, dev(y), None if pr is None else dev(pr)))
+        want = oracle.combine(y, L["dest_row"], pr)
+        nan_g = ((got & 0x7F80) == 0x7F80) & ((got & 0x7F) != 0)
+        nan_w = ((want & 0x7F80) == 0x7F80) & ((want & 0x7F) != 0)
+        assert nan_g.any() and np.array_equal(nan_g, nan_w)
+        assert np.array_equal(got[~nan_g], want[~nan_w])
+        assert ((want & 0x7F80) == 0x7F80)[~nan_w].any()  # infinities reached the output too
 
 
 @pytest.mark.parametrize("name", WORKLOAD_NAMES)
@@ -216,6 +259,7 @@ def test_edge_cases_full_path(case):
     assert np.allclose(host(gp), exp_gp, rtol=1e-4, atol=1e-4 * np.sqrt(H))
     assert np.array_equal(host(moe.moe_permute_backward(p, G, gy)), oracle.permute_backward(exp_gy, L["dest_row"]))
     assert G.status() == 0
+    check_dispatch(p, idx, probs, hidden, L)
 
 
 @pytest.mark.parametrize("C", [0, 5])
@@ -230,6 +274,7 @@ def test_empty_batch(C):
     assert_layout_equal(G, L)
     assert out.shape == (0, 16) and send.shape == (L["rows_max"], 16)
     assert torch.all(send == 0)
+    check_dispatch(p, np.zeros((0, 2), np.int32), None, np.zeros((0, 16), np.uint16), L)
 
 
 def test_padding_tokens_via_route_mask():
@@ -290,16 +335,21 @@ def test_outputs_stay_inside_their_buffers():
     assert torch.all(send_big[RM:] == 1.5) and torch.all(out_big[600:] == -2.0) and torch.all(gy_big[RM:] == 3.0)
 
 
-def test_barrier_timeout_reports_and_recovers():
-    """The layout's grid barrier gives up after its limit and says so; the context stays usable."""
+def test_lookback_timeout_reports_and_recovers():
+    """The layout's look-back gives up on a word that never comes after its limit and says so;
+    the context stays usable and the same workspace serves the next call unchanged."""
     idx, probs, hidden = _small_case(4000, 16, 2, 8, 2, seed=4)
-    p_bad = moe.Problem(N=4000, H=16, k=2, E_log=8, R=2, flags=moe.MOE_FLAG_TEST_BARRIER_TIMEOUT)
+    p_bad = moe.Problem(N=4000, H=16, k=2, E_log=8, R=2, flags=moe.MOE_FLAG_TEST_WAIT_TIMEOUT)
     G = moe.moe_dispatch_layout(p_bad, dev(idx), dev(probs))
     torch.cuda.synchronize()
     assert G.status() & moe.MOE_DEV_TIMEOUT
-    # after a timeout the workspace is zeroed, then a normal call works
+    # the timed-out call's outputs are invalid but stay inside their buffers
+    d = host(G["dest_row"])
+    assert d.min() >= -1 and d.max() < G.problem.rows_max
+    # the next call on the very same workspace (not zeroed again) is exact
     p = dataclasses.replace(p_bad, flags=0)
     G2 = moe.Layout.allocate(p)
+    G2.workspace = G.workspace
     moe.moe_dispatch_layout(p, dev(idx), dev(probs), layout=G2)
     torch.cuda.synchronize()
     assert G2.status() == 0
@@ -599,6 +649,7 @@ def test_random_sweep_full_path(case):
     assert np.allclose(host(gp), exp_gp, rtol=1e-4, atol=1e-4 * np.sqrt(H))
     assert np.array_equal(host(gh), oracle.permute_backward(exp_gy, L["dest_row"]))
     assert G.status() == 0
+    check_dispatch(p, idx, probs, hidden, L)
 
 
 def _sweep_next_cases(n=36, seed=20261203):
@@ -636,21 +687,30 @@ def test_random_sweep_next_rows(case):
         test_ep_exchange((R, N, H, k, E_log, C, reps, A))
 
 
-def test_grid_barrier_ticket_wraps():
-    """The layout's single-word grid barrier adds 2^20 per launch and wraps modulo 2^32
-    after 4096 launches on one workspace; 4200 launches in a row must all complete."""
-    N, k, E_log, R = 4096, 2, 16, 4  # 8192 assignments: 16 blocks meet at the barrier
-    idx, probs, _ = _small_case(N, 8, k, E_log, R, seed=99)
-    p = moe.Problem(N=N, H=8, k=k, E_log=E_log, R=R)
-    G = moe.Layout.allocate(p)
-    d_idx, d_probs = dev(idx), dev(probs)
-    for _ in range(4200):
-        moe.moe_dispatch_layout(p, d_idx, d_probs, layout=G)
+def test_lookback_epochs_across_many_launches():
+    """Every launch of the layout advances the workspace's epoch by one and leaves its ticket
+    count at zero; 4200 launches in a row on one workspace, alternating two grid sizes, stay
+    exact (each launch's look-back ignores the words of the launches before it)."""
+    cases = []
+    for N, seed in ((4096, 99), (1000, 98)):  # 16 and 4 count blocks
+        idx, probs, _ = _small_case(N, 8, 2, 16, 4, seed=seed)
+        p = moe.Problem(N=N, H=8, k=2, E_log=16, R=4)
+        cases.append((p, idx, probs, dev(idx), dev(probs)))
+    ws = moe.Layout.allocate(cases[0][0]).workspace
+    lays = []
+    for p, *_ in cases:
+        G = moe.Layout.allocate(p)
+        G.workspace = ws
+        lays.append(G)
+    for i in range(4200):
+        p, _, _, d_idx, d_probs = cases[i % 2]
+        moe.moe_dispatch_layout(p, d_idx, d_probs, layout=lays[i % 2])
     torch.cuda.synchronize()
-    assert G.status() == 0
-    assert_layout_equal(G, oracle.layout(idx, probs, E_log=E_log, R=R))
-    word = int(G.workspace[:4].view(torch.int32).item()) & 0xFFFFFFFF
-    assert word == (4200 << 20) & 0xFFFFFFFF  # every launch added exactly 2^20
+    for (p, idx, probs, _, _), G in zip(cases, lays):
+        assert G.status() == 0
+        assert_layout_equal(G, oracle.layout(idx, probs, E_log=16, R=4))
+    ticket = int(ws[:8].view(torch.int64).item())
+    assert ticket == 4200 << 32  # epoch 4200, no ticket outstanding
 
 
 def test_nvtx_ranges_on():

@@ -1,4 +1,4 @@
-"""Host model of the layout's single-word grid barrier (the arithmetic only).
+"""Host model of the dedup layout's single-word grid barrier (the arithmetic only).
 
 Each launch of G blocks adds exactly 2^20 to one 32-bit word: block 0 adds
 2^20 - (G - 1) - extra, every other block 1. A block computes its target from the

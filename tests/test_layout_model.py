@@ -1,8 +1,8 @@
-"""Host model of the dispatch layout kernel's decomposition, against the oracle (CPU).
+"""Host model of the dispatch layout count kernel's decomposition, against the oracle (CPU).
 
-The kernel splits the flattened [N, k] assignments over G blocks of 16 warps;
-warp w of block b owns the slice [(16 b + w) sub, (16 b + w + 1) sub) and takes
-it 32 items at a time in ascending order. An assignment's logical ordinal is
+The count kernel splits the flattened [N, k] assignments over G blocks of 16 warps;
+warp w of the block with ticket b owns the slice [(16 b + w) sub, (16 b + w + 1) sub)
+and takes it 32 items at a time in ascending order. An assignment's logical ordinal is
 then  (same-id items of earlier blocks) + (same-id items of earlier warps of its
 block) + (same-id items earlier in its own slice).  With replicas, the physical
 expert and ordinal follow in closed form from the logical ordinal o: the master
@@ -17,22 +17,24 @@ import pytest
 LAYOUT_THREADS = 512
 LAYOUT_WARPS = 16
 LAYOUT_MAX_BLOCKS = 128
+LAYOUT_TARGET_BLOCKS = 32
 LAYOUT_MAX_IPL = 8
-LAYOUT_ITEMS_PER_BLOCK = 512
 
 
 def layout_grid(NK):
-    G = max(1, min(LAYOUT_MAX_BLOCKS, -(-NK // LAYOUT_ITEMS_PER_BLOCK)))
-    ipl = max(1, -(-NK // (G * LAYOUT_THREADS)))
-    kind = 0
-    if ipl <= LAYOUT_MAX_IPL:
-        p2 = 1
-        while p2 < ipl:
-            p2 <<= 1
-        ipl = kind = p2
-    sub = 32 * ipl
-    G = max(1, -(-NK // (LAYOUT_WARPS * sub)))
-    return G, sub, kind
+    """The host's grid rule: the fewest ids per lane (1, 2, 4, 8) that keep the grid at
+    32 blocks or fewer; else 8 per lane on up to 128 blocks; else longer slices."""
+    ipl = 1
+    while ipl < LAYOUT_MAX_IPL and -(-NK // (LAYOUT_THREADS * ipl)) > LAYOUT_TARGET_BLOCKS:
+        ipl <<= 1
+    G = -(-NK // (LAYOUT_THREADS * ipl))
+    kind, sub = ipl, 32 * ipl
+    if G > LAYOUT_MAX_BLOCKS:
+        kind = 0
+        per_warp = -(-NK // (LAYOUT_MAX_BLOCKS * LAYOUT_WARPS))
+        sub = -(-per_warp // 32) * 32
+        G = -(-NK // (LAYOUT_WARPS * sub))
+    return max(G, 1), sub, kind
 
 
 def model_logical_ordinals(ids, E_log):
@@ -72,12 +74,18 @@ def model_logical_ordinals(ids, E_log):
 
 
 def test_grid_shapes():
-    for NK in [0, 1, 511, 512, 513, 32768, 65535, 65536, 65537, 288000, 600000, 2 ** 22]:
+    for NK in [0, 1, 511, 512, 513, 16384, 16385, 32768, 65535, 65536, 65537, 288000, 524288, 524289,
+               600000, 2 ** 22, 2 ** 31 - 1]:
         G, sub, kind = layout_grid(NK)
         assert 1 <= G <= LAYOUT_MAX_BLOCKS and G * LAYOUT_WARPS * sub >= NK
         assert kind in (0, 1, 2, 4, 8) and (kind == 0 or sub == 32 * kind)
+        assert sub % 32 == 0 and sub < 2 ** 31
         if NK:  # no block is left without items
             assert (G - 1) * LAYOUT_WARPS * sub < NK
+        if NK <= LAYOUT_TARGET_BLOCKS * LAYOUT_THREADS * LAYOUT_MAX_IPL:  # the look-back ends in one round
+            assert G <= LAYOUT_TARGET_BLOCKS
+    # the surveyed shapes: 4096 x 8 and 8192 x 8 assignments take 32 blocks
+    assert layout_grid(32768)[:1] == (32,) and layout_grid(65536)[:1] == (32,)
 
 
 @pytest.mark.parametrize("N,k,E_log,reps,R,seed", [

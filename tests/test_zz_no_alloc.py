@@ -73,10 +73,10 @@ def test_noalloc_matches_allocating_layout_on_consecutive_calls(case):
 
 
 def test_noalloc_recovers_after_a_timed_out_call():
-    """A call whose barrier ran out leaves the shared scratch dirty; the next call clears it."""
+    """A call whose look-back ran out leaves nothing in the shared scratch that the next call must clear."""
     require_cuda()
     idx, probs = _inputs(3000, 4, 32, seed=5)
-    bad = moe.Problem(N=3000, H=8, k=4, E_log=32, R=4, flags=moe.MOE_FLAG_TEST_BARRIER_TIMEOUT)
+    bad = moe.Problem(N=3000, H=8, k=4, E_log=32, R=4, flags=moe.MOE_FLAG_TEST_WAIT_TIMEOUT)
     lay = moe.Layout.allocate(bad)
     assert _noalloc_c_call(bad, idx, probs, lay) == 0
     torch.cuda.synchronize()
