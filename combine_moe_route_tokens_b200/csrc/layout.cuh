@@ -550,6 +550,8 @@ __device__ __forceinline__ bool layout_emit_row(const LayoutArgs &a, const Layou
 // keeps IPL ids in registers (sub = 32 * IPL); 0: any sub, the slice is read
 // twice. It lets the next kernel launch only after its own wait has returned,
 // so that kernel may read the inputs of this call (written before it) early.
+// A ticket beyond the grid (only when two calls share one workspace at once,
+// which the contract forbids) makes the block report MOE_DEV_TIMEOUT and stop.
 template <int IPL>
 __global__ void __launch_bounds__(LAYOUT_THREADS, 1) layout_count_kernel(LayoutArgs a)
 {
@@ -572,16 +574,25 @@ __global__ void __launch_bounds__(LAYOUT_THREADS, 1) layout_count_kernel(LayoutA
         s_err = 0;
         s_timeout = 0;
     }
-    pdl_wait(); // ids, the ticket word and earlier launches' words are settled
-    pdl_trigger();
+    // The ticket is drawn before the wait: only count passes touch the ticket word,
+    // and the next count pass on this workspace launches after this one lets its
+    // dependents launch, which happens below, after every ticket of this launch has
+    // been drawn (stream order; a kernel launches only once its predecessor let it).
     if (tid == 0) {
         uint32_t vb, epoch;
         lb_take_ticket(a.ws_ticket, static_cast<uint32_t>(a.G), &vb, &epoch);
         s_vb = vb;
         s_epoch = epoch;
     }
+    pdl_wait(); // ids and earlier launches' words are settled
     __syncthreads();
+    pdl_trigger();
     const uint32_t vb = s_vb, epoch = s_epoch;
+    if (vb >= static_cast<uint32_t>(a.G)) { // two calls shared the workspace at once: stay inside it
+        if (tid == 0)
+            atomicOr(a.out.status, MOE_DEV_TIMEOUT);
+        return;
+    }
     const int64_t base = (static_cast<int64_t>(vb) * LAYOUT_WARPS + warp) * a.sub;
     uint32_t *my_cnt = wcnt + warp * E_log;
 
