@@ -12,6 +12,7 @@ functions keep the C names:
     moe_restore_combined  the same over the buffers of TP peers (after TP folding)
     moe_dedup_*           DeepEP-style view: one receive row per (token, rank), two-level combine
     moe_ep_*              expert-parallel exchange: dispatch into / combine from the ranks' receive buffers
+    EpGroup               that exchange between processes (CUDA IPC mappings, offsets all-gather, fences)
     moe_permute_backward  grad_hidden[t] = bf16(sum_j grad_send[dest_row[t, j]])
     moe_combine_backward  grad_y[row] = bf16(p * grad_out[t]); grad_probs[t, j] = <grad_out[t], y[row]>
 
@@ -63,6 +64,7 @@ __all__ = [
     "moe_restore_combined",
     "DedupView",
     "EpPlan",
+    "EpGroup",
     "peer_table",
     "moe_ep_recv_rows_max",
     "moe_ep_plan",
@@ -701,3 +703,6 @@ def moe_combine_backward(problem: Problem, layout: Layout, grad_out: torch.Tenso
                                                      _ptr(expert_out), _ptr(topk_probs), _ptr(grad_expert_out),
                                                      _ptr(grad_probs), _stream(stream)))
     return grad_expert_out, grad_probs
+
+
+from .ep_group import EpGroup  # noqa: E402  (the exchange between processes; host plumbing only)

@@ -114,6 +114,16 @@ _PP = ctypes.POINTER(MoeProblem)
 _PL = ctypes.POINTER(MoeLayout)
 _PD = ctypes.POINTER(MoeDedup)
 
+class MoeIpcBuffer(ctypes.Structure):
+    _fields_ = [
+        ("handle", ctypes.c_ubyte * 64),
+        ("offset", ctypes.c_uint64),
+        ("bytes", ctypes.c_uint64),
+        ("device", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+    ]
+
+
 _SIGNATURES = {
     "moe_abi_version": (ctypes.c_int, []),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -123,6 +133,11 @@ _SIGNATURES = {
     "moe_dispatch_layout": (ctypes.c_int, [_PP, _VP, _VP, _PL, _VP, ctypes.c_size_t, _VP]),
     "moe_dispatch_layout_noalloc": (ctypes.c_int, [_PP, _VP, _VP, _PL, _VP]),
     "moe_dispatch": (ctypes.c_int, [_PP, _VP, _VP, _PL, _VP, ctypes.c_size_t, _VP, _VP, _VP]),
+    "moe_ep_publish_offsets": (ctypes.c_int, [_PP, _VP, ctypes.c_int32, _VP, _VP]),
+    "moe_ipc_export": (ctypes.c_int, [_VP, ctypes.c_size_t, ctypes.POINTER(MoeIpcBuffer)]),
+    "moe_ipc_open": (ctypes.c_int, [ctypes.POINTER(MoeIpcBuffer), ctypes.POINTER(ctypes.c_void_p),
+                                    ctypes.POINTER(ctypes.c_void_p)]),
+    "moe_ipc_close": (ctypes.c_int, [_VP]),
     "moe_permute": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP]),
     "moe_combine": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP]),
     "moe_restore_combined": (ctypes.c_int, [_PP, _PL, _VP, _VP, _VP, _VP]),

@@ -113,4 +113,27 @@ __global__ void __launch_bounds__(EP_PLAN_THREADS) ep_plan_kernel(EpPlanArgs a)
         atomicOr(a.status, err);
 }
 
+
+// The all-gather of the ranks' expert_offsets over peer memory: this rank's
+// [E+1] offsets go to row `src` of every rank's [R][E+1] table (peer_tables:
+// R device pointers, own rank's table included). One thread per (rank, entry).
+struct EpPublishArgs {
+    const int32_t *offsets;      // [E + 1] this rank's layout expert_offsets
+    int32_t *const *peer_tables; // [R] each a [R][E + 1] table
+    int32_t R, E, src;
+};
+
+__global__ void __launch_bounds__(256) ep_publish_offsets_kernel(EpPublishArgs a)
+{
+    pdl_trigger();
+    pdl_wait(); // the offsets come from the layout just before
+    const int64_t n = static_cast<int64_t>(a.R) * (a.E + 1);
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int q = static_cast<int>(i / (a.E + 1));
+        const int j = static_cast<int>(i - static_cast<int64_t>(q) * (a.E + 1));
+        a.peer_tables[q][static_cast<int64_t>(a.src) * (a.E + 1) + j] = __ldg(a.offsets + j);
+    }
+}
+
 } // namespace moert

@@ -7,12 +7,14 @@
 // attributes (SM count, shared-memory limit) with the kernel attribute setup,
 // the programmatic-launch fallback flags and the NVTX switch.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
 #include <cstdio>
 #include <atomic>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include <nvtx3/nvToolsExt.h>
@@ -1008,6 +1010,30 @@ int moe_ep_plan(const moe_problem_t *problem, const int32_t *offsets_all, int32_
     return launch(ep_plan_kernel, dim3(1), dim3(EP_PLAN_THREADS), smem, stream, false, a);
 }
 
+int moe_ep_publish_offsets(const moe_problem_t *problem, const int32_t *expert_offsets, int32_t src_rank,
+                           int32_t *const *peer_offsets_tables, void *stream)
+{
+    NvtxRange nvtx_range("moe_ep_publish_offsets");
+    Dims d;
+    int rc = check_problem(problem, &d);
+    if (rc != MOE_OK)
+        return rc;
+    if (problem->tp_size > 1 || problem->R > MOE_MAX_EP_RANKS)
+        return MOE_ERR_UNSUPPORTED;
+    if (src_rank < 0 || src_rank >= problem->R || expert_offsets == nullptr || peer_offsets_tables == nullptr)
+        return MOE_ERR_INVALID;
+    EpPublishArgs a;
+    a.offsets = expert_offsets;
+    a.peer_tables = peer_offsets_tables;
+    a.R = problem->R;
+    a.E = d.E;
+    a.src = src_rank;
+    const int64_t n = static_cast<int64_t>(a.R) * (a.E + 1);
+    const int64_t blocks = (n + 255) / 256;
+    return launch(ep_publish_offsets_kernel, dim3(static_cast<unsigned>(blocks < 64 ? blocks : 64)), dim3(256), 0,
+                  stream, false, a);
+}
+
 int moe_ep_dispatch(const moe_problem_t *problem, const moe_layout_t *layout, const int32_t *base,
                     const uint16_t *hidden, uint16_t *const *peer_recv, void *stream)
 {
@@ -1314,4 +1340,90 @@ extern "C" int moe_dispatch_layout_noalloc(const moe_problem_t *problem, const i
     // carries the epoch of the launch that wrote it, and the ticket word is
     // rolled over by the last block of each launch (also after a timed-out one).
     return moe_dispatch_layout(problem, topk_idx, topk_probs, layout, scratch, MOE_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+// ------------------------------------------------------------- CUDA IPC --
+// Sharing a buffer between processes of the expert-parallel exchange: the
+// allocation that holds it is exported with cudaIpcGetMemHandle together with
+// the buffer's offset inside it (a caching allocator hands out pieces of larger
+// allocations); a peer maps the allocation with cudaIpcOpenMemHandle.
+
+namespace {
+
+using AddressRangeFn = CUresult (*)(CUdeviceptr *, size_t *, CUdeviceptr);
+
+AddressRangeFn address_range_fn()
+{
+    static AddressRangeFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            (void)cudaGetLastError();
+            return static_cast<AddressRangeFn>(nullptr);
+        }
+        return reinterpret_cast<AddressRangeFn>(p);
+    }();
+    return fn;
+}
+
+static_assert(sizeof(cudaIpcMemHandle_t) == sizeof(((moe_ipc_buffer_t *)nullptr)->handle),
+              "moe_ipc_buffer_t.handle must hold a cudaIpcMemHandle_t");
+
+} // namespace
+
+extern "C" int moe_ipc_export(const void *ptr, size_t bytes, moe_ipc_buffer_t *out)
+{
+    if (ptr == nullptr || out == nullptr)
+        return MOE_ERR_INVALID;
+    AddressRangeFn range = address_range_fn();
+    if (range == nullptr)
+        return MOE_ERR_CUDA;
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (range(&base, &size, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS)
+        return MOE_ERR_INVALID; // not device memory of this process
+    const uint64_t offset = reinterpret_cast<uint64_t>(ptr) - static_cast<uint64_t>(base);
+    if (offset + bytes > size)
+        return MOE_ERR_INVALID;
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, reinterpret_cast<void *>(base)) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    memcpy(out->handle, &h, sizeof(h));
+    out->offset = offset;
+    out->bytes = bytes;
+    out->device = dev;
+    return MOE_OK;
+}
+
+extern "C" int moe_ipc_open(const moe_ipc_buffer_t *buf, void **ptr, void **mapping)
+{
+    if (buf == nullptr || ptr == nullptr || mapping == nullptr)
+        return MOE_ERR_INVALID;
+    cudaIpcMemHandle_t h;
+    memcpy(&h, buf->handle, sizeof(h));
+    void *base = nullptr;
+    if (cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    *mapping = base;
+    *ptr = static_cast<uint8_t *>(base) + buf->offset;
+    return MOE_OK;
+}
+
+extern "C" int moe_ipc_close(void *mapping)
+{
+    if (mapping == nullptr)
+        return MOE_ERR_INVALID;
+    if (cudaIpcCloseMemHandle(mapping) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
 }

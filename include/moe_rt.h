@@ -411,6 +411,20 @@ MOE_API int moe_ep_plan(const moe_problem_t *problem, const int32_t *offsets_all
                         int32_t *recv_expert_offsets, int32_t *num_recv, uint32_t *status, void *stream);
 
 /*
+ * The all-gather of expert_offsets that the exchange needs, over peer memory
+ * (the only collective of the exchange): writes this rank's layout
+ * expert_offsets [E+1] into row src_rank of every rank's [R][E+1] offsets
+ * table. peer_offsets_tables: device array of R device pointers (this rank's
+ * own table included; the others mapped from their processes, see
+ * moe_ipc_open, or other buffers on this GPU). Every rank's tables are
+ * complete once every rank's call has run; the caller orders that (for
+ * example an interprocess event per rank and a host barrier) before
+ * moe_ep_plan reads them.
+ */
+MOE_API int moe_ep_publish_offsets(const moe_problem_t *problem, const int32_t *expert_offsets, int32_t src_rank,
+                                   int32_t *const *peer_offsets_tables, void *stream);
+
+/*
  * Dispatch with the exchange fused in: for every kept slot (t, j) of expert q,
  * peer_recv[q / E_loc][base[q] + dest_row[t,j] - expert_offsets[q]] = hidden[t];
  * this rank's padding rows of every expert are zeroed there.
@@ -451,6 +465,38 @@ MOE_API int moe_ep_combine_backward(const moe_problem_t *problem, const moe_layo
                                     const uint16_t *grad_out, const uint16_t *const *peer_expert_out,
                                     const float *topk_probs, uint16_t *const *peer_grad_expert_out,
                                     float *grad_probs, void *stream);
+
+/*
+ * Sharing buffers between the processes of the exchange (one process per rank).
+ * The owner exports a device buffer: the handle of the allocation that holds it
+ * (cudaIpcGetMemHandle), the buffer's byte offset inside that allocation (so
+ * that buffers carved out of a larger allocation, as caching allocators do,
+ * can be shared) and its size. The handle is plain bytes: send it to the
+ * other processes by any means. A peer process maps it with moe_ipc_open
+ * (cudaIpcOpenMemHandle with lazy peer access: the buffer may be on this GPU or
+ * on another one reachable by peer access) and gets the buffer's address and
+ * the mapping, which moe_ipc_close releases. A process cannot open its own
+ * handles. The owner keeps the buffer allocated until every peer has closed it.
+ * Host calls; nothing is enqueued on a stream.
+ */
+typedef struct {
+    unsigned char handle[64]; /* cudaIpcMemHandle_t of the allocation */
+    uint64_t offset;          /* the buffer's byte offset inside that allocation */
+    uint64_t bytes;           /* the buffer's size */
+    int32_t device;           /* the owner's device ordinal (in the owner's process) */
+    int32_t reserved;
+} moe_ipc_buffer_t;
+
+/* Export [ptr, ptr + bytes) of this process's device memory. MOE_ERR_INVALID if
+ * the range is not inside one allocation of this process. */
+MOE_API int moe_ipc_export(const void *ptr, size_t bytes, moe_ipc_buffer_t *out);
+
+/* Map a buffer another process exported: *ptr = its address here, *mapping = the
+ * mapping to pass to moe_ipc_close. */
+MOE_API int moe_ipc_open(const moe_ipc_buffer_t *buf, void **ptr, void **mapping);
+
+/* Release a mapping made by moe_ipc_open. */
+MOE_API int moe_ipc_close(void *mapping);
 
 /*
  * Backward of permute ([Megatron MORI]: dispatch backward sums the row
