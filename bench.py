@@ -236,15 +236,16 @@ class Step:
     layout and the send buffer of every peer in turn (all on this GPU), and
     restores with one slot-ordered combine over the peers' buffers."""
 
-    def __init__(self, w, moe, native, torch, sets, device, unfused=False):
+    def __init__(self, w, moe, native, torch, sets, device, unfused=False, bulk_copy=False):
         self.w = w
         self.torch = torch
         self.lib = native.lib()
         T = max(w.tp_size, 1)
         self.T = T
+        flags = moe.MOE_FLAG_DISPATCH_BULK_COPY if bulk_copy else 0
         self.problems = [moe.Problem(N=w.N, H=w.H, k=w.k, E_log=w.E_log, R=w.R, capacity=w.capacity,
                                      num_replicas=w.num_replicas, row_align=w.row_align,
-                                     tp_size=w.tp_size, tp_rank=r) for r in range(T)]
+                                     tp_size=w.tp_size, tp_rank=r, flags=flags) for r in range(T)]
         p = self.problems[0]
         self.problem = p
         self.layouts = [moe.Layout.allocate(q, device) for q in self.problems]
@@ -543,7 +544,8 @@ def measure(w, host, steps, warmup, eager, hot_l2, ctx):
     work_stream = torch.cuda.Stream(device)
     with torch.cuda.stream(work_stream):
         step = EpStep(w, moe, _native, torch, sets, device) if w.ep else \
-            Step(w, moe, _native, torch, sets, device, unfused=ctx.get("unfused", False))
+            Step(w, moe, _native, torch, sets, device, unfused=ctx.get("unfused", False),
+                 bulk_copy=ctx.get("bulk_copy", False))
     for i in range(warmup):
         step.run(i)
     torch.cuda.synchronize()
@@ -683,7 +685,7 @@ def run_ours(args, ws, rank, local):
     host = rank_inputs(w, rank)
     sampler = ClockSampler(local)
     ctx = {"torch": torch, "moe": moe, "native": _native, "device": device, "barrier": barrier, "sampler": sampler,
-           "unfused": args.unfused}
+           "unfused": args.unfused, "bulk_copy": args.bulk_copy}
     with sampler:
         m = measure(w, host, args.steps, args.warmup, args.eager, True, ctx)
     step, abytes, elapsed_ms, hot_ms = m["step"], m["abytes"], m["elapsed_ms"], m["hot_ms"]
@@ -761,6 +763,9 @@ def run_ours(args, ws, rank, local):
                 for n in m["step"].kernel_names)),
             "l2": f"inputs rotated over {m['nsets']} buffer sets ({m['nsets'] * m['set_bytes'] / 2**20:.0f} MiB "
                   f"> 126 MB L2), no flush",
+            "dispatch": ("moe_dispatch_layout + moe_permute (separate calls)" if args.unfused else
+                         "moe_dispatch (layout + permute fused), rows copied with "
+                         + ("bulk (TMA) copies through shared memory" if args.bulk_copy else "16-byte vector copies")),
         },
         "effective_gbs": round(path_bytes / (ms_step * 1e-3) / 1e9, 1),
         "effective_hbm_frac": round(path_bytes / (ms_step * 1e-3) / 1e9 / peak, 3),
@@ -808,7 +813,8 @@ def measure_e2e(w, host, step, args, ws, ctx):
         for b in range(depth):
             dset = {key: torch.empty_like(step.sets[0][key]) for key in pin}
             pipes.append(EpStep(w, moe, _native, torch, [dset], device) if w.ep else
-                         Step(w, moe, _native, torch, [dset], device, unfused=ctx.get("unfused", False)))
+                         Step(w, moe, _native, torch, [dset], device, unfused=ctx.get("unfused", False),
+                              bulk_copy=ctx.get("bulk_copy", False)))
     views = [{key: (q.sets[0][key].view(torch.int16) if q.sets[0][key].dtype == torch.bfloat16
                     else q.sets[0][key]) for key in pin} for q in pipes]
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
@@ -1075,6 +1081,9 @@ def main():
                          "(default: ht as the headline, with tiny, qwen3, capacity and ultraep timed beside it)")
     ap.add_argument("--unfused", action="store_true",
                     help="call moe_dispatch_layout and moe_permute separately instead of the fused moe_dispatch")
+    ap.add_argument("--bulk-copy", action="store_true",
+                    help="stage the dispatch's rows through shared memory with bulk (TMA) copies "
+                         "(MOE_FLAG_DISPATCH_BULK_COPY) instead of 16-byte vector copies")
     ap.add_argument("--no-extra", action="store_true",
                     help="time only the headline workload (skip the other surveyed configurations)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

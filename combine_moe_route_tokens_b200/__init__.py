@@ -37,6 +37,7 @@ from ._native import (
     MOE_DEV_TIMEOUT,
     MOE_FLAG_NONE,
     MOE_FLAG_TEST_WAIT_TIMEOUT,
+    MOE_FLAG_DISPATCH_BULK_COPY,
 )
 
 COUNTER_NAMES = (
@@ -84,6 +85,7 @@ __all__ = [
     "MOE_DEV_TIMEOUT",
     "MOE_FLAG_NONE",
     "MOE_FLAG_TEST_WAIT_TIMEOUT",
+    "MOE_FLAG_DISPATCH_BULK_COPY",
 ]
 
 

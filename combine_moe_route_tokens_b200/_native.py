@@ -32,6 +32,7 @@ MOE_DEV_ROW_RANGE = 0x4
 
 MOE_FLAG_NONE = 0
 MOE_FLAG_TEST_WAIT_TIMEOUT = 0x80000000
+MOE_FLAG_DISPATCH_BULK_COPY = 0x1
 
 ABI_VERSION = 6
 

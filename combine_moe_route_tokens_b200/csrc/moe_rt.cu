@@ -72,6 +72,13 @@ DispatchKernel dispatch_for(bool reroute, bool dense)
     return dense ? dispatch_kernel<false, true> : dispatch_kernel<false, false>;
 }
 
+DispatchKernel dispatch_bulk_for(bool reroute, bool dense)
+{
+    if (reroute)
+        return dense ? dispatch_bulk_kernel<true, true> : dispatch_bulk_kernel<true, false>;
+    return dense ? dispatch_bulk_kernel<false, true> : dispatch_bulk_kernel<false, false>;
+}
+
 constexpr int LAYOUT_IPLS[] = {0, 1, 2, 4, 8};
 
 // NVTX ranges around the enqueuing entry points, for profilers' timelines: on
@@ -199,6 +206,12 @@ int device_info(DeviceInfo *out)
                     e = cudaFuncGetAttributes(&fa1, layout_fill_for(rr != 0, dn != 0));
                 if (e == cudaSuccess)
                     e = cudaFuncGetAttributes(&fa2, dispatch_for(rr != 0, dn != 0));
+                cudaFuncAttributes fa3;
+                if (e == cudaSuccess)
+                    e = cudaFuncGetAttributes(&fa3, dispatch_bulk_for(rr != 0, dn != 0));
+                if (e == cudaSuccess)
+                    static2 = static_cast<int>(fa3.sharedSizeBytes) > static2 ? static_cast<int>(fa3.sharedSizeBytes)
+                                                                             : static2;
                 if (e == cudaSuccess) {
                     static2 = static_cast<int>(fa1.sharedSizeBytes) > static2 ? static_cast<int>(fa1.sharedSizeBytes)
                                                                              : static2;
@@ -214,6 +227,9 @@ int device_info(DeviceInfo *out)
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, d.tables_dyn_max);
                 if (e == cudaSuccess)
                     e = cudaFuncSetAttribute(dispatch_for(rr != 0, dn != 0),
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, d.tables_dyn_max);
+                if (e == cudaSuccess)
+                    e = cudaFuncSetAttribute(dispatch_bulk_for(rr != 0, dn != 0),
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, d.tables_dyn_max);
             }
         if (e != cudaSuccess || d.layout_dyn_max <= 0)
@@ -245,7 +261,7 @@ int check_problem(const moe_problem_t *p, Dims *d)
         return MOE_ERR_INVALID;
     if (p->E_log % p->R != 0 || p->num_replicas % p->R != 0 || p->num_replicas > p->E_log)
         return MOE_ERR_INVALID;
-    if ((p->flags & ~MOE_FLAG_TEST_WAIT_TIMEOUT) != 0)
+    if ((p->flags & ~(MOE_FLAG_TEST_WAIT_TIMEOUT | MOE_FLAG_DISPATCH_BULK_COPY)) != 0)
         return MOE_ERR_INVALID;
     if (p->row_align < 0 || p->tp_size < 0 || p->tp_rank < 0)
         return MOE_ERR_INVALID;
@@ -524,23 +540,49 @@ int moe_dispatch(const moe_problem_t *problem, const int32_t *topk_idx, const fl
     da.send = reinterpret_cast<uint4 *>(send);
     da.N = problem->N;
     da.V = problem->H / 8;
-    da.group = da.V <= 32 * PERMUTE_CHUNKS ? 32 : (da.V <= 64 * PERMUTE_CHUNKS ? 64 : PERMUTE_THREADS);
-    da.pieces = (da.V + da.group * PERMUTE_CHUNKS - 1) / (da.group * PERMUTE_CHUNKS);
-    // row CTAs: one thread per row per pass, at most four CTAs per SM; CTA 0 writes the tables
-    const int64_t rb = (d.rows_max + PERMUTE_THREADS - 1) / PERMUTE_THREADS;
-    da.row_ctas = static_cast<int32_t>(rb < 1 ? 1 : (rb < 4 * dev.sms ? rb : 4 * dev.sms));
-    const int64_t groups = PERMUTE_THREADS / da.group;
-    const int64_t blocks = da.row_ctas + (problem->N * da.pieces + groups - 1) / groups;
-    if (blocks > INT32_MAX)
-        return MOE_ERR_UNSUPPORTED;
     const bool reroute = problem->num_replicas > 0;
     const bool dense = problem->capacity == 0 && d.A == 1;
+    const size_t tables_bytes = layout_tables_smem_words(problem->E_log, d.E) * 4;
+    DispatchKernel kernel;
+    int64_t blocks;
+    size_t smem;
+    int threads;
+    if ((problem->flags & MOE_FLAG_DISPATCH_BULK_COPY) == 0) {
+        da.group = da.V <= 32 * PERMUTE_CHUNKS ? 32 : (da.V <= 64 * PERMUTE_CHUNKS ? 64 : PERMUTE_THREADS);
+        da.pieces = (da.V + da.group * PERMUTE_CHUNKS - 1) / (da.group * PERMUTE_CHUNKS);
+        const int64_t groups = PERMUTE_THREADS / da.group;
+        threads = PERMUTE_THREADS;
+        const int64_t rb = (d.rows_max + threads - 1) / threads; // row CTAs: at most four per SM; CTA 0 writes the tables
+        da.row_ctas = static_cast<int32_t>(rb < 1 ? 1 : (rb < 4 * dev.sms ? rb : 4 * dev.sms));
+        blocks = da.row_ctas + (problem->N * da.pieces + groups - 1) / groups;
+        smem = tables_bytes;
+        kernel = dispatch_for(reroute, dense);
+    } else {
+        // rows staged in shared memory: pieces of at most 32 KB; rows of at most 16 KB go several to a CTA
+        const int64_t row_bytes = static_cast<int64_t>(da.V) * 16;
+        da.pieces = static_cast<int32_t>((row_bytes + 32768 - 1) / 32768);
+        da.group = da.pieces > 1 ? 1
+                                 : static_cast<int32_t>(row_bytes >= 16384 ? 1
+                                                                           : (16384 / row_bytes > TMA_MAX_TOKENS
+                                                                                  ? TMA_MAX_TOKENS
+                                                                                  : 16384 / row_bytes));
+        threads = TMA_THREADS;
+        const int64_t rb = (d.rows_max + threads - 1) / threads;
+        da.row_ctas = static_cast<int32_t>(rb < 1 ? 1 : (rb < 4 * dev.sms ? rb : 4 * dev.sms));
+        blocks = da.row_ctas + (da.pieces > 1 ? problem->N * da.pieces : (problem->N + da.group - 1) / da.group);
+        const int64_t pchunks = (da.V + da.pieces - 1) / da.pieces;
+        smem = ((tables_bytes / 4 + 31) & ~size_t(31)) * 4 + static_cast<size_t>(da.group) * pchunks * 16;
+        if (smem > static_cast<size_t>(dev.tables_dyn_max))
+            return MOE_ERR_UNSUPPORTED;
+        kernel = dispatch_bulk_for(reroute, dense);
+    }
+    if (blocks > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
     rc = launch(layout_count_for(lg.ipl), dim3(lg.G), dim3(LAYOUT_THREADS),
                 layout_count_smem_words(problem->E_log) * 4, stream, false, da.L);
     if (rc != MOE_OK)
         return rc;
-    return launch(dispatch_for(reroute, dense), dim3(static_cast<unsigned>(blocks)), dim3(PERMUTE_THREADS),
-                  layout_tables_smem_words(problem->E_log, d.E) * 4, stream, false, da);
+    return launch(kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), smem, stream, false, da);
 }
 
 int moe_permute(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *hidden, uint16_t *send,

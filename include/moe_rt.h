@@ -73,6 +73,11 @@ extern "C" {
  * its counts, so the next block's look-back waits for a word that never comes,
  * with a ~10 ms limit; the timeout path runs without hanging anything. */
 #define MOE_FLAG_TEST_WAIT_TIMEOUT 0x80000000u
+/* moe_dispatch only: stage each token row through shared memory with bulk (TMA)
+ * copies, one bulk load per row and one bulk store per kept destination row,
+ * instead of 16-byte vector loads and stores. Same results bit for bit; on B200
+ * slower for this one-read / k-write scatter, so it is not the default. */
+#define MOE_FLAG_DISPATCH_BULK_COPY 0x1u
 
 /* The problem statement ([DeepSpeed EP] RoutedAssignmentPayload; it follows the
  * pages' shapes: hidden [N,H] bf16, topk ids [N,k] int32, probs [N,k] fp32). */

@@ -68,7 +68,7 @@ def test_rows_max(lib, kw, rows):
         dict(N=4, H=8, k=1, E_log=4, R=2, num_replicas=6),  # more replicas than experts
         dict(N=4, H=8, k=1, E_log=4, R=1, capacity=-1),
         dict(N=2**31, H=8, k=2, E_log=4, R=1),  # N*k overflows int32
-        dict(N=4, H=8, k=1, E_log=4, R=1, flags=0x1),  # unknown flag
+        dict(N=4, H=8, k=1, E_log=4, R=1, flags=0x2),  # unknown flag
         dict(N=4, H=8, k=1, E_log=4, R=1, row_align=-2),
         dict(N=4, H=8, k=1, E_log=4, R=1, capacity=10, row_align=4),  # capacity not a multiple of the alignment
         dict(N=4, H=8, k=1, E_log=4, R=1, tp_size=2, tp_rank=2),  # rank outside the peers

@@ -89,6 +89,9 @@ def check_dispatch(p, idx, probs, hidden, L):
 def test_dispatch_fused(name):
     w, d, idx, probs, L = workload_case(name)
     check_dispatch(problem_of(w), idx, probs, d["hidden"], L)
+    # the same call with the rows staged through shared memory by bulk copies
+    check_dispatch(dataclasses.replace(problem_of(w), flags=moe.MOE_FLAG_DISPATCH_BULK_COPY), idx, probs,
+                   d["hidden"], L)
 
 
 @pytest.mark.parametrize("name", WORKLOAD_NAMES)
@@ -260,6 +263,7 @@ def test_edge_cases_full_path(case):
     assert np.array_equal(host(moe.moe_permute_backward(p, G, gy)), oracle.permute_backward(exp_gy, L["dest_row"]))
     assert G.status() == 0
     check_dispatch(p, idx, probs, hidden, L)
+    check_dispatch(dataclasses.replace(p, flags=moe.MOE_FLAG_DISPATCH_BULK_COPY), idx, probs, hidden, L)
 
 
 @pytest.mark.parametrize("C", [0, 5])
@@ -650,6 +654,7 @@ def test_random_sweep_full_path(case):
     assert np.array_equal(host(gh), oracle.permute_backward(exp_gy, L["dest_row"]))
     assert G.status() == 0
     check_dispatch(p, idx, probs, hidden, L)
+    check_dispatch(dataclasses.replace(p, flags=moe.MOE_FLAG_DISPATCH_BULK_COPY), idx, probs, hidden, L)
 
 
 def _sweep_next_cases(n=36, seed=20261203):
