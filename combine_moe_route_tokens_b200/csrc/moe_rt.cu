@@ -638,7 +638,12 @@ int launch_combine_args(CombineArgs a, int k, void *stream)
         // short rows with one or two slots: several tokens per CTA, four chunks per thread
         if ((k == 1 || k == 2) && (a.V == 128 || a.V == 256 || a.V == 512 || a.V == 1024)) {
             const int64_t per_cta = COMBINE_THREADS / (a.V / COMBINE_ROW_CPT);
-            const int64_t blocks = (a.N + per_cta - 1) / per_cta;
+            int64_t blocks = (a.N + per_cta - 1) / per_cta;
+            DeviceInfo dev;
+            if (device_info(&dev) != MOE_OK)
+                return MOE_ERR_CUDA;
+            if (blocks > 4 * static_cast<int64_t>(dev.sms)) // grid-stride: four CTAs per SM (the register limit)
+                blocks = 4 * static_cast<int64_t>(dev.sms);
             if (blocks > INT32_MAX)
                 return MOE_ERR_UNSUPPORTED;
             const dim3 grid(static_cast<unsigned>(blocks)), block(COMBINE_THREADS);
