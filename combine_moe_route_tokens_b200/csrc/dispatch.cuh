@@ -196,7 +196,7 @@ constexpr int TMA_MAX_TOKENS = 8;
 template <bool REROUTE, bool DENSE>
 __global__ void __launch_bounds__(TMA_THREADS) dispatch_bulk_kernel(DispatchArgs d)
 {
-    extern __shared__ __align__(128) int32_t dispatch_smem[];
+    extern __shared__ __align__(16) int32_t bulk_smem[]; // bulk copies need 16-byte alignment
     __shared__ int32_t s_dest[TMA_MAX_TOKENS][32];
     __shared__ __align__(8) uint64_t s_bar;
     const LayoutArgs &a = d.L;
@@ -213,10 +213,10 @@ __global__ void __launch_bounds__(TMA_THREADS) dispatch_bulk_kernel(DispatchArgs
     const int32_t c_first = piece * pchunks;
     const int32_t nchunks = min(pchunks, d.V - c_first);
     const uint32_t pbytes = static_cast<uint32_t>(nchunks) * 16u;
-    LayoutTables tb = layout_tables_carve(a, dispatch_smem);
-    // the row buffer follows the tables, 128-byte aligned
+    LayoutTables tb = layout_tables_carve(a, bulk_smem);
+    // the row buffer follows the tables, at a 128-byte offset
     const size_t tw = layout_tables_smem_words(a.E_log, a.E);
-    uint4 *s_rows = reinterpret_cast<uint4 *>(dispatch_smem + ((tw + 31) & ~size_t(31)));
+    uint4 *s_rows = reinterpret_cast<uint4 *>(bulk_smem + ((tw + 31) & ~size_t(31)));
     const bool early = a.C == 0;
     if (!row_cta && tid == 0) {
         mbar_init(&s_bar, 1);
