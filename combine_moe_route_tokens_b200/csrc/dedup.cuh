@@ -7,23 +7,20 @@
 // with probs. The combine comes back in two levels: every rank reduces its
 // local slots per received token, the sender sums the partials over ranks.
 //
-// dedup_layout_kernel (one cooperative launch, bounded grid barrier):
-//   phase 1  each lane builds, for its tokens, the bit set of ranks holding a
-//            kept slot (register-resident); per warp and rank the tokens are
-//            counted with __ballot_sync; the block publishes per-rank totals;
-//   phase 2  every block reads all block totals (one batch of loads), scans
-//            them into rank offsets, and places each (token, rank) pair at
-//            offset + earlier blocks + earlier warps + earlier lanes of the
-//            same rank (so rows are rank-major and token-ascending).
-// dedup_fill_kernel then writes the receive-side ids, weights, multihot map
-// and probs row by row over the whole GPU (they are a function of the row).
+// dedup_count_kernel (blocks in ticket order, any grid size): each (token,
+//            rank) pair's position among the tokens rank r receives, from
+//            per-warp ballots and a decoupled look-back over the blocks' per-rank
+//            counts (rows are rank-major and token-ascending);
+// dedup_fill_kernel (one thread per pair and per receive row): the rank
+//            offsets from the per-rank totals, the receive rows and their data
+//            (ids, weights, multihot map, probs), the tail rows.
 #pragma once
 
 #include <cstdint>
 
 #include "moe_rt.h"
 #include "combine.cuh"
-#include "grid_barrier.cuh"
+#include "lookback.cuh"
 #include "ptx.cuh"
 
 namespace moert {
@@ -32,6 +29,7 @@ constexpr int DEDUP_THREADS = 256;
 constexpr int DEDUP_WARPS = DEDUP_THREADS / 32;
 constexpr int DEDUP_MAX_BLOCKS = 128;
 constexpr int DEDUP_MAX_TPL = 8; // tokens per lane kept in registers
+constexpr int LB_CHUNK_DEDUP = 16; // predecessors one thread reads per look-back round
 
 struct DedupArgs {
     const int32_t *phys_idx; // [N, k]
@@ -40,10 +38,10 @@ struct DedupArgs {
     int64_t N;
     int64_t recv_max;
     int32_t k, R, E_loc;
-    int32_t G;
-    int32_t *ws_counts;   // [G][R]
-    uint32_t *ws_barrier; // [3] as in the layout: ticket word, unused, error bits
-    uint64_t barrier_limit_ns;
+    int32_t G;                     // count blocks
+    unsigned long long *ws_ticket; // ticket word (lookback.cuh)
+    unsigned long long *ws_flags;  // [G][R] look-back words
+    uint64_t wait_limit_ns;
     moe_dedup_t out;
 };
 
@@ -54,27 +52,47 @@ __device__ __forceinline__ uint32_t dedup_lanemask_lt()
     return m;
 }
 
+// The count pass: blocks in ticket order (lookback.cuh). Each lane builds, for
+// its tokens, the bit set of ranks holding a kept slot; per warp and rank the
+// tokens are counted with __ballot_sync; per rank the block publishes its count
+// and looks back over its predecessors (the same decoupled look-back as the
+// dispatch layout, R columns). Every (token, rank) pair gets its position among
+// rank r's tokens (earlier blocks + earlier warps + earlier lanes), written into
+// token_rank_row as a rank-relative row; dedup_fill_kernel adds the rank's offset.
 template <int TPL> // tokens per lane; a warp owns 32 * TPL consecutive tokens
-__global__ void __launch_bounds__(DEDUP_THREADS) dedup_layout_kernel(DedupArgs a)
+__global__ void __launch_bounds__(DEDUP_THREADS) dedup_count_kernel(DedupArgs a)
 {
+    constexpr int W = LB_CHUNK_DEDUP;
     __shared__ uint32_t s_wcnt[DEDUP_WARPS][MOE_MAX_DEDUP_RANKS]; // per-warp counts, then exclusive prefixes
-    __shared__ int32_t s_part[2][DEDUP_THREADS];
-    __shared__ int32_t s_pre[MOE_MAX_DEDUP_RANKS];
-    __shared__ int32_t s_off[MOE_MAX_DEDUP_RANKS + 1];
+    __shared__ uint32_t s_agg[MOE_MAX_DEDUP_RANKS], s_excl[MOE_MAX_DEDUP_RANKS], s_state[MOE_MAX_DEDUP_RANKS];
+    __shared__ uint32_t s_psum[DEDUP_THREADS], s_pflag[DEDUP_THREADS];
+    __shared__ uint32_t s_vb, s_epoch, s_timeout;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int b = blockIdx.x;
     const int R = a.R, k = a.k;
+    const int P = DEDUP_THREADS / R > 32 ? 32 : DEDUP_THREADS / R; // look-back parts per rank
     const uint32_t lt = dedup_lanemask_lt();
 
     for (int i = tid; i < DEDUP_WARPS * MOE_MAX_DEDUP_RANKS; i += DEDUP_THREADS)
         (&s_wcnt[0][0])[i] = 0;
+    if (tid == 0) { // drawn before the wait, as in the dispatch layout's count pass
+        uint32_t vb, epoch;
+        lb_take_ticket(a.ws_ticket, static_cast<uint32_t>(a.G), &vb, &epoch);
+        s_vb = vb;
+        s_epoch = epoch;
+        s_timeout = 0;
+    }
+    pdl_wait();
     __syncthreads();
     pdl_trigger();
-    pdl_wait();
+    const uint32_t vb = s_vb, epoch = s_epoch;
+    if (vb >= static_cast<uint32_t>(a.G)) { // two calls shared the workspace at once: stay inside it
+        if (tid == 0)
+            atomicOr(a.out.status, MOE_DEV_TIMEOUT);
+        return;
+    }
+    const int64_t base = (static_cast<int64_t>(vb) * DEDUP_WARPS + warp) * (32 * TPL);
 
-    const int64_t base = (static_cast<int64_t>(b) * DEDUP_WARPS + warp) * (32 * TPL);
-
-    // ---- phase 1: rank sets of this lane's tokens, per-warp per-rank counts
+    // ---- rank sets of this lane's tokens, per-warp per-rank counts
     uint32_t mask[TPL];
 #pragma unroll
     for (int u = 0; u < TPL; ++u) {
@@ -98,6 +116,7 @@ __global__ void __launch_bounds__(DEDUP_THREADS) dedup_layout_kernel(DedupArgs a
                 s_wcnt[warp][r] += __popc(bal);
         }
     __syncthreads();
+    unsigned long long *my_words = a.ws_flags + static_cast<int64_t>(vb) * R;
     if (tid < R) {
         uint32_t run = 0;
 #pragma unroll
@@ -106,70 +125,53 @@ __global__ void __launch_bounds__(DEDUP_THREADS) dedup_layout_kernel(DedupArgs a
             s_wcnt[w][tid] = run;
             run += c;
         }
-        a.ws_counts[static_cast<int64_t>(b) * R + tid] = static_cast<int32_t>(run);
+        s_agg[tid] = run;
+        s_excl[tid] = 0;
+        s_state[tid] = 0;
+        st_relaxed_u64(my_words + tid, lb_word(epoch, vb == 0 ? LB_INCL : LB_AGG, run, false));
     }
+    __syncthreads();
 
-    if (!grid_barrier_ticket(a.ws_barrier, static_cast<uint32_t>(a.G), 0u, a.barrier_limit_ns)) {
-        if (tid == 0)
+    // ---- decoupled look-back over the R rank columns
+    if (vb > 0) {
+        int32_t hi = static_cast<int32_t>(vb) - 1;
+        for (;;) {
+            if (tid < P * R) {
+                const int r = tid % R, part = tid / R;
+                if (!(s_state[r] & 1u)) {
+                    const LbChunk c = lb_scan_chunk<W>(a.ws_flags, R, r, hi - part * W, epoch, a.wait_limit_ns);
+                    s_psum[tid] = c.sum;
+                    s_pflag[tid] = c.closed ? 1u : 0u;
+                    if (c.timeout)
+                        s_timeout = 1;
+                }
+            }
+            __syncthreads();
+            int more = 0;
+            if (tid < R && !(s_state[tid] & 1u)) {
+                uint32_t sum = s_excl[tid];
+                for (int part = 0; part < P; ++part) {
+                    sum += s_psum[part * R + tid];
+                    if (s_pflag[part * R + tid]) {
+                        s_state[tid] = 1u;
+                        break;
+                    }
+                }
+                s_excl[tid] = sum;
+                if (s_state[tid] & 1u)
+                    st_relaxed_u64(my_words + tid, lb_word(epoch, LB_INCL, sum + s_agg[tid], false));
+                else
+                    more = 1;
+            }
+            hi -= P * W;
+            if (!__syncthreads_or(more))
+                break;
+        }
+        if (tid == 0 && s_timeout)
             atomicOr(a.out.status, MOE_DEV_TIMEOUT);
-        return;
     }
 
-    // ---- phase 2a: earlier-block prefix and total per rank (P threads per rank)
-    const int P = DEDUP_THREADS / R;
-    if (tid < P * R) {
-        const int r = tid % R, part = tid / R;
-        int32_t pre = 0, tot = 0;
-        for (int bb0 = part; bb0 < a.G; bb0 += 16 * P) {
-            int32_t c[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int bb = bb0 + u * P;
-                c[u] = bb < a.G ? __ldcg(a.ws_counts + static_cast<int64_t>(bb) * R + r) : 0;
-            }
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                tot += c[u];
-                pre += (bb0 + u * P < b) ? c[u] : 0;
-            }
-        }
-        s_part[0][tid] = pre;
-        s_part[1][tid] = tot;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        int32_t pre = 0, tot = 0;
-        if (lane < R)
-            for (int part = 0; part < P; ++part) {
-                pre += s_part[0][part * R + lane];
-                tot += s_part[1][part * R + lane];
-            }
-        int32_t inc = tot; // exclusive scan of the rank totals over the warp
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int32_t n = __shfl_up_sync(0xffffffffu, inc, o);
-            if (lane >= o)
-                inc += n;
-        }
-        if (lane < R) {
-            s_pre[lane] = pre;
-            s_off[lane] = inc - tot;
-        }
-        if (lane == R - 1)
-            s_off[R] = inc;
-        if (b == 0 && lane < R) {
-            a.out.num_tokens_per_rank[lane] = tot;
-            a.out.recv_rank_offsets[lane] = inc - tot;
-            if (lane == R - 1) {
-                a.out.recv_rank_offsets[R] = inc;
-                *a.out.num_recv = inc;
-            }
-        }
-    }
-    __syncthreads();
-
-    // ---- phase 2b: the row of each of this lane's (token, rank) pairs; the
-    // per-row receive data is written row by row by dedup_fill_kernel
+    // ---- each (token, rank) pair's position among rank r's tokens
     const moe_dedup_t &o = a.out;
 #pragma unroll
     for (int u = 0; u < TPL; ++u) {
@@ -177,119 +179,211 @@ __global__ void __launch_bounds__(DEDUP_THREADS) dedup_layout_kernel(DedupArgs a
         for (int r = 0; r < R; ++r) {
             const bool in = (mask[u] >> r) & 1u;
             const uint32_t bal = __ballot_sync(0xffffffffu, in);
-            const int32_t row = in ? s_off[r] + s_pre[r] + static_cast<int32_t>(s_wcnt[warp][r]) + __popc(bal & lt)
-                                   : -1;
+            const int32_t rel = in ? static_cast<int32_t>(s_excl[r] + s_wcnt[warp][r] + __popc(bal & lt)) : -1;
             __syncwarp();
             if (lane == 0)
                 s_wcnt[warp][r] += __popc(bal);
             __syncwarp();
             if (t >= a.N)
                 continue;
-            o.token_rank_row[t * R + r] = row;
+            o.token_rank_row[t * R + r] = rel;
             o.is_token_in_rank[t * R + r] = in ? 1 : 0;
-            if (!in)
-                continue;
-            if (row >= a.recv_max) { // cannot happen for consistent inputs; never write out of bounds
-                atomicOr(o.status, MOE_DEV_ROW_RANGE);
-                continue;
-            }
-            o.recv_src_token[row] = static_cast<int32_t>(t);
         }
     }
 }
 
-// Per receive row (one thread each): rank from recv_rank_offsets, then the
-// rank-local top-k ids and weights of the source token, the multihot map and
-// its probs; tail rows get -1 / 0 and pad 1. Rows past num_recv are tail rows;
-// recv_src_token of those rows is written here too.
+// The fill pass: a group of DEDUP_FILL_LANES threads per (rank, token) pair
+// (pairs rank-major, so neighbouring groups write neighbouring rows) and per
+// receive row. Every CTA turns the last count block's inclusive words (the
+// per-rank token totals) into rank offsets; CTA 0 writes them out. A pair that
+// sends its token to rank r turns its rank-relative row into the receive row w
+// and writes that row's data: the source token, the rank-local top-k ids and
+// weights, the multihot map with its probs (Megatron MORI page:
+// _indices_to_multihot), pad 0. Each lane of the group holds some of the
+// token's slots; the map and prob rows are split among the lanes, each lane
+// builds its part from the slots (shuffled within the group) and stores it
+// once. Rows past num_recv are tail rows: token -1, ids -1, weights / map /
+// probs 0, pad 1.
+constexpr int DEDUP_FILL_LANES = 8;
+constexpr int DEDUP_FILL_THREADS = 256;
+
 struct DedupFillArgs {
     const int32_t *phys_idx; // [N, k]
     const int32_t *dest_row; // [N, k]
     const float *probs;      // [N, k] or null
+    int64_t N;
     int64_t recv_max;
-    int32_t k, R, E_loc;
+    int32_t k, R, E_loc, G;
+    const unsigned long long *ws_ticket;
+    const unsigned long long *ws_flags;
     moe_dedup_t out;
 };
 
-__global__ void __launch_bounds__(256) dedup_fill_kernel(DedupFillArgs a)
+// Row w's ids, weights, map and probs from the (local id, weight) of the token's
+// slots held by the group's lanes (slot j on lane j % LANES, register j / LANES);
+// local -1 marks a slot that is not on this rank (or a tail row).
+__device__ __forceinline__ void dedup_write_row(const DedupFillArgs &a, int64_t w, const int32_t (&loc)[4],
+                                                const float (&wt)[4], int gl, uint32_t gmask)
+{
+    const moe_dedup_t &o = a.out;
+    const int k = a.k, E_loc = a.E_loc;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int j = u * DEDUP_FILL_LANES + gl;
+        if (j < k) {
+            o.recv_topk_idx[w * k + j] = loc[u];
+            o.recv_topk_weights[w * k + j] = wt[u];
+        }
+    }
+    uint8_t *map_row = o.recv_routing_map + w * E_loc;
+    float *prob_row = o.recv_probs + w * E_loc;
+    const int nu = (k + DEDUP_FILL_LANES - 1) / DEDUP_FILL_LANES;
+    // every lane of the group runs the same iterations (the shuffles need all of them)
+    if ((E_loc & 3) == 0) { // four entries at a time: one 16-byte prob store and one 4-byte map store
+        for (int c0 = 0; c0 < E_loc; c0 += DEDUP_FILL_LANES * 4) {
+            const int c = c0 + gl * 4;
+            float4 pv = make_float4(0.f, 0.f, 0.f, 0.f);
+            uint32_t mv = 0;
+            for (int u = 0; u < nu; ++u)
+                for (int sl = 0; sl < DEDUP_FILL_LANES; ++sl) {
+                    const int32_t x = __shfl_sync(gmask, loc[u], sl, DEDUP_FILL_LANES);
+                    const float y = __shfl_sync(gmask, wt[u], sl, DEDUP_FILL_LANES);
+                    const int off = x - c;
+                    if (x >= 0 && off >= 0 && off < 4) {
+                        mv |= 1u << (8 * off);
+                        if (off == 0)
+                            pv.x = y;
+                        else if (off == 1)
+                            pv.y = y;
+                        else if (off == 2)
+                            pv.z = y;
+                        else
+                            pv.w = y;
+                    }
+                }
+            if (c < E_loc) {
+                *reinterpret_cast<float4 *>(prob_row + c) = pv;
+                *reinterpret_cast<uint32_t *>(map_row + c) = mv;
+            }
+        }
+    } else {
+        for (int c0 = 0; c0 < E_loc; c0 += DEDUP_FILL_LANES) {
+            const int c = c0 + gl;
+            float pv = 0.0f;
+            uint8_t mv = 0;
+            for (int u = 0; u < nu; ++u)
+                for (int sl = 0; sl < DEDUP_FILL_LANES; ++sl) {
+                    const int32_t x = __shfl_sync(gmask, loc[u], sl, DEDUP_FILL_LANES);
+                    const float y = __shfl_sync(gmask, wt[u], sl, DEDUP_FILL_LANES);
+                    if (x == c) {
+                        mv = 1;
+                        pv = y;
+                    }
+                }
+            if (c < E_loc) {
+                prob_row[c] = pv;
+                map_row[c] = mv;
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(DEDUP_FILL_THREADS) dedup_fill_kernel(DedupFillArgs a)
 {
     __shared__ int32_t s_roff[MOE_MAX_DEDUP_RANKS + 1];
     pdl_trigger();
-    pdl_wait();
+    pdl_wait(); // the count pass is complete
     const moe_dedup_t &o = a.out;
-    if (threadIdx.x <= a.R)
-        s_roff[threadIdx.x] = __ldg(o.recv_rank_offsets + threadIdx.x);
+    const int tid = threadIdx.x, R = a.R, k = a.k;
+    if (tid < 32) { // rank totals from the last block's inclusive words, then their exclusive scan
+        const uint32_t epoch = static_cast<uint32_t>(__ldcg(a.ws_ticket) >> 32) - 1u;
+        int32_t tot = 0;
+        bool ok = true;
+        if (tid < R) {
+            const uint64_t w = __ldcg(a.ws_flags + static_cast<int64_t>(a.G - 1) * R + tid);
+            ok = lb_ready(w, epoch) && lb_incl(w);
+            tot = ok ? static_cast<int32_t>(lb_value(w)) : 0;
+        }
+        if (__any_sync(0xffffffffu, !ok) && tid == 0 && blockIdx.x == 0)
+            atomicOr(o.status, MOE_DEV_TIMEOUT);
+        int32_t inc = tot;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int32_t n = __shfl_up_sync(0xffffffffu, inc, d);
+            if (tid >= d)
+                inc += n;
+        }
+        if (tid < R)
+            s_roff[tid] = inc - tot;
+        if (tid == R - 1)
+            s_roff[R] = inc;
+        if (blockIdx.x == 0 && tid < R) {
+            o.num_tokens_per_rank[tid] = tot;
+            o.recv_rank_offsets[tid] = inc - tot;
+            if (tid == R - 1) {
+                o.recv_rank_offsets[R] = inc;
+                *o.num_recv = inc;
+            }
+        }
+    }
     __syncthreads();
-    const int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (w >= a.recv_max)
+    const int gl = tid % DEDUP_FILL_LANES; // lane within the group
+    const uint32_t gmask = 0xFFu << ((tid & 31) & ~(DEDUP_FILL_LANES - 1));
+    const int64_t g = (static_cast<int64_t>(blockIdx.x) * DEDUP_FILL_THREADS + tid) / DEDUP_FILL_LANES;
+    const int32_t num_recv = s_roff[R];
+    int32_t loc[4];
+    float wt[4];
+    if (g < a.recv_max && g >= num_recv) { // a tail row
+        if (gl == 0) {
+            o.recv_src_token[g] = -1;
+            o.recv_pad_mask[g] = 1;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            loc[u] = -1;
+            wt[u] = 0.0f;
+        }
+        dedup_write_row(a, g, loc, wt, gl, gmask);
+    }
+    if (g >= a.N * R) // uniform over the group
         return;
-    const int32_t num_recv = s_roff[a.R];
-    const int k = a.k, E_loc = a.E_loc;
-    int32_t t = -1, r = -1;
-    if (w < num_recv) {
-        t = __ldg(o.recv_src_token + w);
-        r = 0;
-        while (r + 1 < a.R && s_roff[r + 1] <= w)
-            ++r;
-    } else {
-        o.recv_src_token[w] = -1;
+    // pairs rank-major: neighbouring groups take neighbouring tokens of one rank, whose
+    // rows are neighbours too
+    const int r = static_cast<int>(g / a.N);
+    const int64_t t = g - static_cast<int64_t>(r) * a.N;
+    const int64_t pair = t * R + r;
+    const int32_t rel = __ldcg(o.token_rank_row + pair);
+    if (rel < 0)
+        return;
+    const int64_t w = static_cast<int64_t>(s_roff[r]) + rel;
+    if (w >= a.recv_max || w >= s_roff[r + 1]) { // cannot happen for consistent counts; never write out of bounds
+        if (gl == 0) {
+            atomicOr(o.status, MOE_DEV_ROW_RANGE);
+            o.token_rank_row[pair] = -1;
+        }
+        return;
     }
-    o.recv_pad_mask[w] = t < 0 ? 1 : 0;
-    uint8_t *map_row = o.recv_routing_map + w * E_loc;
-    float *prob_row = o.recv_probs + w * E_loc;
-    // the token's slots, eight at a time, all loads of a batch in flight together
-    // (the first batch before the row is zeroed, so that nothing waits in between)
-    constexpr int B = 8;
-    int32_t dj[B], qj[B];
-    float wj[B];
-    auto load_batch = [&](int j0) {
 #pragma unroll
-        for (int u = 0; u < B; ++u) {
-            const int j = j0 + u;
-            dj[u] = -1;
-            qj[u] = -1;
-            wj[u] = 0.0f;
-            if (t >= 0 && j < k) {
-                const int64_t s = static_cast<int64_t>(t) * k + j;
-                dj[u] = __ldg(a.dest_row + s);
-                qj[u] = __ldg(a.phys_idx + s);
-                if (a.probs != nullptr)
-                    wj[u] = __ldg(a.probs + s);
+    for (int u = 0; u < 4; ++u) { // this lane's slots of the token: local id on rank r and weight
+        const int j = u * DEDUP_FILL_LANES + gl;
+        loc[u] = -1;
+        wt[u] = 0.0f;
+        if (j < k) {
+            const int64_t sidx = t * k + j;
+            const int32_t d = __ldg(a.dest_row + sidx);
+            const int32_t q = __ldg(a.phys_idx + sidx);
+            if (d >= 0 && q >= 0 && q / a.E_loc == r) {
+                loc[u] = q - r * a.E_loc;
+                wt[u] = a.probs != nullptr ? __ldg(a.probs + sidx) : 0.0f;
             }
         }
-    };
-    load_batch(0);
-    if ((E_loc & 15) == 0) {
-        for (int c = 0; c < E_loc; c += 16)
-            *reinterpret_cast<uint4 *>(map_row + c) = make_uint4(0, 0, 0, 0);
-        for (int c = 0; c < E_loc; c += 4)
-            *reinterpret_cast<float4 *>(prob_row + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-    } else {
-        for (int c = 0; c < E_loc; ++c) {
-            map_row[c] = 0;
-            prob_row[c] = 0.0f;
-        }
     }
-    for (int j0 = 0; j0 < k; j0 += B) {
-        if (j0 > 0)
-            load_batch(j0);
-#pragma unroll
-        for (int u = 0; u < B; ++u) {
-            const int j = j0 + u;
-            if (j >= k)
-                break;
-            int32_t local = -1;
-            float wt = 0.0f;
-            if (dj[u] >= 0 && qj[u] >= 0 && qj[u] / E_loc == r) {
-                local = qj[u] - r * E_loc;
-                wt = wj[u];
-                map_row[local] = 1;
-                prob_row[local] = wt;
-            }
-            o.recv_topk_idx[w * k + j] = local;
-            o.recv_topk_weights[w * k + j] = wt;
-        }
+    if (gl == 0) {
+        o.token_rank_row[pair] = static_cast<int32_t>(w);
+        o.recv_src_token[w] = static_cast<int32_t>(t);
+        o.recv_pad_mask[w] = 0;
     }
+    dedup_write_row(a, w, loc, wt, gl, gmask);
 }
 
 // Receiver-side partials, token-major: one thread per 16-byte column chunk of

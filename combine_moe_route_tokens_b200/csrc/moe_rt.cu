@@ -36,8 +36,7 @@ using namespace moert;
 
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;     // 1 s: every device-side wait gives up after this
 constexpr uint64_t TEST_WAIT_LIMIT_NS = 10000000ull;  // 10 ms for MOE_FLAG_TEST_WAIT_TIMEOUT
-constexpr size_t WS_BARRIER_BYTES = 256;  // dedup layout: grid barrier words
-constexpr size_t WS_TICKET_BYTES = 256;   // dispatch layout: the ticket word, then the look-back words
+constexpr size_t WS_TICKET_BYTES = 256; // layout workspaces: the ticket word, then the look-back words
 
 using LayoutKernel = void (*)(LayoutArgs);
 using DispatchKernel = void (*)(DispatchArgs);
@@ -109,29 +108,20 @@ struct NvtxRange {
     NvtxRange &operator=(const NvtxRange &) = delete;
 };
 
-// Programmatic dependent launch is used unless the driver refuses it for a
-// kind of launch; then that kind falls back to ordinary stream order.
-std::atomic<bool> g_pdl_plain{true};
-std::atomic<bool> g_pdl_coop{true};
+// Programmatic dependent launch is used unless the driver refuses it; then
+// launches fall back to ordinary stream order.
+std::atomic<bool> g_pdl_ok{true};
 
 // Every kernel goes through cudaLaunchKernelEx with programmatic stream
 // serialization, so its launch overlaps the tail of the previous kernel in the
-// stream (each kernel calls pdl_wait() before reading anything); cooperative
-// kernels add the cooperative attribute.
+// stream (each kernel calls pdl_wait() before reading anything a predecessor
+// may have written).
 template <typename... KArgs, typename... Args>
-int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, void *stream, bool cooperative,
-           Args... args)
+int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, void *stream, Args... args)
 {
-    std::atomic<bool> &pdl_ok = cooperative ? g_pdl_coop : g_pdl_plain;
-    cudaLaunchAttribute attrs[2];
+    cudaLaunchAttribute attrs[1];
     unsigned n = 0;
-    if (cooperative) {
-        attrs[n].id = cudaLaunchAttributeCooperative;
-        attrs[n].val.cooperative = 1;
-        ++n;
-    }
-    const unsigned n_base = n;
-    if (pdl_ok.load(std::memory_order_relaxed)) {
+    if (g_pdl_ok.load(std::memory_order_relaxed)) {
         attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attrs[n].val.programmaticStreamSerializationAllowed = 1;
         ++n;
@@ -144,14 +134,14 @@ int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, void *s
     cfg.attrs = attrs;
     cfg.numAttrs = n;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
-    if (e != cudaSuccess && n > n_base) {
+    if (e != cudaSuccess && n > 0) {
         // retry without the programmatic attribute; only if that launch succeeds was the
-        // attribute the cause, and only then is it dropped for later launches of this kind
+        // attribute the cause, and only then is it dropped for later launches
         (void)cudaGetLastError();
-        cfg.numAttrs = n_base;
+        cfg.numAttrs = 0;
         e = cudaLaunchKernelEx(&cfg, kernel, args...);
         if (e == cudaSuccess)
-            pdl_ok.store(false, std::memory_order_relaxed);
+            g_pdl_ok.store(false, std::memory_order_relaxed);
     }
     if (e != cudaSuccess) {
         (void)cudaGetLastError();
@@ -415,7 +405,7 @@ int moe_route_topk(const float *logits, const uint8_t *token_mask, int64_t N, in
     const dim3 grid(static_cast<unsigned>(blocks64)), block(ROUTE_WARPS_PER_BLOCK * 32);
     const int vpl = (E + 31) / 32;
     auto go = [&](auto kernel) {
-        return launch(kernel, grid, block, 0, stream, false, logits, token_mask, N, E, k, topk_idx, topk_probs);
+        return launch(kernel, grid, block, 0, stream, logits, token_mask, N, E, k, topk_idx, topk_probs);
     };
     if (vpl <= 1)
         return go(route_topk_kernel<1>);
@@ -513,12 +503,11 @@ int moe_dispatch_layout(const moe_problem_t *problem, const int32_t *topk_idx, c
         return MOE_ERR_UNSUPPORTED;
     const bool reroute = problem->num_replicas > 0;
     const bool dense = problem->capacity == 0 && d.A == 1;
-    rc = launch(layout_count_for(lg.ipl), dim3(lg.G), dim3(LAYOUT_THREADS), layout_count_smem_words(a.E_log) * 4,
-                stream, false, a);
+    rc = launch(layout_count_for(lg.ipl), dim3(lg.G), dim3(LAYOUT_THREADS), layout_count_smem_words(a.E_log) * 4, stream, a);
     if (rc != MOE_OK)
         return rc;
     return launch(layout_fill_for(reroute, dense), dim3(static_cast<unsigned>(fill_blocks)), dim3(FILL_THREADS),
-                  layout_tables_smem_words(a.E_log, a.E) * 4, stream, false, a);
+                  layout_tables_smem_words(a.E_log, a.E) * 4, stream, a);
 }
 
 int moe_dispatch(const moe_problem_t *problem, const int32_t *topk_idx, const float *topk_probs,
@@ -579,10 +568,10 @@ int moe_dispatch(const moe_problem_t *problem, const int32_t *topk_idx, const fl
     if (blocks > INT32_MAX)
         return MOE_ERR_UNSUPPORTED;
     rc = launch(layout_count_for(lg.ipl), dim3(lg.G), dim3(LAYOUT_THREADS),
-                layout_count_smem_words(problem->E_log) * 4, stream, false, da.L);
+                layout_count_smem_words(problem->E_log) * 4, stream, da.L);
     if (rc != MOE_OK)
         return rc;
-    return launch(kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), smem, stream, false, da);
+    return launch(kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), smem, stream, da);
 }
 
 int moe_permute(const moe_problem_t *problem, const moe_layout_t *layout, const uint16_t *hidden, uint16_t *send,
@@ -623,7 +612,7 @@ int moe_permute(const moe_problem_t *problem, const moe_layout_t *layout, const 
     const int64_t blocks = a.zero_blocks + (problem->N * a.pieces + groups - 1) / groups;
     if (blocks > INT32_MAX)
         return MOE_ERR_UNSUPPORTED;
-    return launch(permute_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(PERMUTE_THREADS), 0, stream, false, a);
+    return launch(permute_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(PERMUTE_THREADS), 0, stream, a);
 }
 
 namespace {
@@ -648,8 +637,8 @@ int launch_combine_args(CombineArgs a, int k, void *stream)
                 return MOE_ERR_UNSUPPORTED;
             const dim3 grid(static_cast<unsigned>(blocks)), block(COMBINE_THREADS);
             if (k == 1)
-                return launch(combine_rows_kernel<1>, grid, block, 0, stream, false, a);
-            return launch(combine_rows_kernel<2>, grid, block, 0, stream, false, a);
+                return launch(combine_rows_kernel<1>, grid, block, 0, stream, a);
+            return launch(combine_rows_kernel<2>, grid, block, 0, stream, a);
         }
     }
     // the widest CTA (up to 256 threads) that splits the row into equal parts
@@ -662,17 +651,17 @@ int launch_combine_args(CombineArgs a, int k, void *stream)
     const dim3 grid(static_cast<unsigned>(blocks)), block(threads);
     switch (k) {
     case 1:
-        return launch(combine_kernel<1, SRC>, grid, block, 0, stream, false, a);
+        return launch(combine_kernel<1, SRC>, grid, block, 0, stream, a);
     case 2:
-        return launch(combine_kernel<2, SRC>, grid, block, 0, stream, false, a);
+        return launch(combine_kernel<2, SRC>, grid, block, 0, stream, a);
     case 4:
-        return launch(combine_kernel<4, SRC>, grid, block, 0, stream, false, a);
+        return launch(combine_kernel<4, SRC>, grid, block, 0, stream, a);
     case 6:
-        return launch(combine_kernel<6, SRC>, grid, block, 0, stream, false, a);
+        return launch(combine_kernel<6, SRC>, grid, block, 0, stream, a);
     case 8:
-        return launch(combine_kernel<8, SRC>, grid, block, 0, stream, false, a);
+        return launch(combine_kernel<8, SRC>, grid, block, 0, stream, a);
     default:
-        return launch(combine_kernel<0, SRC>, grid, block, 0, stream, false, a);
+        return launch(combine_kernel<0, SRC>, grid, block, 0, stream, a);
     }
 }
 
@@ -774,7 +763,7 @@ int moe_dedup_workspace_bytes(const moe_problem_t *problem, size_t *bytes)
         return rc;
     if (bytes == nullptr)
         return MOE_ERR_INVALID;
-    *bytes = WS_BARRIER_BYTES + static_cast<size_t>(DEDUP_MAX_BLOCKS) * problem->R * 4;
+    *bytes = WS_TICKET_BYTES + static_cast<size_t>(DEDUP_MAX_BLOCKS) * problem->R * 8;
     return MOE_OK;
 }
 
@@ -800,14 +789,12 @@ int moe_dedup_layout(const moe_problem_t *problem, const moe_layout_t *layout, c
                          o->recv_topk_weights == nullptr || o->recv_routing_map == nullptr ||
                          o->recv_probs == nullptr || o->recv_pad_mask == nullptr))
         return MOE_ERR_INVALID;
-    if (recv_max > 0 && (d.E_loc & 15) == 0 && (!aligned16(o->recv_routing_map) || !aligned16(o->recv_probs)))
+    if (recv_max > 0 && (d.E_loc & 3) == 0 &&
+        (!aligned16(o->recv_probs) || (reinterpret_cast<uintptr_t>(o->recv_routing_map) & 3u) != 0))
         return MOE_ERR_INVALID;
     if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
-        workspace_bytes < WS_BARRIER_BYTES + static_cast<size_t>(DEDUP_MAX_BLOCKS) * problem->R * 4)
+        workspace_bytes < WS_TICKET_BYTES + static_cast<size_t>(DEDUP_MAX_BLOCKS) * problem->R * 8)
         return MOE_ERR_INVALID;
-    DeviceInfo dev;
-    if ((rc = device_info(&dev)) != MOE_OK)
-        return rc;
     int tpl = 1;
     while (tpl <= DEDUP_MAX_TPL &&
            (problem->N + static_cast<int64_t>(DEDUP_THREADS) * tpl - 1) / (static_cast<int64_t>(DEDUP_THREADS) * tpl) >
@@ -818,7 +805,10 @@ int moe_dedup_layout(const moe_problem_t *problem, const moe_layout_t *layout, c
     int64_t G = (problem->N + static_cast<int64_t>(DEDUP_THREADS) * tpl - 1) / (static_cast<int64_t>(DEDUP_THREADS) * tpl);
     if (G < 1)
         G = 1;
-    if (G > dev.sms)
+    const int64_t pairs = problem->N * problem->R;
+    const int64_t fill_items = (pairs > recv_max ? pairs : recv_max) * DEDUP_FILL_LANES; // a group per pair and row
+    const int64_t fill_blocks = fill_items > 0 ? (fill_items + DEDUP_FILL_THREADS - 1) / DEDUP_FILL_THREADS : 1;
+    if (fill_blocks > INT32_MAX)
         return MOE_ERR_UNSUPPORTED;
     DedupArgs a;
     a.phys_idx = layout->phys_idx;
@@ -830,40 +820,42 @@ int moe_dedup_layout(const moe_problem_t *problem, const moe_layout_t *layout, c
     a.R = problem->R;
     a.E_loc = d.E_loc;
     a.G = static_cast<int32_t>(G);
-    a.ws_barrier = static_cast<uint32_t *>(workspace);
-    a.ws_counts = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + WS_BARRIER_BYTES);
-    a.barrier_limit_ns = WAIT_LIMIT_NS;
+    a.ws_ticket = static_cast<unsigned long long *>(workspace);
+    a.ws_flags = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(workspace) + WS_TICKET_BYTES);
+    a.wait_limit_ns = WAIT_LIMIT_NS;
     a.out = *o;
     const dim3 grid(static_cast<unsigned>(G)), block(DEDUP_THREADS);
     switch (tpl) {
     case 1:
-        rc = launch(dedup_layout_kernel<1>, grid, block, 0, stream, true, a);
+        rc = launch(dedup_count_kernel<1>, grid, block, 0, stream, a);
         break;
     case 2:
-        rc = launch(dedup_layout_kernel<2>, grid, block, 0, stream, true, a);
+        rc = launch(dedup_count_kernel<2>, grid, block, 0, stream, a);
         break;
     case 4:
-        rc = launch(dedup_layout_kernel<4>, grid, block, 0, stream, true, a);
+        rc = launch(dedup_count_kernel<4>, grid, block, 0, stream, a);
         break;
     default:
-        rc = launch(dedup_layout_kernel<8>, grid, block, 0, stream, true, a);
+        rc = launch(dedup_count_kernel<8>, grid, block, 0, stream, a);
         break;
     }
-    if (rc != MOE_OK || recv_max == 0)
+    if (rc != MOE_OK)
         return rc;
     DedupFillArgs f;
     f.phys_idx = layout->phys_idx;
     f.dest_row = layout->dest_row;
     f.probs = topk_probs;
+    f.N = problem->N;
     f.recv_max = recv_max;
     f.k = problem->k;
     f.R = problem->R;
     f.E_loc = d.E_loc;
+    f.G = a.G;
+    f.ws_ticket = a.ws_ticket;
+    f.ws_flags = a.ws_flags;
     f.out = *o;
-    const int64_t fill_blocks = (recv_max + 255) / 256;
-    if (fill_blocks > INT32_MAX)
-        return MOE_ERR_UNSUPPORTED;
-    return launch(dedup_fill_kernel, dim3(static_cast<unsigned>(fill_blocks)), dim3(256), 0, stream, false, f);
+    return launch(dedup_fill_kernel, dim3(static_cast<unsigned>(fill_blocks)), dim3(DEDUP_FILL_THREADS), 0, stream,
+                  f);
 }
 
 int moe_dedup_dispatch(const moe_problem_t *problem, const moe_dedup_t *dedup, const uint16_t *hidden,
@@ -906,7 +898,7 @@ int moe_dedup_dispatch(const moe_problem_t *problem, const moe_dedup_t *dedup, c
     const int64_t blocks = a.zero_blocks + (problem->N * a.pieces + groups - 1) / groups;
     if (blocks > INT32_MAX)
         return MOE_ERR_UNSUPPORTED;
-    return launch(permute_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(PERMUTE_THREADS), 0, stream, false, a);
+    return launch(permute_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(PERMUTE_THREADS), 0, stream, a);
 }
 
 int moe_dedup_combine_local(const moe_problem_t *problem, const moe_layout_t *layout, const moe_dedup_t *dedup,
@@ -962,17 +954,17 @@ int moe_dedup_combine_local(const moe_problem_t *problem, const moe_layout_t *la
     const dim3 grid(static_cast<unsigned>(blocks)), block(threads);
     switch (problem->k) {
     case 1:
-        return launch(dedup_combine_local_kernel<1>, grid, block, 0, stream, false, a);
+        return launch(dedup_combine_local_kernel<1>, grid, block, 0, stream, a);
     case 2:
-        return launch(dedup_combine_local_kernel<2>, grid, block, 0, stream, false, a);
+        return launch(dedup_combine_local_kernel<2>, grid, block, 0, stream, a);
     case 4:
-        return launch(dedup_combine_local_kernel<4>, grid, block, 0, stream, false, a);
+        return launch(dedup_combine_local_kernel<4>, grid, block, 0, stream, a);
     case 6:
-        return launch(dedup_combine_local_kernel<6>, grid, block, 0, stream, false, a);
+        return launch(dedup_combine_local_kernel<6>, grid, block, 0, stream, a);
     case 8:
-        return launch(dedup_combine_local_kernel<8>, grid, block, 0, stream, false, a);
+        return launch(dedup_combine_local_kernel<8>, grid, block, 0, stream, a);
     default:
-        return launch(dedup_combine_local_kernel<0>, grid, block, 0, stream, false, a);
+        return launch(dedup_combine_local_kernel<0>, grid, block, 0, stream, a);
     }
 }
 
@@ -1054,7 +1046,7 @@ int moe_ep_plan(const moe_problem_t *problem, const int32_t *offsets_all, int32_
     a.num_recv = num_recv;
     a.status = status;
     const size_t smem = (2 * static_cast<size_t>(d.E) + 1) * sizeof(int32_t);
-    return launch(ep_plan_kernel, dim3(1), dim3(EP_PLAN_THREADS), smem, stream, false, a);
+    return launch(ep_plan_kernel, dim3(1), dim3(EP_PLAN_THREADS), smem, stream, a);
 }
 
 int moe_ep_publish_offsets(const moe_problem_t *problem, const int32_t *expert_offsets, int32_t src_rank,
@@ -1077,8 +1069,7 @@ int moe_ep_publish_offsets(const moe_problem_t *problem, const int32_t *expert_o
     a.src = src_rank;
     const int64_t n = static_cast<int64_t>(a.R) * (a.E + 1);
     const int64_t blocks = (n + 255) / 256;
-    return launch(ep_publish_offsets_kernel, dim3(static_cast<unsigned>(blocks < 64 ? blocks : 64)), dim3(256), 0,
-                  stream, false, a);
+    return launch(ep_publish_offsets_kernel, dim3(static_cast<unsigned>(blocks < 64 ? blocks : 64)), dim3(256), 0, stream, a);
 }
 
 int moe_ep_dispatch(const moe_problem_t *problem, const moe_layout_t *layout, const int32_t *base,
@@ -1130,7 +1121,7 @@ int moe_ep_dispatch(const moe_problem_t *problem, const moe_layout_t *layout, co
     const int64_t blocks = a.zero_blocks + (problem->N * a.pieces + groups - 1) / groups;
     if (blocks > INT32_MAX)
         return MOE_ERR_UNSUPPORTED;
-    return launch(permute_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(PERMUTE_THREADS), 0, stream, false, a);
+    return launch(permute_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(PERMUTE_THREADS), 0, stream, a);
 }
 
 int moe_ep_combine(const moe_problem_t *problem, const moe_layout_t *layout, const int32_t *base,
@@ -1228,17 +1219,17 @@ int moe_ep_combine_backward(const moe_problem_t *problem, const moe_layout_t *la
     const dim3 grid(static_cast<unsigned>(blocks)), block(COMBINE_BWD_THREADS);
     switch (problem->k) {
     case 1:
-        return launch(combine_backward_kernel<1, true>, grid, block, 0, stream, false, a);
+        return launch(combine_backward_kernel<1, true>, grid, block, 0, stream, a);
     case 2:
-        return launch(combine_backward_kernel<2, true>, grid, block, 0, stream, false, a);
+        return launch(combine_backward_kernel<2, true>, grid, block, 0, stream, a);
     case 4:
-        return launch(combine_backward_kernel<4, true>, grid, block, 0, stream, false, a);
+        return launch(combine_backward_kernel<4, true>, grid, block, 0, stream, a);
     case 6:
-        return launch(combine_backward_kernel<6, true>, grid, block, 0, stream, false, a);
+        return launch(combine_backward_kernel<6, true>, grid, block, 0, stream, a);
     case 8:
-        return launch(combine_backward_kernel<8, true>, grid, block, 0, stream, false, a);
+        return launch(combine_backward_kernel<8, true>, grid, block, 0, stream, a);
     default:
-        return launch(combine_backward_kernel<0, true>, grid, block, 0, stream, false, a);
+        return launch(combine_backward_kernel<0, true>, grid, block, 0, stream, a);
     }
 }
 
@@ -1286,17 +1277,17 @@ int moe_combine_backward(const moe_problem_t *problem, const moe_layout_t *layou
     const dim3 grid(static_cast<unsigned>(blocks)), block(COMBINE_BWD_THREADS);
     switch (problem->k) {
     case 1:
-        return launch(combine_backward_kernel<1>, grid, block, 0, stream, false, a);
+        return launch(combine_backward_kernel<1>, grid, block, 0, stream, a);
     case 2:
-        return launch(combine_backward_kernel<2>, grid, block, 0, stream, false, a);
+        return launch(combine_backward_kernel<2>, grid, block, 0, stream, a);
     case 4:
-        return launch(combine_backward_kernel<4>, grid, block, 0, stream, false, a);
+        return launch(combine_backward_kernel<4>, grid, block, 0, stream, a);
     case 6:
-        return launch(combine_backward_kernel<6>, grid, block, 0, stream, false, a);
+        return launch(combine_backward_kernel<6>, grid, block, 0, stream, a);
     case 8:
-        return launch(combine_backward_kernel<8>, grid, block, 0, stream, false, a);
+        return launch(combine_backward_kernel<8>, grid, block, 0, stream, a);
     default:
-        return launch(combine_backward_kernel<0>, grid, block, 0, stream, false, a);
+        return launch(combine_backward_kernel<0>, grid, block, 0, stream, a);
     }
 }
 

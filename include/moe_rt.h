@@ -316,6 +316,8 @@ MOE_API int moe_restore_combined(const moe_problem_t *problem, const moe_layout_
  * (token, rank) pair, rank-major and token-ascending within a rank;
  * recv_max = N * min(k, R) rows, the rows past num_recv are tail rows
  * (token -1, ids -1, weights / map / probs 0, pad 1). R <= MOE_MAX_DEDUP_RANKS.
+ * When E_loc is a multiple of 4, recv_probs must be 16-byte and
+ * recv_routing_map 4-byte aligned (their rows are written four entries at a time).
  */
 #define MOE_MAX_DEDUP_RANKS 32
 
@@ -337,15 +339,18 @@ typedef struct {
 /* recv_max = N * min(k, R), or a negative MOE_ERR_* for an invalid problem. Host only. */
 MOE_API int64_t moe_dedup_rows_max(const moe_problem_t *problem);
 
-/* Scratch bytes of moe_dedup_layout (zero-filled before first use, as for the layout). Host only. */
+/* Scratch bytes of moe_dedup_layout (zero-filled once before first use, as for the layout;
+ * it then stays ready for every later call). Host only. */
 MOE_API int moe_dedup_workspace_bytes(const moe_problem_t *problem, size_t *bytes);
 
 /*
  * Build the dedup view from a dispatch layout (reads layout->phys_idx and
- * layout->dest_row: a slot counts where dest_row >= 0): one cooperative
- * launch with a bounded grid barrier places the (token, rank) pairs, a second
- * launch fills the per-row receive data. topk_probs [N, k] fp32 or NULL
- * (weights 0). Limits: R <= MOE_MAX_DEDUP_RANKS, N <= 262144.
+ * layout->dest_row: a slot counts where dest_row >= 0): a count pass whose
+ * blocks, in atomic-ticket order, rank the (token, rank) pairs with a decoupled
+ * look-back over their per-rank counts (no block waits for one that started
+ * after it), then a fill pass writes the receive rows and their data.
+ * topk_probs [N, k] fp32 or NULL (weights 0). Limits: R <= MOE_MAX_DEDUP_RANKS,
+ * N <= 262144.
  */
 MOE_API int moe_dedup_layout(const moe_problem_t *problem, const moe_layout_t *layout, const float *topk_probs,
                              const moe_dedup_t *dedup, void *workspace, size_t workspace_bytes, void *stream);
