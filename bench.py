@@ -282,13 +282,21 @@ class Step:
             if T == 1 and w.dedup:
                 ws = self.layout.workspace
                 D = ctypes.byref(self._D)
+                if unfused:
+                    c += [("layout", self.lib.moe_dispatch_layout,
+                           (P, vp(self.idx), vp(self.probs), L, vp(ws), ws.numel(), self._s))]
+                else:  # the layout and the send buffer in one call
+                    c += [("dispatch", self.lib.moe_dispatch,
+                           (P, vp(self.idx), vp(self.probs), L, vp(ws), ws.numel(), vp(s["hidden"]), vp(self.send),
+                            self._s))]
                 c += [
-                    ("layout", self.lib.moe_dispatch_layout,
-                     (P, vp(self.idx), vp(self.probs), L, vp(ws), ws.numel(), self._s)),
                     ("dedup_layout", self.lib.moe_dedup_layout,
                      (P, L, vp(self.probs), D, vp(self.dedup.workspace), self.dedup.workspace.numel(), self._s)),
                     ("dedup_dispatch", self.lib.moe_dedup_dispatch, (P, D, vp(s["hidden"]), vp(self.recv_x), self._s)),
-                    ("permute", self.lib.moe_permute, (P, L, vp(s["hidden"]), vp(self.send), self._s)),
+                ]
+                if unfused:
+                    c += [("permute", self.lib.moe_permute, (P, L, vp(s["hidden"]), vp(self.send), self._s))]
+                c += [
                     ("dedup_combine_local", self.lib.moe_dedup_combine_local,
                      (P, L, D, vp(self.send), vp(self.probs), vp(self.partial), self._s)),
                     ("dedup_combine", self.lib.moe_dedup_combine, (P, D, vp(self.partial), vp(self.out), self._s)),
@@ -313,11 +321,17 @@ class Step:
                 for r in range(T):
                     Pr, Lr = ctypes.byref(self._ps[r]), ctypes.byref(self._Ls[r])
                     ws = self.layouts[r].workspace
-                    c += [
-                        (f"layout.{r}", self.lib.moe_dispatch_layout,
-                         (Pr, vp(self.idx), vp(self.probs), Lr, vp(ws), ws.numel(), self._s)),
-                        (f"permute.{r}", self.lib.moe_permute, (Pr, Lr, vp(s["hidden"]), vp(self.sends[r]), self._s)),
-                    ]
+                    if unfused:
+                        c += [
+                            (f"layout.{r}", self.lib.moe_dispatch_layout,
+                             (Pr, vp(self.idx), vp(self.probs), Lr, vp(ws), ws.numel(), self._s)),
+                            (f"permute.{r}", self.lib.moe_permute,
+                             (Pr, Lr, vp(s["hidden"]), vp(self.sends[r]), self._s)),
+                        ]
+                    else:  # each peer's layout and send buffer in one call
+                        c += [(f"dispatch.{r}", self.lib.moe_dispatch,
+                               (Pr, vp(self.idx), vp(self.probs), Lr, vp(ws), ws.numel(), vp(s["hidden"]),
+                                vp(self.sends[r]), self._s))]
                 c += [("restore", self.lib.moe_restore_combined,
                        (P, self._L_arr, self._y_arr, vp(self.probs), vp(self.out), self._s))]
             if w.backward:
@@ -370,6 +384,7 @@ class Step:
             for r in range(T):
                 out[f"layout.{r}"] = layout_bytes
                 out[f"permute.{r}"] = read[r] * row + RM * row + NK * 4 + RM
+                out[f"dispatch.{r}"] = layout_bytes + read[r] * row + RM * row
             out["restore"] = sum(kept) * row + N * row + NK * 4 * (T + 1)
         if w.dedup:
             RR = self.dedup.recv_max
@@ -650,9 +665,11 @@ def kernel_table(m, peak):
     return kernels
 
 
-# The surveyed configurations timed beside the headline in the default run (parity cases
-# of the same path; each gets its step time, per-call figures and roofline fractions).
-EXTRA_WORKLOADS = ("tiny", "qwen3", "capacity", "ultraep")
+# Timed beside the headline in the default run: the other surveyed configurations and the
+# workloads of the rows built past them (row alignment, TP folding, the DeepEP-style dedup
+# view, the exchange between 4 ranks on this GPU); each gets its step time, per-call figures
+# and roofline fractions.
+EXTRA_WORKLOADS = ("tiny", "qwen3", "capacity", "ultraep", "ht_align16", "ht_tp2", "ht_dedup", "ht_ep4")
 EXTRA_STEPS, EXTRA_WARMUP = 20, 3
 
 
