@@ -343,8 +343,11 @@ class Step:
             self.calls.append(c)
         self.kernel_names = [name for name, _, _ in self.calls[0]]
 
-    def run(self, i, events=None):
+    def run(self, i, events=None, skip=()):
+        """Enqueue step i (buffer set i mod sets); calls named in `skip` are left out."""
         for n, (name, fn, args) in enumerate(self.calls[i % len(self.calls)]):
+            if name in skip:
+                continue
             if events is not None:
                 events[n][0].record(self.stream)
             rc = fn(*args)
@@ -352,6 +355,12 @@ class Step:
                 raise RuntimeError(f"{name} returned {rc}")
             if events is not None:
                 events[n][1].record(self.stream)
+
+    def clear_status(self) -> None:
+        for L in self.layouts:
+            L.clear_status()
+        if self.w.dedup:
+            self.dedup.tensors["status"].zero_()
 
     def status(self) -> int:
         st = 0
@@ -473,8 +482,9 @@ class EpStep:
             self.calls.append(ph)
         self.kernel_names = [name for phase in self.PHASES for name, _, _ in self.calls[0][phase]]
 
-    def run(self, i, events=None):
-        """Fork to the ranks' streams; join where a phase needs every rank's previous one."""
+    def run(self, i, events=None, skip=()):
+        """Fork to the ranks' streams; join where a phase needs every rank's previous one.
+        Calls named in `skip` are left out (their phase's join events are still recorded)."""
         R = self.w.R
         ph = self.calls[i % len(self.calls)]
         self._start.record(self.stream)
@@ -489,7 +499,7 @@ class EpStep:
             for r, (name, fn, args) in enumerate(ph[phase]):
                 if events is not None:
                     events[n][0].record(self.rank_streams[r])
-                rc = fn(*args)
+                rc = 0 if name in skip else fn(*args)
                 if rc != 0:
                     raise RuntimeError(f"{name} returned {rc}")
                 if events is not None:
@@ -506,6 +516,12 @@ class EpStep:
         for pl in self.plans:
             st |= int(pl.status.item())
         return st
+
+    def clear_status(self) -> None:
+        for G in self.layouts:
+            G.clear_status()
+        for pl in self.plans:
+            pl.status.zero_()
 
     def algorithmic_bytes(self) -> dict:
         """Bytes per call (the mean over the R ranks), each row moved once."""
@@ -566,32 +582,57 @@ def measure(w, host, steps, warmup, eager, hot_l2, ctx):
     torch.cuda.synchronize()
     abytes = step.algorithmic_bytes()
 
-    # one CUDA graph per buffer set, captured from the same C-ABI calls (the launches
-    # keep their programmatic-dependent-launch edges) and replayed in the timed region
+    # The steps captured from the same C-ABI calls into CUDA graphs (the launches keep
+    # their programmatic-dependent-launch edges, also from one step's last kernel to the
+    # next step's first): one graph per buffer set, and one holding the steps of all sets
+    # in order, which the timed region replays whenever a whole round of sets is left.
+    nsets_g = len(step.calls)
     run_step = step.run
     launch_mode = "eager C-ABI calls, programmatic dependent launch"
-    graphs = []
+    graphs, rounds = [], {}
+
+    def capture_round(skip=()):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=work_stream):
+            for i in range(nsets_g):
+                step.run(i, skip=skip)
+        return g
+
     if not eager:
         try:
-            for i in range(len(step.calls)):
+            for i in range(nsets_g):
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g, stream=work_stream):
                     step.run(i)
                 graphs.append(g)
+            rounds[()] = capture_round()
         except Exception as exc:  # a driver without capture support: time the calls themselves
-            graphs = []
+            graphs, rounds = [], {}
             torch.cuda.synchronize()
             launch_mode += f" (graph capture failed: {type(exc).__name__})"
     if graphs:
-        launch_mode = "one CUDA graph per buffer set (captured C-ABI calls, programmatic dependent launch), replayed"
+        launch_mode = (f"CUDA graphs of the captured C-ABI calls (programmatic dependent launch), replayed: one "
+                       f"holding the steps of all {nsets_g} buffer sets in order, one per set for the rest")
 
         def run_step(i, events=None):
             with torch.cuda.stream(work_stream):  # replay where the events are recorded
-                graphs[i % len(graphs)].replay()
+                graphs[i % nsets_g].replay()
 
         for i in range(warmup):
             run_step(i)
         torch.cuda.synchronize()
+
+    def run_steps(first, count):
+        """Steps first .. first+count-1: whole rounds of buffer sets from the round graph."""
+        i = 0
+        while i < count:
+            if rounds and (first + i) % nsets_g == 0 and count - i >= nsets_g:
+                with torch.cuda.stream(work_stream):
+                    rounds[()].replay()
+                i += nsets_g
+            else:
+                run_step(first + i)
+                i += 1
 
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
@@ -599,13 +640,16 @@ def measure(w, host, steps, warmup, eager, hot_l2, ctx):
     torch.cuda.synchronize()
     tr0 = ctx["sampler"].mark()
     t0.record(step.stream)
-    for i in range(steps):
-        run_step(warmup + i)
+    run_steps(warmup, steps)
     t1.record(step.stream)
     torch.cuda.synchronize()
     tr1 = ctx["sampler"].mark()
     barrier()
     elapsed_ms = t0.elapsed_time(t1)
+    status = step.status()
+    if status != 0:
+        raise RuntimeError(f"device status {status:#x} after the timed steps of '{w.name}'")
+    in_step = in_step_costs(step, rounds, capture_round, work_stream, torch) if rounds else {}
     hot_ms = None
     if hot_l2:
         h0 = torch.cuda.Event(enable_timing=True)
@@ -636,11 +680,47 @@ def measure(w, host, steps, warmup, eager, hot_l2, ctx):
     if status != 0:
         raise RuntimeError(f"device status {status:#x} after the timed steps of '{w.name}'")
     elapsed_ms = max_over_ranks(elapsed_ms, device)
-    del graphs
+    del graphs, rounds
     return {
         "step": step, "abytes": abytes, "elapsed_ms": elapsed_ms, "hot_ms": hot_ms, "per_kernel_ms": per_kernel_ms,
+        "in_step_us": in_step,
         "launch_mode": launch_mode, "nsets": nsets, "set_bytes": set_bytes, "timed_window": (tr0, tr1),
     }
+
+
+def in_step_costs(step, rounds, capture_round, stream, torch, target_steps=40, trials=3):
+    """What each call costs inside the replayed steps: the time of a round of all buffer
+    sets' steps, minus the same round captured without that call (the other calls then
+    read what earlier steps left, which stays inside their buffers), per call. Rounds are
+    replayed back to back, alternating between the variants; the median of `trials`.
+    Leaves the device status words cleared (a call left out can make a later one report
+    rows of another layout)."""
+    names = list(dict.fromkeys(step.kernel_names))
+    nsets = len(step.calls)
+    reps = max(2, -(-target_steps // nsets))
+    variants = {(): rounds[()]}
+    for n in names:
+        variants[(n,)] = capture_round(skip=(n,))
+    times = {key: [] for key in variants}
+    for _ in range(trials):
+        for key, g in variants.items():
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                g.replay()  # warm
+                e0.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                e1.record(stream)
+            torch.cuda.synchronize()
+            times[key].append(e0.elapsed_time(e1) * 1e3 / (reps * nsets))  # µs per step
+    med = {key: statistics.median(v) for key, v in times.items()}
+    del variants
+    step.clear_status()
+    torch.cuda.synchronize()
+    out = {"step_us": round(med[()], 2)}
+    for n in names:
+        out[n] = round((med[()] - med[(n,)]) / step.kernel_names.count(n), 2)
+    return out
 
 
 def kernel_table(m, peak):
@@ -662,6 +742,10 @@ def kernel_table(m, peak):
             "gbs": round(gbs, 1),
             "frac": round(gbs / peak, 3),
         }
+        ins = m.get("in_step_us", {}).get(name)
+        if ins is not None and ins > 0:
+            kernels[name]["in_step_us"] = ins
+            kernels[name]["in_step_frac"] = round(m["abytes"][name] / (ins * 1e-6) / 1e9 / peak, 3)
     return kernels
 
 
@@ -799,6 +883,8 @@ def run_ours(args, ws, rank, local):
         },
         "gpu_launches": args.steps * sum(kernels_per_call(n) for n in m["step"].kernel_names),
         "kernel_timing": "per-kernel CUDA events in a second pass of the same K steps (launched eagerly)",
+        "in_step_timing": ("in_step_us: a round of replayed steps minus the same round captured without the call, "
+                           "per call (CUDA events, median of 3); in_step_frac from it"),
         "launch": m["launch_mode"],
         "hot_l2": {
             "ms_per_step": round(hot_ms / args.steps, 4),
