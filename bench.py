@@ -4,16 +4,22 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ht] [--impl ours|reference]
 
 A step is one pass of the whole hot path over one batch of synthetic input:
-router top-k -> dispatch (the layout and the permute, fused: moe_dispatch) ->
-(identity experts) -> combine,
-plus combine-backward and permute-backward for workloads that train
+router top-k -> dispatch (the layout and the permute) -> (identity experts) ->
+combine, plus combine-backward and permute-backward for workloads that train
 (``ultraep``). Inputs are resident in HBM when the timed region starts and
 rotate over several buffer sets whose total size exceeds the 126 MB L2, so no
-step reads inputs that a previous step left in L2. Each set's step is captured once
-into a CUDA graph (the same C-ABI calls) and replayed in the timed region
-(``--eager``: the calls themselves); per-call times come from a second, eager pass
-with CUDA events around every call.
+step reads inputs that a previous step left in L2.
 
+Headline schedule (``--schedule pipelined``, the default where the step is route,
+layout, permute and combine on one rank): two batches in flight
+(combine_moe_route_tokens_b200.Pipeline) — batch i's route and layout run on a side
+stream beside batch i-1's combine, the permutes and combines stay in batch order —
+the K batches captured as one CUDA graph and replayed once. Beside it (``serial``):
+the same K batches one at a time through the fused dispatch call (moe_dispatch), each
+round of buffer sets captured as one CUDA graph of the same C-ABI calls and replayed
+(``--schedule serial`` makes that the headline; ``--eager``: the calls themselves).
+Per-call times come from an eager pass with CUDA events around every call, and from
+the step's own replays (a round minus the round without the call).
 N > 1 (torchrun, one process per GPU): each rank processes its own batch
 (data-parallel, independent seeds, no collective on the data path); timing is
 the max over ranks; ``value`` counts the tokens of all ranks.
@@ -688,6 +694,67 @@ def measure(w, host, steps, warmup, eager, hot_l2, ctx):
     }
 
 
+def pipelined_eligible(w) -> bool:
+    """Workloads whose step is route -> layout -> permute -> combine on one rank."""
+    return w.tp_size <= 1 and not w.dedup and not w.ep and not w.backward
+
+
+def measure_pipelined(w, host, steps, warmup, ctx):
+    """The same steps with two batches in flight (combine_moe_route_tokens_b200.Pipeline):
+    batch i's route and layout run on a side stream beside batch i-1's combine; the
+    permutes and combines stay in batch order on the launching stream. Warm-up: `warmup`
+    batches enqueued from the host, then one untimed replay of the timed graph (its
+    upload); timed: the K batches captured as one CUDA graph, replayed once between two
+    CUDA events on the launching stream, barrier and synchronize on both sides."""
+    torch, moe, device, barrier = ctx["torch"], ctx["moe"], ctx["device"], ctx["barrier"]
+    sets, nsets, set_bytes = device_sets(w, host, torch, device)
+    p = moe.Problem(N=w.N, H=w.H, k=w.k, E_log=w.E_log, R=w.R, capacity=w.capacity,
+                    num_replicas=w.num_replicas, row_align=w.row_align)
+    work = torch.cuda.Stream(device)
+    pipe = moe.Pipeline(p, device=device, stream=work)
+
+    def enqueue(first, count):
+        ready = torch.cuda.Event()  # the inputs are resident before the first batch
+        ready.record(work)
+        for i in range(first, first + count):
+            s = sets[i % nsets]
+            pipe.submit(s["logits"], s["hidden"], ready=ready)
+        pipe.join()
+
+    with torch.cuda.stream(work):
+        enqueue(0, warmup)
+    torch.cuda.synchronize()
+    pipe.reset()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=work):
+        enqueue(warmup, steps)
+    with torch.cuda.stream(work):
+        g.replay()
+    torch.cuda.synchronize()
+    status = pipe.status()
+    if status != 0:
+        raise RuntimeError(f"device status {status:#x} after the pipelined warm-up of '{w.name}'")
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    tr0 = ctx["sampler"].mark()
+    t0.record(work)
+    with torch.cuda.stream(work):
+        g.replay()
+    t1.record(work)
+    torch.cuda.synchronize()
+    tr1 = ctx["sampler"].mark()
+    barrier()
+    status = pipe.status()
+    if status != 0:
+        raise RuntimeError(f"device status {status:#x} after the pipelined steps of '{w.name}'")
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), device)
+    del g, pipe, sets
+    torch.cuda.synchronize()
+    return {"elapsed_ms": elapsed_ms, "timed_window": (tr0, tr1), "nsets": nsets, "set_bytes": set_bytes}
+
+
 def in_step_costs(step, rounds, capture_round, stream, torch, target_steps=40, trials=3):
     """What each call costs inside the replayed steps: the time of a round of all buffer
     sets' steps, minus the same round captured without that call (the other calls then
@@ -787,9 +854,22 @@ def run_ours(args, ws, rank, local):
     sampler = ClockSampler(local)
     ctx = {"torch": torch, "moe": moe, "native": _native, "device": device, "barrier": barrier, "sampler": sampler,
            "unfused": args.unfused, "bulk_copy": args.bulk_copy}
+    # The headline schedule: two batches in flight (the layout as its own call on a side
+    # stream, so the per-call figures are those of route, layout, permute and combine), with
+    # the one-batch-at-a-time step of the fused dispatch beside it; or that serial step.
+    pipelined = (args.schedule == "pipelined" and pipelined_eligible(w) and not args.eager and not args.bulk_copy
+                 and not args.unfused)
+    mp = m_serial = None
     with sampler:
-        m = measure(w, host, args.steps, args.warmup, args.eager, True, ctx)
+        if pipelined:
+            m = measure(w, host, args.steps, args.warmup, args.eager, True, {**ctx, "unfused": True})
+            m_serial = measure(w, host, args.steps, args.warmup, args.eager, False, ctx)
+            mp = measure_pipelined(w, host, args.steps, args.warmup, ctx)
+        else:
+            m = measure(w, host, args.steps, args.warmup, args.eager, True, ctx)
     step, abytes, elapsed_ms, hot_ms = m["step"], m["abytes"], m["elapsed_ms"], m["hot_ms"]
+    if mp is not None:
+        elapsed_ms = mp["elapsed_ms"]
 
     # end to end through the public API: every step copies its inputs in from pinned host
     # memory and its combined output back out. E2E_DEPTH sets of device buffers rotate, so
@@ -864,9 +944,14 @@ def run_ours(args, ws, rank, local):
                 for n in m["step"].kernel_names)),
             "l2": f"inputs rotated over {m['nsets']} buffer sets ({m['nsets'] * m['set_bytes'] / 2**20:.0f} MiB "
                   f"> 126 MB L2), no flush",
-            "dispatch": ("moe_dispatch_layout + moe_permute (separate calls)" if args.unfused else
+            "dispatch": ("moe_dispatch_layout on a side stream, then moe_permute (two batches in flight)"
+                         if mp is not None else
+                         "moe_dispatch_layout + moe_permute (separate calls)" if args.unfused else
                          "moe_dispatch (layout + permute fused), rows copied with "
                          + ("bulk (TMA) copies through shared memory" if args.bulk_copy else "16-byte vector copies")),
+            "schedule": ("two batches in flight (combine_moe_route_tokens_b200.Pipeline): batch i's route and "
+                         "layout on a side stream beside batch i-1's combine; permutes and combines in batch order"
+                         if mp is not None else "one batch at a time"),
         },
         "effective_gbs": round(path_bytes / (ms_step * 1e-3) / 1e9, 1),
         "effective_hbm_frac": round(path_bytes / (ms_step * 1e-3) / 1e9 / peak, 3),
@@ -880,20 +965,35 @@ def run_ours(args, ws, rank, local):
             "unit": "GB/s",
             "frac": round(ach / peak, 3),
             "traffic": stored_traffic(dominant, w.name),
+            **({"in_step_achieved": round(m["abytes"][dominant] / (kernels[dominant]["in_step_us"] * 1e-6) / 1e9, 1),
+                "in_step_frac": kernels[dominant]["in_step_frac"]} if "in_step_us" in kernels[dominant] else {}),
         },
         "gpu_launches": args.steps * sum(kernels_per_call(n) for n in m["step"].kernel_names),
         "kernel_timing": "per-kernel CUDA events in a second pass of the same K steps (launched eagerly)",
         "in_step_timing": ("in_step_us: a round of replayed steps minus the same round captured without the call, "
                            "per call (CUDA events, median of 3); in_step_frac from it"),
-        "launch": m["launch_mode"],
+        "launch": ("the K batches captured as one CUDA graph of the binding's calls on two lanes of buffers "
+                   "(programmatic dependent launch within each stream), replayed once" if mp is not None
+                   else m["launch_mode"]),
         "hot_l2": {
             "ms_per_step": round(hot_ms / args.steps, 4),
             "value": round(w.N * args.steps * ws / (hot_ms / 1e3), 1),
-            "note": "the same K steps on one input set (inputs resident in L2); not the headline",
+            "note": "the same K steps, one batch at a time, on one input set (inputs resident in L2); not the headline",
         },
-        "clocks": sampler.summary(m["timed_window"]),
+        "clocks": sampler.summary(mp["timed_window"] if mp is not None else m["timed_window"]),
         "e2e": e2e,
     }
+    if m_serial is not None:  # the same batches one at a time through the fused dispatch call
+        ms_ser = m_serial["elapsed_ms"] / args.steps
+        result["serial"] = {
+            "ms_per_step": round(ms_ser, 4),
+            "value": round(w.N * args.steps * ws / (m_serial["elapsed_ms"] / 1e3), 1),
+            "step": "+".join(dict.fromkeys(m_serial["step"].kernel_names)),
+            "dispatch": "moe_dispatch (layout + permute fused)",
+            "note": "one batch at a time, the step's latency; the headline overlaps two batches",
+            "in_step_us": m_serial.get("in_step_us", {}),
+        }
+        result["serial_unfused_ms_per_step"] = round(m["elapsed_ms"] / args.steps, 4)
     if workloads:
         result["workloads"] = workloads
     if not args.no_cpu_baseline and ws == 1:
@@ -1190,6 +1290,9 @@ def main():
     ap.add_argument("--no-extra", action="store_true",
                     help="time only the headline workload (skip the other surveyed configurations)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--schedule", default="pipelined", choices=["pipelined", "serial"],
+                    help="headline schedule: two batches in flight (default, for workloads whose step is route, "
+                         "layout, permute, combine on one rank) or one batch at a time")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--tokens", type=int, default=0, help="run the workload with this many tokens (profiling)")
     ap.add_argument("--eager", action="store_true",

@@ -13,6 +13,7 @@ functions keep the C names:
     moe_dedup_*           DeepEP-style view: one receive row per (token, rank), two-level combine
     moe_ep_*              expert-parallel exchange: dispatch into / combine from the ranks' receive buffers
     EpGroup               that exchange between processes (CUDA IPC mappings, offsets all-gather, fences)
+    Pipeline              two batches in flight: one's route and layout beside the other's combine
     moe_permute_backward  grad_hidden[t] = bf16(sum_j grad_send[dest_row[t, j]])
     moe_combine_backward  grad_y[row] = bf16(p * grad_out[t]); grad_probs[t, j] = <grad_out[t], y[row]>
 
@@ -66,6 +67,7 @@ __all__ = [
     "DedupView",
     "EpPlan",
     "EpGroup",
+    "Pipeline",
     "peer_table",
     "moe_ep_recv_rows_max",
     "moe_ep_plan",
@@ -708,3 +710,4 @@ def moe_combine_backward(problem: Problem, layout: Layout, grad_out: torch.Tenso
 
 
 from .ep_group import EpGroup  # noqa: E402  (the exchange between processes; host plumbing only)
+from .pipeline import Pipeline  # noqa: E402  (two batches in flight; host scheduling only)
