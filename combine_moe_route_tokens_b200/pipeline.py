@@ -86,6 +86,7 @@ class Pipeline:
         moe_route_topk(logits, p.k, token_mask=token_mask, topk_idx=lane.idx, topk_probs=lane.probs, stream=side)
         moe_dispatch_layout(p, lane.idx, lane.probs, layout=lane.layout, stream=side)
         lane.laid_out.record(side)
+        self.main.wait_event(ready)  # the permute reads `hidden` (a no-op if `ready` is on this stream)
         self.main.wait_event(lane.laid_out)
         moe_permute(p, lane.layout, hidden, send=lane.send, stream=self.main)
         y = lane.send if self.experts is None else self.experts(lane.send, lane)
