@@ -886,7 +886,10 @@ def run_ours(args, ws, rank, local):
         with sampler:
             for name in EXTRA_WORKLOADS:
                 wx = get_workload(name)
-                mx = measure(wx, rank_inputs(wx, rank), EXTRA_STEPS, EXTRA_WARMUP, args.eager, False, ctx)
+                hx = rank_inputs(wx, rank)
+                mx = measure(wx, hx, EXTRA_STEPS, EXTRA_WARMUP, args.eager, False, ctx)
+                if pipelined_eligible(wx) and not args.eager and not args.bulk_copy and not args.unfused:
+                    mx["pipelined"] = measure_pipelined(wx, hx, EXTRA_STEPS, EXTRA_WARMUP, ctx)
                 extra[name] = mx
                 torch.cuda.empty_cache()
 
@@ -921,7 +924,15 @@ def run_ours(args, ws, rank, local):
             "kernels": kx,
             "l2": f"inputs rotated over {mx['nsets']} buffer sets ({mx['nsets'] * mx['set_bytes'] / 2**20:.0f} MiB)",
             "launch": mx["launch_mode"],
+            "schedule": "one batch at a time",
         }
+        if "pipelined" in mx:  # the same calls split (layout, then permute), two batches in flight
+            pm = mx["pipelined"]["elapsed_ms"]
+            workloads[name]["pipelined"] = {
+                "ms_per_step": round(pm / EXTRA_STEPS, 4),
+                "tokens_per_s": round(wx.N * EXTRA_STEPS * ws / (pm / 1e3), 1),
+                "schedule": "two batches in flight (Pipeline): route and layout beside the previous combine",
+            }
     result = {
         "metric": METRIC,
         "value": round(w.N * args.steps * ws / (elapsed_ms / 1e3), 1),

@@ -605,6 +605,7 @@ int moe_permute(const moe_problem_t *problem, const moe_layout_t *layout, const 
     a.V = problem->H / 8;
     a.group = a.V <= 32 * PERMUTE_CHUNKS ? 32 : (a.V <= 64 * PERMUTE_CHUNKS ? 64 : PERMUTE_THREADS);
     a.pieces = (a.V + a.group * PERMUTE_CHUNKS - 1) / (a.group * PERMUTE_CHUNKS);
+    a.load_first = problem->capacity == 0 ? 1 : 0;
     // pad-row workers: one warp checks 32 rows per pass, at most four CTAs per SM
     const int64_t zb = (d.rows_max + PERMUTE_THREADS - 1) / PERMUTE_THREADS;
     a.zero_blocks = static_cast<int32_t>(zb < 4 * dev.sms ? zb : 4 * dev.sms);
@@ -892,6 +893,7 @@ int moe_dedup_dispatch(const moe_problem_t *problem, const moe_dedup_t *dedup, c
     a.V = problem->H / 8;
     a.group = a.V <= 32 * PERMUTE_CHUNKS ? 32 : (a.V <= 64 * PERMUTE_CHUNKS ? 64 : PERMUTE_THREADS);
     a.pieces = (a.V + a.group * PERMUTE_CHUNKS - 1) / (a.group * PERMUTE_CHUNKS);
+    a.load_first = problem->capacity == 0 ? 1 : 0;
     const int64_t zb = (recv_max + PERMUTE_THREADS - 1) / PERMUTE_THREADS;
     a.zero_blocks = static_cast<int32_t>(zb < 4 * dev.sms ? zb : 4 * dev.sms);
     const int64_t groups = PERMUTE_THREADS / a.group;
@@ -1105,6 +1107,7 @@ int moe_ep_dispatch(const moe_problem_t *problem, const moe_layout_t *layout, co
     a.V = problem->H / 8;
     a.group = a.V <= 32 * PERMUTE_CHUNKS ? 32 : (a.V <= 64 * PERMUTE_CHUNKS ? 64 : PERMUTE_THREADS);
     a.pieces = (a.V + a.group * PERMUTE_CHUNKS - 1) / (a.group * PERMUTE_CHUNKS);
+    a.load_first = problem->capacity == 0 ? 1 : 0;
     a.ep_peers = reinterpret_cast<uint4 *const *>(peer_recv);
     a.phys_idx = layout->phys_idx;
     a.ep_base = base;

@@ -45,6 +45,8 @@ struct PermuteArgs {
     int32_t group;       // threads per token piece: 32, 64 or 128
     int32_t pieces;      // pieces per token
     int32_t zero_blocks; // leading CTAs that zero pad rows
+    int32_t load_first = 0; // 1: every token keeps a slot (no capacity), so its row is loaded
+                            // together with its destinations rather than after them
     // expert-parallel exchange: slot j's row d of expert q goes to the receive
     // buffer of q's owner, row ep_base[q] + d - ep_offsets[q]; the leading CTAs
     // zero this source's padding rows there (rows tokens[q] .. of each expert)
@@ -130,6 +132,17 @@ __global__ void __launch_bounds__(PERMUTE_THREADS) permute_kernel(PermuteArgs a)
     const bool active = unit < units;
     const int64_t t = active ? unit / a.pieces : 0;
     const int piece = static_cast<int>(unit - t * a.pieces);
+    const int32_t c0 = piece * (a.group * PERMUTE_CHUNKS) + gt;
+    const uint4 *src = a.hidden + t * a.V;
+    uint4 v[PERMUTE_CHUNKS];
+    if (active && a.load_first) { // both round trips in flight at once
+#pragma unroll
+        for (int c = 0; c < PERMUTE_CHUNKS; ++c) {
+            const int32_t idx = c0 + c * a.group;
+            if (idx < a.V)
+                v[c] = ld_stream_u4(src + idx);
+        }
+    }
     if (active && gt < a.k) {
         int32_t d = __ldg(a.dest_row + t * a.k + gt);
         if (d < -1 || d >= a.rows_max) {
@@ -165,14 +178,13 @@ __global__ void __launch_bounds__(PERMUTE_THREADS) permute_kernel(PermuteArgs a)
     }
     if (!any)
         return;
-    const int32_t c0 = piece * (a.group * PERMUTE_CHUNKS) + gt;
-    const uint4 *src = a.hidden + t * a.V;
-    uint4 v[PERMUTE_CHUNKS];
+    if (!a.load_first) {
 #pragma unroll
-    for (int c = 0; c < PERMUTE_CHUNKS; ++c) {
-        const int32_t idx = c0 + c * a.group;
-        if (idx < a.V)
-            v[c] = ld_stream_u4(src + idx);
+        for (int c = 0; c < PERMUTE_CHUNKS; ++c) {
+            const int32_t idx = c0 + c * a.group;
+            if (idx < a.V)
+                v[c] = ld_stream_u4(src + idx);
+        }
     }
     for (int j = 0; j < a.k; ++j) {
         uint4 *dst;
