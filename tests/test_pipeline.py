@@ -12,9 +12,11 @@ import pytest
 import torch
 
 CASES = [
-    # N, H, k, E, R, capacity
-    (512, 1024, 8, 64, 4, 0),
-    (300, 256, 2, 16, 2, 40),  # capacity: drops and pad rows
+    # N, H, k, E, R, capacity, replicas, row alignment
+    (512, 1024, 8, 64, 4, 0, 0, 0),
+    (300, 256, 2, 16, 2, 40, 0, 0),  # capacity: drops and pad rows
+    (513, 512, 8, 32, 4, 0, 4, 0),  # hot-expert replicas (reroute)
+    (257, 768, 4, 16, 2, 0, 0, 8),  # rows aligned to 8 per expert
 ]
 
 
@@ -23,15 +25,15 @@ def _bits(t):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("case", CASES, ids=[f"N{c[0]}_H{c[1]}_k{c[2]}_E{c[3]}_C{c[5]}" for c in CASES])
+@pytest.mark.parametrize("case", CASES, ids=[f"N{c[0]}_H{c[1]}_k{c[2]}_E{c[3]}_C{c[5]}_rep{c[6]}_A{c[7]}" for c in CASES])
 def test_pipeline_matches_one_batch_at_a_time(case):
     from gpu_util import require_cuda
 
     require_cuda()
     import combine_moe_route_tokens_b200 as moe
 
-    N, H, k, E, R, C = case
-    p = moe.Problem(N=N, H=H, k=k, E_log=E, R=R, capacity=C)
+    N, H, k, E, R, C, reps, A = case
+    p = moe.Problem(N=N, H=H, k=k, E_log=E, R=R, capacity=C, num_replicas=reps, row_align=A)
     g = torch.Generator(device="cuda").manual_seed(1234 + N)
     B = 6
     logits = [torch.randn(N, E, device="cuda", generator=g) for _ in range(B)]
