@@ -4,8 +4,9 @@ Each batch's output under the pipelined schedule (route and layout on a side str
 beside the previous batch's combine, permutes and combines in batch order on the main
 stream, two lanes of buffers) must equal, bit for bit, the output of the same batch
 through moe_route_topk -> moe_dispatch -> moe_combine on one stream, which the parity
-tests compare with the oracle. Six batches, so that both lanes come round several
-times, enqueued eagerly and replayed from a CUDA graph.
+tests compare with the oracle at every workload's full size. Six batches, so that both
+lanes come round several times, enqueued eagerly and replayed from a CUDA graph; small
+problems with each layout option, and the headline's batch.
 """
 
 import pytest
@@ -17,6 +18,7 @@ CASES = [
     (300, 256, 2, 16, 2, 40, 0, 0),  # capacity: drops and pad rows
     (513, 512, 8, 32, 4, 0, 4, 0),  # hot-expert replicas (reroute)
     (257, 768, 4, 16, 2, 0, 0, 8),  # rows aligned to 8 per expert
+    (4096, 7168, 8, 256, 4, 0, 0, 0),  # the headline's batch (4096 x 7168, e256, top-8, 4 ranks)
 ]
 
 
