@@ -7,18 +7,18 @@
 // Read once, write k times. A group of 32, 64 or 128 threads (the smallest
 // that covers the row with PERMUTE_CHUNKS 16-byte chunks per thread; longer
 // rows are cut into pieces of 128 x PERMUTE_CHUNKS chunks) copies one token:
-// it reads the token's destination rows, skips the token if every slot was
-// dropped, loads its chunks with streaming (L1 no-allocate) loads, all in
-// flight together, then stores them to each kept destination row; a warp
-// writes 512 contiguous bytes per store instruction. A CTA holds 128 / group
+// it reads the token's destination rows and its chunks with streaming (L1
+// no-allocate) loads, all in flight together (with a capacity, where most
+// tokens may keep no slot, the chunks only after the destinations show that
+// one is kept), then stores them to each kept destination row; a warp writes
+// 512 contiguous bytes per store instruction. A CTA holds 128 / group
 // tokens. The leading CTAs zero the pad rows (pad_mask = 1) while the copy
 // CTAs stream. Every needed byte of hidden is read once and every byte of
 // send written once.
 //
-// A variant that stages each row through shared memory with TMA bulk copies
-// (cp.async.bulk global->shared, mbarrier completion, k bulk shared->global
-// stores) was measured on B200 at 96-98 us for the 4096 x 7168 / top-8 shape
-// against 92 us for this one, so the plain vector path is the one built.
+// Staging each row through shared memory with bulk (TMA) copies is the fused
+// dispatch's opt-in path (dispatch_bulk_kernel); in the replayed steps it is
+// slower than this vector copy on every workload measured.
 #pragma once
 
 #include <cstdint>
