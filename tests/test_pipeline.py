@@ -83,3 +83,46 @@ def test_pipeline_matches_one_batch_at_a_time(case):
         assert gp.status() == 0
         for b in range(B):
             assert torch.equal(_bits(got[b]), _bits(ref[b])), f"graph batch {b}"
+
+
+WORKLOADS = ["tiny", "ht", "qwen3", "capacity", "ultraep"]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_pipeline_at_full_size(name):
+    """The forward path of each surveyed configuration at its full size with the benchmark's
+    input recipe (four batches: seed offsets 0-3), two batches in flight against each batch
+    alone; the batches alone are the calls the parity tests compare with the oracle."""
+    from gpu_util import require_cuda
+
+    require_cuda()
+    import numpy as np
+
+    import combine_moe_route_tokens_b200 as moe
+    from synthetic import get_workload, make_inputs
+
+    w = get_workload(name)
+    p = moe.Problem(N=w.N, H=w.H, k=w.k, E_log=w.E_log, R=w.R, capacity=w.capacity,
+                    num_replicas=w.num_replicas, row_align=w.row_align)
+    B = 4
+    logits, hidden = [], []
+    for b in range(B):
+        d = make_inputs(w, grad=False, seed_offset=b)
+        logits.append(torch.from_numpy(d["logits"]).cuda())
+        hidden.append(torch.from_numpy(d["hidden"].view(np.int16)).cuda().view(torch.bfloat16))
+    ref = []
+    for b in range(B):
+        idx, probs = moe.moe_route_topk(logits[b], w.k)
+        L, send = moe.moe_dispatch(p, idx, probs, hidden[b])
+        ref.append(moe.moe_combine(p, L, send, probs))
+        assert L.status() == 0
+    pipe = moe.Pipeline(p)
+    ready = torch.cuda.Event()
+    ready.record()
+    outs = [pipe.submit(logits[b], hidden[b], ready=ready).clone() for b in range(B)]
+    pipe.join()
+    torch.cuda.synchronize()
+    assert pipe.status() == 0
+    for b in range(B):
+        assert torch.equal(_bits(outs[b]), _bits(ref[b])), f"{name} batch {b}"
