@@ -1273,6 +1273,10 @@ def run_calibration(args) -> dict:
     half = a[: nbytes // 4]
     copy_ms = timed(lambda: b.copy_(half))  # device-to-device copy: 235 MB read + 235 MB written
     fill_ms = timed(lambda: a.zero_())  # 470 MB written by torch's fill kernel
+    # the capacity workload's send buffer (40,960 rows of 4 KB): a short write-only stream
+    cap_bytes = 40960 * 4096
+    cap = a[: cap_bytes // 2]
+    fill_cap_ms = timed(lambda: cap.zero_())
     # host links at the end-to-end step's sizes (ht: 62.9 MB in, 58.7 MB out), pinned host memory
     h_in = torch.empty(62914560 // 2, dtype=torch.int16).pin_memory()
     h_out = torch.empty(58720256 // 2, dtype=torch.int16).pin_memory()
@@ -1299,6 +1303,8 @@ def run_calibration(args) -> dict:
         "copy_d2d_gbs": round(nbytes / (copy_ms * 1e-3) / 1e9, 1),
         "torch_zero_gbs": round(nbytes / (fill_ms * 1e-3) / 1e9, 1),
         "bytes": nbytes,
+        "torch_zero_capacity_send_gbs": round(cap_bytes / (fill_cap_ms * 1e-3) / 1e9, 1),
+        "capacity_send_bytes": cap_bytes,
         "h2d_gbs": round(h_in.numel() * 2 / (h2d_ms * 1e-3) / 1e9, 1),
         "d2h_gbs": round(h_out.numel() * 2 / (d2h_ms * 1e-3) / 1e9, 1),
         "h2d_d2h_together_ms": round(both_ms, 3),
