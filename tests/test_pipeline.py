@@ -32,7 +32,10 @@ def test_pipeline_matches_one_batch_at_a_time(case):
     from gpu_util import require_cuda
 
     require_cuda()
+    import numpy as np
+
     import combine_moe_route_tokens_b200 as moe
+    import oracle
 
     N, H, k, E, R, C, reps, A = case
     p = moe.Problem(N=N, H=H, k=k, E_log=E, R=R, capacity=C, num_replicas=reps, row_align=A)
@@ -47,6 +50,12 @@ def test_pipeline_matches_one_batch_at_a_time(case):
         L, send = moe.moe_dispatch(p, idx, probs, hidden[b])
         ref.append(moe.moe_combine(p, L, send, probs))
         assert L.status() == 0
+        # and the oracle's combine of the same routing (ids and probs from the router above)
+        ids_h, probs_h = idx.cpu().numpy(), probs.cpu().numpy()
+        h = hidden[b].cpu().view(torch.int16).numpy().view(np.uint16)
+        OL = oracle.layout(ids_h, probs_h, E_log=E, R=R, C=C, num_replicas=reps, align=A)
+        exp = oracle.combine(oracle.permute(h, OL["dest_row"], OL["rows_max"]), OL["dest_row"], probs_h)
+        assert np.array_equal(ref[b].cpu().view(torch.int16).numpy().view(np.uint16), exp), f"oracle batch {b}"
     torch.cuda.synchronize()
 
     # eager
