@@ -135,3 +135,45 @@ def test_pipeline_at_full_size(name):
     assert pipe.status() == 0
     for b in range(B):
         assert torch.equal(_bits(outs[b]), _bits(ref[b])), f"{name} batch {b}"
+
+
+@pytest.mark.gpu
+def test_pipeline_token_mask_and_empty_batches():
+    """Padding tokens masked out of routing (Megatron MORI page: router.py) go through the
+    pipeline like one batch at a time; an empty batch enqueues nothing and breaks nothing."""
+    from gpu_util import require_cuda
+
+    require_cuda()
+    import combine_moe_route_tokens_b200 as moe
+
+    N, H, k, E, R = 300, 512, 4, 32, 4
+    p = moe.Problem(N=N, H=H, k=k, E_log=E, R=R)
+    g = torch.Generator(device="cuda").manual_seed(99)
+    B = 4
+    logits = [torch.randn(N, E, device="cuda", generator=g) for _ in range(B)]
+    hidden = [torch.randn(N, H, device="cuda", generator=g).to(torch.bfloat16) for _ in range(B)]
+    masks = [(torch.rand(N, device="cuda", generator=g) < 0.3).to(torch.uint8) for _ in range(B)]
+    ref = []
+    for b in range(B):
+        idx, probs = moe.moe_route_topk(logits[b], k, token_mask=masks[b])
+        L, send = moe.moe_dispatch(p, idx, probs, hidden[b])
+        ref.append(moe.moe_combine(p, L, send, probs))
+    pipe = moe.Pipeline(p)
+    ready = torch.cuda.Event()
+    ready.record()
+    outs = [pipe.submit(logits[b], hidden[b], token_mask=masks[b], ready=ready).clone() for b in range(B)]
+    pipe.join()
+    torch.cuda.synchronize()
+    assert pipe.status() == 0
+    for b in range(B):
+        assert torch.equal(_bits(outs[b]), _bits(ref[b])), f"masked batch {b}"
+        assert torch.all(_bits(outs[b])[masks[b].bool()] == 0)  # a masked token keeps no slot: zero row
+
+    p0 = moe.Problem(N=0, H=H, k=k, E_log=E, R=R)
+    pipe0 = moe.Pipeline(p0)
+    for _ in range(3):
+        out = pipe0.submit(torch.empty((0, E), device="cuda"), torch.empty((0, H), dtype=torch.bfloat16, device="cuda"))
+        assert out.shape == (0, H)
+    pipe0.join()
+    torch.cuda.synchronize()
+    assert pipe0.status() == 0
