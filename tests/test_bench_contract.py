@@ -66,3 +66,33 @@ def test_traffic_digest_ignores_comments_and_layout_only():
     assert bench._code_only(code) == bench._code_only(same)
     assert bench._code_only(code) != bench._code_only(other)
     assert bench.stored_traffic("permute", "no_such_workload") is None
+
+
+def test_clock_window_tail():
+    """The clock record's window: the timed region plus untimed repetitions up to ~30 ms."""
+    import bench
+
+    assert bench.clock_tail_reps(3.3) == 9  # 3.3 ms timed + 9 x 3.3 ms = 33 ms
+    assert bench.clock_tail_reps(bench.CLOCK_WINDOW_MS) == 0
+    assert bench.clock_tail_reps(100.0) == 0
+    assert bench.clock_tail_reps(0.0) > 0
+
+
+def test_pipelined_schedule_applies_to_plain_forward_steps():
+    """Two batches in flight only where a step is route -> layout -> permute -> combine on
+    one rank (no backward, TP folding, dedup view or exchange)."""
+    import bench
+    from synthetic import get_workload
+
+    eligible = {name for name in ["tiny", "ht", "qwen3", "capacity", "ultraep"] + list(bench.EXTRA_WORKLOADS)
+                if bench.pipelined_eligible(get_workload(name))}
+    assert eligible == {"tiny", "ht", "qwen3", "capacity", "ht_align16"}
+
+
+def test_kernels_per_call():
+    import bench
+
+    assert bench.kernels_per_call("layout") == 2 and bench.kernels_per_call("layout.1") == 2
+    assert bench.kernels_per_call("dispatch") == 2 and bench.kernels_per_call("permute") == 1
+    # the pipelined headline's step: route, layout (count + fill), permute, combine
+    assert sum(bench.kernels_per_call(n) for n in ("route", "layout", "permute", "combine")) == 5
