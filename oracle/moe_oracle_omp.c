@@ -1,7 +1,7 @@
 /*
  * moe_oracle_omp.c — the oracle's token-independent steps on every host core.
  *
- * TEST INFRASTRUCTURE / BASELINE ONLY: the benchmark times it as the all-cores
+ * TEST INFRASTRUCTURE ONLY (and a timed CPU reference): the benchmark times it as the all-cores
  * CPU baseline beside the single-threaded oracle; the tests check it against
  * that oracle. It is built into a library of its own (libmoe_oracle_omp.so,
  * gcc -fopenmp) from this file and moe_oracle.c; the single-threaded library
