@@ -909,6 +909,10 @@ def run_ours(args, ws, rank, local):
                 wx = get_workload(name)
                 hx = rank_inputs(wx, rank)
                 mx = measure(wx, hx, EXTRA_STEPS, EXTRA_WARMUP, args.eager, False, ctx)
+                if wx.tp_size <= 1 and not wx.dedup and not wx.ep and not args.unfused and not args.bulk_copy:
+                    # the same step with the layout and the permute as separate calls (the permute's own figures)
+                    mx["separate"] = measure(wx, hx, EXTRA_STEPS, EXTRA_WARMUP, args.eager, False,
+                                             {**ctx, "unfused": True})
                 if pipelined_eligible(wx) and not args.eager and not args.bulk_copy and not args.unfused:
                     mx["pipelined"] = measure_pipelined(wx, hx, EXTRA_STEPS, EXTRA_WARMUP, ctx)
                 extra[name] = mx
@@ -947,6 +951,13 @@ def run_ours(args, ws, rank, local):
             "launch": mx["launch_mode"],
             "schedule": "one batch at a time",
         }
+        if "separate" in mx:
+            ms_sep = mx["separate"]
+            workloads[name]["separate_calls"] = {
+                "ms_per_step": round(ms_sep["elapsed_ms"] / EXTRA_STEPS, 4),
+                "kernels": kernel_table(ms_sep, peak),
+                "note": "one batch at a time, moe_dispatch_layout then moe_permute",
+            }
         if "pipelined" in mx:  # the same calls split (layout, then permute), two batches in flight
             pm = mx["pipelined"]["elapsed_ms"]
             workloads[name]["pipelined"] = {
